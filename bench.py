@@ -1,0 +1,507 @@
+"""Benchmark of the fused group-wise dequant matmul on B200.
+
+Default workload (the headline): pre-packed int4 decode GEMV, M = 1, over the
+24-layer Qwen2.5-0.5B linear-layer set (q/k/v/o/gate/up/down, hidden 896),
+fp16 scale/zero per 64-block, fp32 x.  One step = one grouped launch over
+all 168 matrices of the set.  The metric is HBM GB/s of algorithmic bytes
+(packed codes + scales/zeros + x + y), plus the fraction of the measured
+HBM copy peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+Under torchrun (N > 1) every rank runs its own replica of the workload
+("weak" scaling: the path needs no exchange); rank 0 prints one JSON line.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the
+same workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "fused dequant-matmul: HBM GB/s (M=1 GEMV), TFLOP/s (M≥128), % roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+WORKLOADS = {
+    # name: (shape set, layers, mode, bits, group, M, workload seed)
+    "qwen2.5-0.5b-int4-decode": ("qwen2.5-0.5b", 24, "packed", 4, 64, 1, 1),
+    "qwen3-0.6b-rtn3-decode": ("qwen3-0.6b", 28, "runtime", 3, 64, 1, 2),
+    "qwen3-0.6b-rtn3-channel-decode": ("qwen3-0.6b", 28, "runtime", 3, 0, 1, 2),
+    "qwen3-0.6b-fp16-decode": ("qwen3-0.6b", 28, "runtime", 16, 64, 1, 2),
+    "qwen3-8b-int4-decode": ("qwen3-8b", 36, "packed", 4, 64, 1, 4),
+    "qwen3-8b-int4-decode-m16": ("qwen3-8b", 36, "packed", 4, 64, 16, 4),
+    "qwen3-8b-rtn3-decode": ("qwen3-8b", 36, "runtime", 3, 64, 1, 4),
+    "qwen3-8b-rtn3-decode-m16": ("qwen3-8b", 36, "runtime", 3, 64, 16, 4),
+}
+DEFAULT_WORKLOAD = "qwen2.5-0.5b-int4-decode"
+
+
+# ---------------------------------------------------------------------------
+# host-side helpers (no GPU needed; covered by the CPU tests)
+# ---------------------------------------------------------------------------
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained",
+                                                     d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def workload_bytes(name: str) -> int:
+    shape_set, layers, mode, bits, group, M, _ = WORKLOADS[name]
+    return sum(wl.gemv_bytes(m.K, m.N, M, mode, bits, m.K if group == 0 else group)
+               for m in wl.layer_set(shape_set, layers))
+
+
+def workload_flops(name: str) -> int:
+    shape_set, layers, _, _, _, M, _ = WORKLOADS[name]
+    return sum(2 * M * m.N * m.K for m in wl.layer_set(shape_set, layers))
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    for f in ("bc_gemv.cu", "bc_internal.cuh"):
+        with open(os.path.join(ROOT, "quantized_matmul_02_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(name: str):
+    """DRAM bytes per launch from a committed ncu summary, if the summary's
+    kernel-source digest matches the current sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{name}.txt")
+    try:
+        fields = dict(line.split(":", 1) for line in open(path) if ":" in line)
+    except OSError:
+        return None
+    if fields.get("source_digest", "").strip() != kernel_source_digest():
+        return None
+    try:
+        return int(fields["dram_bytes_per_launch"].strip())
+    except (KeyError, ValueError):
+        return None
+
+
+def aggregate_times(times_ms, n_gpus: int, units_per_rank: float):
+    """Whole-job throughput from per-rank elapsed times: the job takes the
+    slowest rank's time; every rank processed `units_per_rank`."""
+    t = max(times_ms)
+    return {"ms": t, "value": units_per_rank * n_gpus / (t / 1e3)}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML on a thread."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown",
+               0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap",
+               0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self._stop = [], threading.Event()
+        self.window = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: report no clocks
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM)
+                r = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, r))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0}
+        t0, t1 = self.window
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        used = inside if inside else self.samples
+        reasons = set()
+        for _, _, r in used:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[1] for s in used),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(used), "samples_in_timed_region": len(inside)}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--copies", type=int, default=0,
+                    help="weight copies rotated between steps (0 = enough to "
+                         "exceed 4x the L2)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# workload construction on the GPU
+# ---------------------------------------------------------------------------
+
+def build_workload(qmm, torch, name: str, copies: int):
+    """Upload the seeded fp16 weights, run the one-time precompute (group
+    params / int4 pack) with the library, and return `copies` independent
+    device copies of the step's inputs plus the shared x / y buffers."""
+    shape_set, layers, mode, bits, group, M, seed = WORKLOADS[name]
+    mats = wl.layer_set(shape_set, layers)
+    sigma = wl.SIGMA[shape_set]
+    xs_host, xs_dev = {}, {}
+    per_copy = [[] for _ in range(copies)]
+    ys = []
+    for m in mats:
+        key = (m.layer, m.x_tag)
+        if key not in xs_dev:
+            xh = wl.activation(seed, m.layer, m.x_tag, M, m.K)
+            xs_host[key] = xh
+            xs_dev[key] = torch.from_numpy(xh).cuda()
+        W = torch.from_numpy(wl.weight(seed, m.layer, m.name, m.K, m.N, sigma)).cuda()
+        if mode == "packed":
+            s, z = qmm.group_params(W, 4, 64, torch.float16)
+            Wk = qmm.pack_int4(W, s, z)
+            del W
+        elif bits == 16:
+            s = z = None
+            Wk = W
+        else:
+            s, z = qmm.group_params(W, bits, group, torch.float32)
+            Wk = W
+        y = torch.empty((M, m.N), dtype=torch.float32, device="cuda")
+        ys.append(y)
+        for c in range(copies):
+            if c == 0:
+                per_copy[c].append((xs_dev[key], Wk, s, z, y))
+            else:
+                per_copy[c].append((xs_dev[key], Wk.clone(),
+                                    None if s is None else s.clone(),
+                                    None if z is None else z.clone(), y))
+    torch.cuda.synchronize()
+    descs = [qmm.make_descs(items) for items in per_copy]
+    return {"mats": mats, "descs": descs, "xs_host": xs_host, "xs_dev": xs_dev,
+            "ys": ys, "per_copy": per_copy, "mode": mode, "bits": bits,
+            "group": group, "M": M}
+
+
+def cpu_baseline_sample(name: str, target_s: float = 12.0):
+    """The oracle (as it stands) on a bounded sample of the workload: for
+    whole matrices of the first layers, dequantize the codes and multiply
+    (the work one GPU step does), until about `target_s` seconds pass."""
+    import oracle
+    shape_set, layers, mode, bits, group, M, seed = WORKLOADS[name]
+    mats = wl.layer_set(shape_set, layers)
+    sigma = wl.SIGMA[shape_set]
+    done_bytes, spent = 0, 0.0
+    done = 0
+    for m in mats:
+        W = wl.weight(seed, m.layer, m.name, m.K, m.N, sigma)
+        x = wl.activation(seed, m.layer, m.x_tag, M, m.K).astype(np.float64)
+        g = m.K if group == 0 else group
+        if mode == "runtime" and bits == 16:
+            t0 = time.perf_counter()
+            oracle.matmul(x, oracle.half_to_f64(W))
+            spent += time.perf_counter() - t0
+        else:
+            s, z = oracle.group_params(W, bits, g, mode == "packed")
+            q = oracle.codes(W, s, z, bits, g)
+            t0 = time.perf_counter()
+            if mode == "runtime":   # runtime mode re-derives the codes per step
+                s, z = oracle.group_params(W, bits, g, False)
+                q = oracle.codes(W, s, z, bits, g)
+            oracle.matmul(x, oracle.dequant(q, s, z, g))
+            spent += time.perf_counter() - t0
+        done_bytes += wl.gemv_bytes(m.K, m.N, M, mode, bits, g)
+        done += 1
+        if spent >= target_s:
+            break
+    return {"value": done_bytes / spent / 1e9, "unit": "GB/s",
+            "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{done} of {len(mats)} matrices of {name} (first layers), "
+                      f"fp64 dequant + matmul, {spent:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def _reference_sample(name: str, rows: int):
+    """Layer 0's matrices of the workload, first `rows` rows of each, with
+    the codes precomputed (the one-time part): what one oracle step eats."""
+    import oracle
+    shape_set, layers, mode, bits, group, M, seed = WORKLOADS[name]
+    out = []
+    for m in wl.layer_set(shape_set, 1):
+        n = min(rows, m.N)
+        W = wl.weight(seed, m.layer, m.name, m.K, m.N, wl.SIGMA[shape_set])[:n]
+        x = wl.activation(seed, m.layer, m.x_tag, M, m.K).astype(np.float64)
+        g = m.K if group == 0 else group
+        item = {"W": W, "x": x, "g": g,
+                "bytes": wl.gemv_bytes(m.K, n, M, mode, bits, g)}
+        if not (mode == "runtime" and bits == 16):
+            s, z = oracle.group_params(W, bits, g, mode == "packed")
+            item.update(s=s, z=z, q=oracle.codes(W, s, z, bits, g))
+        out.append(item)
+    return out
+
+
+def _reference_pass(name: str, sample) -> None:
+    import oracle
+    _, _, mode, bits, _, _, _ = WORKLOADS[name]
+    for it in sample:
+        if mode == "runtime" and bits == 16:
+            oracle.matmul(it["x"], oracle.half_to_f64(it["W"]))
+            continue
+        s, z, q = it["s"], it["z"], it["q"]
+        if mode == "runtime":     # runtime mode re-derives the codes per step
+            s, z = oracle.group_params(it["W"], bits, it["g"], False)
+            q = oracle.codes(it["W"], s, z, bits, it["g"])
+        oracle.matmul(it["x"], oracle.dequant(q, s, z, it["g"]))
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, timed on this host's cores: each step is one
+    pass over a bounded sample of the workload (the first rows of every
+    matrix of layer 0), sized so the whole run stays within ~2 minutes."""
+    if rank != 0:
+        return 0
+    import oracle
+    name = args.workload
+    rows = 512
+    sample = _reference_sample(name, rows)
+    t0 = time.perf_counter()
+    _reference_pass(name, sample)
+    one = time.perf_counter() - t0
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    if one > budget:
+        rows = max(8, int(rows * budget / one))
+        sample = _reference_sample(name, rows)
+    for _ in range(args.warmup):
+        _reference_pass(name, sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _reference_pass(name, sample)
+    spent = time.perf_counter() - t0
+    sbytes = sum(it["bytes"] for it in sample)
+    value = sbytes * args.steps / spent / 1e9
+    desc = (f"first {rows} rows of each of layer 0's {len(sample)} matrices "
+            f"({sbytes} algorithmic bytes per step), fp64 oracle")
+    line = {"metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": spent / max(1, args.steps) * 1e3,
+            "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": name, "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "GB/s",
+                             "cores": oracle.threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "GB/s",
+                    "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import quantized_matmul_02_b200 as qmm
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    name = args.workload
+    shape_set, layers, mode, bits, group, M, _ = WORKLOADS[name]
+    step_bytes = workload_bytes(name)
+    l2 = torch.cuda.get_device_properties(local_rank).L2_cache_size
+    copies = args.copies or max(2, int(np.ceil(4 * l2 / step_bytes)) + 1)
+    copies = min(copies, 8)
+    W = build_workload(qmm, torch, name, copies)
+    mode_id = qmm.BC_MODE_PACKED_INT4 if mode == "packed" else qmm.BC_MODE_RUNTIME
+    ws_bytes = max(qmm.workspace_size_batched(d, M, mode_id, qmm.BC_F32) for d in W["descs"])
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        qmm.matmul_q_batched(W["descs"][i % copies], M, bits, group, mode_id,
+                             workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.05)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    if dist:
+        dist.barrier()
+    sampler.mark(t0, t1)
+    time.sleep(0.02)
+    sampler.stop()
+    elapsed_ms = start.elapsed_time(end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    times = [elapsed_ms]
+    if dist:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        times = [float(t.item())]
+    agg = aggregate_times(times, world, step_bytes * args.steps / 1e9)
+    ms_per_step = agg["ms"] / args.steps
+
+    # ---- end to end through the public API: pinned host x in, y out ----
+    xs_pinned = {k: torch.from_numpy(v).pin_memory() for k, v in W["xs_host"].items()}
+    ys_pinned = [torch.empty(y.shape, dtype=torch.float32).pin_memory() for y in W["ys"]]
+    h2d = sum(v.numel() * 4 for v in xs_pinned.values())
+    d2h = sum(y.numel() * 4 for y in ys_pinned)
+
+    def e2e_step(i):
+        for k, v in xs_pinned.items():
+            W["xs_dev"][k].copy_(v, non_blocking=True)
+        step(i)
+        for yd, yh in zip(W["ys"], ys_pinned):
+            yh.copy_(yd, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    e_steps = max(10, min(args.steps, 200))
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    es.record(stream)
+    for i in range(e_steps):
+        e2e_step(i)
+    ee.record(stream)
+    torch.cuda.synchronize()
+    e_ms = es.elapsed_time(ee)
+    if dist:
+        t = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e_value = step_bytes * e_steps * world / (e_ms / 1e3) / 1e9
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks = measured_peaks()
+    avg_launch_ms = float(np.mean(launch_ms))
+    achieved = step_bytes / (avg_launch_ms / 1e3) / 1e9
+    traffic = recorded_traffic(name)
+    line = {
+        "metric": METRIC, "value": agg["value"], "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": name, "shape_set": shape_set, "layers": layers,
+                   "matrices": len(W["mats"]), "mode": mode, "bits": bits,
+                   "group": group if group else "per-channel", "M": M,
+                   "weights": "int4 packed, fp16 scale/zero per 64-block"
+                   if mode == "packed" else "fp16, runtime RTN",
+                   "x": "fp32", "bytes_per_step": step_bytes,
+                   "l2": f"inputs larger than L2: {copies} weight copies "
+                         f"({copies * step_bytes / 1e6:.0f} MB) rotated between "
+                         f"steps, L2 {l2 / 1e6:.0f} MB",
+                   "launch": "one grouped launch per step"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": traffic,
+                     "peak_source": f"{peaks['source']} copy bandwidth "
+                                    "(MEASURED_PEAKS.json hbm_gbs)",
+                     "kernel": "gemv_kernel (bc_gemv.cu)",
+                     "avg_launch_us": avg_launch_ms * 1e3},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "ms_per_step": e_ms / e_steps, "steps": e_steps},
+        "gpu_launches": args.steps * ((M + 15) // 16) * ((len(W["mats"]) + 367) // 368),
+        "clocks": sampler.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_sample(name)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,197 @@
+/*
+ * bc.h -- C ABI of the B200 fused group-wise quantize/dequantize matmul.
+ *
+ * The operation (BITCRUSH BC-06, "Under the hood"): matmul_q multiplies an
+ * activation by a weight matrix whose entries are re-quantized group-wise
+ * with an affine round-to-nearest (RTN) code as they are read; a separate
+ * kernel precomputes one scale and one zero point per group.  The NAIVE /
+ * SMART row of the same page's "The machine" table fixes the two group
+ * shapes: one scale per output channel (group = K) or one per 64-weight
+ * group.  Enargeia ("Four bits per weight") fixes the packed mode: int4
+ * codes in blocks of 64 along the reduction axis, each block with its own
+ * scale and zero point, unpacked in registers and never written back.
+ *
+ * Arithmetic convention (the pages leave it open):
+ *   L      = 2^bits - 1
+ *   scale  = fl32(fl32(max - min) / L)            over the group's fp16 weights
+ *            (a constant group c takes scale |c|, or 1 when c == 0)
+ *   zero   = round(-min / scale)
+ *   q      = clamp(round(w / scale) + zero, 0, L)
+ *   w'     = (q - zero) * scale
+ *   y[m,n] = sum_k x[m,k] * w'[n,k]
+ * round() is round-half-to-even of the EXACT real quotient.  fp16-stored
+ * parameters (packed mode) round the fp32 scale to fp16 (RNE, floored at
+ * 2^-24), derive zero and codes from that stored scale, and store zero as
+ * fp16 (RNE).
+ *
+ * Layouts (all row-major, C order):
+ *   W       fp16 [N][K]            (PyTorch Linear weight: N = out, K = in)
+ *   scales  [N][K/group]           fp32 (runtime mode) or fp16 (packed mode)
+ *   zeros   [N][K/group]           same dtype as scales
+ *   codes   uint8 [N][K]
+ *   packed  uint8 [N][K/2]         byte = q[n][2i] | q[n][2i+1] << 4
+ *   x       [M][K]                 fp32, or bf16 for the tensor-core path
+ *   y       fp32 [M][N]
+ *
+ * Conventions shared by every call:
+ *   - Pointers named W, x, y, scales, zeros, codes, packed, workspace are
+ *     DEVICE pointers owned by the caller; the library never allocates,
+ *     frees or keeps them, and keeps no per-call device state.
+ *   - Calls only enqueue work on `stream` (NULL = legacy default stream)
+ *     and return without synchronising.  Arguments are validated on the
+ *     host before anything is enqueued; a rejected call enqueues nothing.
+ *   - Launch failures are reported as BC_ERR_CUDA (cudaGetLastError); an
+ *     asynchronous fault surfaces at the caller's next synchronisation.
+ *   - K must be a multiple of 64; W, x and packed must be 16-byte aligned;
+ *     scales/zeros aligned to their element size; y 4-byte aligned.
+ *   - Inputs must be finite (no NaN / Inf weights or activations).
+ *   - No call throws; nothing falls back to the CPU.
+ */
+#ifndef BC_H_
+#define BC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define BC_API __attribute__((visibility("default")))
+#else
+#define BC_API
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st *bc_stream_t;
+
+typedef enum bc_status {
+    BC_OK = 0,
+    BC_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, K % 64 != 0 */
+    BC_ERR_UNSUPPORTED = 2,   /* bits / group / mode / dtype combination not offered */
+    BC_ERR_ALIGNMENT = 3,     /* a pointer is not aligned as stated above */
+    BC_ERR_WORKSPACE = 4,     /* workspace smaller than bc_workspace_size() */
+    BC_ERR_CUDA = 5           /* a CUDA launch or runtime call failed */
+} bc_status;
+
+typedef enum bc_dtype { BC_F32 = 0, BC_F16 = 1, BC_BF16 = 2 } bc_dtype;
+
+typedef enum bc_mode {
+    BC_MODE_RUNTIME = 0,      /* fp16 W re-quantized inline to `bits` (2..8), or 16 = passthrough */
+    BC_MODE_PACKED_INT4 = 1   /* pre-packed int4 codes, fp16 scale/zero per 64-block */
+} bc_mode;
+
+/* Per-channel grouping may be requested as group == K or group == 0. */
+#define BC_GROUP_PER_CHANNEL 0
+
+/*
+ * bc_group_params -- per-group scale/zero precompute (BITCRUSH BC-06,
+ * "Under the hood": the per-group scale/zero precompute kernel; a lever
+ * move reruns it once, then decoding uses one uniform).
+ *   W          fp16 [N][K], device
+ *   bits       2..8
+ *   group      64, or K / 0 for per-channel
+ *   out_dtype  BC_F32 (runtime mode) or BC_F16 (packed int4 mode)
+ *   scales     [N][K/group] of out_dtype, device, written
+ *   zeros      [N][K/group] of out_dtype, device, written
+ */
+BC_API bc_status bc_group_params(const void *W, int64_t N, int64_t K, int bits,
+                          int64_t group, bc_dtype out_dtype, void *scales,
+                          void *zeros, bc_stream_t stream);
+
+/*
+ * bc_quantize_codes -- the RTN codes q = clamp(round(w/scale)+zero, 0, L)
+ * as a standalone output (the same codes matmul_q forms inline; BITCRUSH
+ * BC-06, "Under the hood").  Used for validation and the WEIGHT SCOPE-style
+ * code histogram.
+ *   W        fp16 [N][K], device
+ *   scales, zeros  [N][K/group], dtype sz_dtype (BC_F32 or BC_F16), device
+ *   codes    uint8 [N][K], device, written
+ */
+BC_API bc_status bc_quantize_codes(const void *W, const void *scales,
+                            const void *zeros, bc_dtype sz_dtype, int64_t N,
+                            int64_t K, int bits, int64_t group,
+                            uint8_t *codes, bc_stream_t stream);
+
+/*
+ * bc_pack_int4 -- one-time int4 packing (Enargeia, "Four bits per weight":
+ * four bits per weight, blocks of 64 along K with their own scale and
+ * zero point).
+ *   W                  fp16 [N][K], device
+ *   scales_f16, zeros_f16  fp16 [N][K/64] from bc_group_params(..., BC_F16)
+ *   packed             uint8 [N][K/2], device, written; low nibble = even k
+ */
+BC_API bc_status bc_pack_int4(const void *W, const void *scales_f16,
+                       const void *zeros_f16, int64_t N, int64_t K,
+                       uint8_t *packed, bc_stream_t stream);
+
+/*
+ * bc_matmul_q -- y = x . deq(W)^T (BITCRUSH BC-06 matmul_q; Enargeia int4
+ * weights unpacked in registers).
+ *   x, x_dtype   [M][K]: BC_F32 for any M; BC_BF16 only for M >= 64 in
+ *                BC_MODE_PACKED_INT4 (tensor-core prefill, fp32 accumulate)
+ *   W_or_packed  fp16 W [N][K] (runtime) or packed uint8 [N][K/2] (packed)
+ *   scales, zeros  fp32 [N][K/group] (runtime) or fp16 [N][K/64] (packed);
+ *                ignored (may be NULL) when bits == 16
+ *   bits         runtime: 2..8 or 16 (fp16 passthrough); packed: 4
+ *   group        runtime: 64, or K / 0 (per channel); packed: 64
+ *   y            fp32 [M][N], device, written (not accumulated into)
+ *   workspace    device scratch of at least bc_workspace_size() bytes
+ *                (may be NULL when that size is 0); its contents on entry
+ *                do not matter; overlapping calls must not share it
+ * Decode shapes (M < 64, fp32 x) use the fused dequant GEMV; M >= 64 with
+ * bf16 x uses the tcgen05 tensor-core GEMM.
+ */
+BC_API bc_status bc_matmul_q(const void *x, bc_dtype x_dtype, const void *W_or_packed,
+                      const void *scales, const void *zeros, int64_t M,
+                      int64_t N, int64_t K, int bits, int64_t group,
+                      bc_mode mode, float *y, void *workspace,
+                      size_t workspace_bytes, bc_stream_t stream);
+
+/* Workspace bytes bc_matmul_q needs for this shape (0 if none). */
+BC_API size_t bc_workspace_size(int64_t M, int64_t N, int64_t K, bc_mode mode);
+
+/*
+ * One matrix of a grouped launch.  All pointers are device pointers with
+ * the layouts above; several descriptors may share one x.
+ */
+typedef struct bc_matmul_desc {
+    const void *x;
+    const void *W_or_packed;
+    const void *scales;
+    const void *zeros;
+    float *y;
+    int64_t N;
+    int64_t K;
+} bc_matmul_desc;
+
+/*
+ * bc_matmul_q_batched -- one grouped launch over many independent matrices
+ * that share M, bits, group rule, mode and x dtype (a whole layer set).
+ * Enargeia ("One decode step") shows that a decode step is a list of
+ * hundreds of small passes; launching them one by one costs more than the
+ * work of the small ones.
+ *   descs   HOST array of `count` descriptors (read before return)
+ *   group   64, or 0 for per-channel (each matrix uses its own K)
+ *   workspace  as for bc_matmul_q, at least bc_workspace_size_batched()
+ */
+BC_API bc_status bc_matmul_q_batched(const bc_matmul_desc *descs, int count,
+                              int64_t M, int bits, int64_t group,
+                              bc_mode mode, bc_dtype x_dtype, void *workspace,
+                              size_t workspace_bytes, bc_stream_t stream);
+
+BC_API size_t bc_workspace_size_batched(const bc_matmul_desc *descs, int count,
+                                 int64_t M, bc_mode mode, bc_dtype x_dtype);
+
+/* Static description of a status code. */
+BC_API const char *bc_status_string(bc_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+BC_API int bc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BC_H_ */

@@ -1,0 +1,80 @@
+// bc_internal.cuh -- shared declarations of the CUDA library (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/bc.h"
+
+namespace bc {
+
+// ---------------------------------------------------------------------------
+// Host-side helpers
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+    int sm_count = 0;
+    int cc_major = 0, cc_minor = 0;
+    int max_smem_optin = 0;
+};
+// Cached per device; returns false if the CUDA runtime fails.
+bool device_info(DeviceInfo *out);
+
+inline bool aligned(const void *p, size_t a) {
+    return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+inline bc_status cuda_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? BC_OK : BC_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Quantizer kernels (bc_quant.cu)
+// ---------------------------------------------------------------------------
+bc_status launch_group_params(const __half *W, int64_t N, int64_t K, int bits,
+                              int64_t group, bool f16_out, void *scales,
+                              void *zeros, cudaStream_t s);
+bc_status launch_quantize_codes(const __half *W, const void *scales,
+                                const void *zeros, bool f16_sz, int64_t N,
+                                int64_t K, int bits, int64_t group,
+                                uint8_t *codes, cudaStream_t s);
+bc_status launch_pack_int4(const __half *W, const __half *scales,
+                           const __half *zeros, int64_t N, int64_t K,
+                           uint8_t *packed, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// Fused dequant GEMV (bc_gemv.cu), M < 64, fp32 x
+// ---------------------------------------------------------------------------
+struct GemvJob {             // one matrix of a launch
+    const float *x;          // [M][K]
+    const void *w;           // fp16 [N][K] or packed [N][K/2]
+    const void *s;           // fp32 / fp16 [N][K/g]
+    const void *z;
+    float *y;                // [M][N]
+    int64_t N, K;
+    int64_t group;           // 64 or K
+};
+// Bytes of split-K scratch a launch over these jobs needs.
+size_t gemv_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed,
+                            int sm_count);
+bc_status launch_gemv(const GemvJob *jobs, int count, int M, int bits,
+                      bool packed, void *workspace, size_t ws_bytes,
+                      cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// tcgen05 prefill GEMM (bc_gemm_sm100.cu), packed int4 W, bf16 x, M >= 64
+// ---------------------------------------------------------------------------
+struct GemmJob {
+    const __nv_bfloat16 *x;  // [M][K]
+    const uint8_t *w;        // packed [N][K/2]
+    const __half *s;         // [N][K/64]
+    const __half *z;
+    float *y;                // [M][N]
+    int64_t N, K;
+};
+bc_status launch_gemm_packed(const GemmJob *jobs, int count, int64_t M,
+                             cudaStream_t s);
+
+}  // namespace bc

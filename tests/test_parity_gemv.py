@@ -1,0 +1,211 @@
+"""GPU parity of the fused dequant GEMV (decode shapes, fp32 x) against the
+oracle: max |y - y_ref| <= 1e-4 * sum_k |x_k * w'_nk| per output element.
+
+BITCRUSH BC-06 "Under the hood" (matmul_q: runtime RTN inline as weights
+are read; NAIVE / SMART row: per-channel vs per-group) and Enargeia "Four
+bits per weight" (packed int4 unpacked in registers)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from parity_util import TOL_FP32, assert_close, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _runtime_case(qmm, W, x, bits, group):
+    N, K = W.shape
+    g = K if group == 0 else group
+    Wd, xd = dev(W), dev(x)
+    if bits == 16:
+        s = z = None
+        ref = oracle.matmul_q(x, W, 16, g, "runtime")
+    else:
+        s, z = qmm.group_params(Wd, bits, group, torch.float32)
+        ref = oracle.matmul_q(x, W, bits, g, "runtime")
+        np.testing.assert_array_equal(host(s).astype(np.float64), ref["s"])
+    y = qmm.matmul_q(xd, Wd, s, z, bits, group, qmm.BC_MODE_RUNTIME)
+    return host(y), ref
+
+
+def _packed_case(qmm, W, x):
+    Wd, xd = dev(W), dev(x)
+    s, z = qmm.group_params(Wd, 4, 64, torch.float16)
+    p = qmm.pack_int4(Wd, s, z)
+    ref = oracle.matmul_q(x, W, 4, 64, "packed")
+    np.testing.assert_array_equal(host(p), ref["packed"])
+    y = qmm.matmul_q(xd, p, s, z, 4, 64, qmm.BC_MODE_PACKED_INT4)
+    return host(y), ref
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("group", [64, 0])
+def test_single_layer_1024_runtime(cuda_lib, bits, group):
+    """The 1024 x 1024 single-layer workload (seed 0), M = 1."""
+    W = wl.weight(0, 0, "single", 1024, 1024, 0.02)
+    x = wl.activation(0, 0, "x", 1, 1024)
+    y, ref = _runtime_case(cuda_lib, W, x, bits, group)
+    assert_close(y, ref["y"], ref["A"], TOL_FP32, f"bits={bits} group={group}")
+
+
+def test_single_layer_1024_group_beats_channel_on_gpu(cuda_lib):
+    """NAIVE / SMART on the GPU output: per-group output error against the
+    fp16 reference matmul is smaller than per-channel at 3 bits."""
+    W = wl.weight(0, 0, "single", 1024, 1024, 0.02)
+    x = wl.activation(0, 0, "x", 1, 1024)
+    y16, _ = _runtime_case(cuda_lib, W, x, 16, 64)
+    err = {}
+    for group in (64, 0):
+        y, _ = _runtime_case(cuda_lib, W, x, 3, group)
+        err[group] = np.mean((y.astype(np.float64) - y16) ** 2)
+    assert err[64] < err[0]
+
+
+@pytest.mark.parametrize("M", [2, 5, 16, 17, 40])
+@pytest.mark.parametrize("bits,group", [(3, 64), (8, 0), (16, 64)])
+def test_runtime_multi_row(cuda_lib, M, bits, group):
+    W = wl.weight(11, 0, "single", 1024, 300, 0.02)
+    x = wl.activation(11, 0, "x", M, 1024)
+    y, ref = _runtime_case(cuda_lib, W, x, bits, group)
+    assert_close(y, ref["y"], ref["A"], TOL_FP32, f"M={M} bits={bits}")
+
+
+@pytest.mark.parametrize("M", [1, 3, 16, 21])
+@pytest.mark.parametrize("NK", [(896, 896), (128, 896), (896, 4864), (37, 192),
+                                (1, 64)])
+def test_packed_shapes(cuda_lib, M, NK):
+    N, K = NK
+    W = wl.weight(12, M, "single", K, N, 0.02)
+    x = wl.activation(12, M, "x", M, K)
+    y, ref = _packed_case(cuda_lib, W, x)
+    assert_close(y, ref["y"], ref["A"], TOL_FP32, f"packed M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
+def test_runtime_ties_take_exact_path(cuda_lib, bits):
+    """Weights on the quantization grid with many exact half-way points:
+    the fast reciprocal path must hand these to the exact quotient."""
+    rng = np.random.default_rng(40 + bits)
+    L = (1 << bits) - 1
+    N, K = 64, 512
+    G = K // 64
+    e = rng.integers(4, 10, size=(N, G)).astype(np.float64)
+    z = rng.integers(1, L, size=(N, G))
+    h = rng.integers(0, L, size=(N, K)) + 0.5 * rng.integers(0, 2, size=(N, K))
+    h[:, 0::64] = 0
+    h[:, 1::64] = L
+    w = (h - np.repeat(z, 64, axis=1)) * np.repeat(np.ldexp(1.0, -e), 64, axis=1)
+    W = w.astype(np.float16)
+    assert np.array_equal(W.astype(np.float64), w)
+    x = wl.activation(13, bits, "x", 1, K)
+    y, ref = _runtime_case(cuda_lib, W, x, bits, 64)
+    assert_close(y, ref["y"], ref["A"], TOL_FP32, f"ties bits={bits}")
+
+
+def test_edge_rows_runtime_and_packed(cuda_lib):
+    from test_parity_quant import _edge_matrix
+    W = _edge_matrix(8)
+    x = wl.activation(14, 0, "x", 3, W.shape[1])
+    for bits, group in ((2, 64), (4, 0), (8, 64)):
+        y, ref = _runtime_case(cuda_lib, W, x, bits, group)
+        assert_close(y, ref["y"], ref["A"], TOL_FP32, f"edges bits={bits}")
+    y, ref = _packed_case(cuda_lib, W, x)
+    assert_close(y, ref["y"], ref["A"], TOL_FP32, "edges packed")
+
+
+@pytest.mark.parametrize("mode", ["runtime", "packed"])
+def test_split_k_small_n_is_deterministic(cuda_lib, mode):
+    """A lone small-N matrix is split along K; the last CTA reduces the
+    partials in split order, so repeated calls are bit-identical."""
+    N, K = 128, 4864
+    assert cuda_lib.workspace_size(1, N, K, int(mode == "packed")) > 0
+    W = wl.weight(15, 0, "single", K, N, 0.02)
+    x = wl.activation(15, 0, "x", 1, K)
+    if mode == "runtime":
+        y, ref = _runtime_case(cuda_lib, W, x, 4, 64)
+    else:
+        y, ref = _packed_case(cuda_lib, W, x)
+    assert_close(y, ref["y"], ref["A"], TOL_FP32, f"split-K {mode}")
+    Wd, xd = dev(W), dev(x)
+    s, z = cuda_lib.group_params(Wd, 4, 64,
+                                 torch.float32 if mode == "runtime" else torch.float16)
+    Wk = Wd if mode == "runtime" else cuda_lib.pack_int4(Wd, s, z)
+    m = cuda_lib.BC_MODE_RUNTIME if mode == "runtime" else cuda_lib.BC_MODE_PACKED_INT4
+    outs = [host(cuda_lib.matmul_q(xd, Wk, s, z, 4, 64, m)) for _ in range(5)]
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+
+
+def _layer_set_case(qmm, shape_set, layers, workload, mode, bits, group, M=1):
+    mats = wl.layer_set(shape_set, layers)
+    xs, items, refs = {}, [], []
+    keep = []
+    for m in mats:
+        key = (m.layer, m.x_tag)
+        if key not in xs:
+            xs[key] = wl.activation(workload, m.layer, m.x_tag, M, m.K)
+        x = xs[key]
+        W = wl.weight(workload, m.layer, m.name, m.K, m.N, wl.SIGMA[shape_set])
+        g = m.K if group == 0 else group
+        Wd = dev(W)
+        if mode == "packed":
+            s, z = qmm.group_params(Wd, 4, 64, torch.float16)
+            Wk = qmm.pack_int4(Wd, s, z)
+            ref = oracle.matmul_q(x, W, 4, 64, "packed")
+        elif bits == 16:
+            s = z = None
+            Wk = Wd
+            ref = oracle.matmul_q(x, W, 16, g, "runtime")
+        else:
+            s, z = qmm.group_params(Wd, bits, group, torch.float32)
+            Wk = Wd
+            ref = oracle.matmul_q(x, W, bits, g, "runtime")
+        y = torch.full((M, m.N), float("nan"), device="cuda")
+        xd = dev(x)
+        keep.append((xd, Wk, s, z, y))
+        items.append((xd, Wk, s, z, y))
+        refs.append((m, ref))
+    descs = qmm.make_descs(items)
+    mode_id = qmm.BC_MODE_PACKED_INT4 if mode == "packed" else qmm.BC_MODE_RUNTIME
+    ws_bytes = qmm.workspace_size_batched(descs, M, mode_id, qmm.BC_F32)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
+    qmm.matmul_q_batched(descs, M, bits, group, mode_id, workspace=ws)
+    torch.cuda.synchronize()
+    for (m, ref), it in zip(refs, items):
+        assert_close(host(it[4]), ref["y"], ref["A"], TOL_FP32,
+                     f"{shape_set} L{m.layer} {m.name}")
+
+
+def test_batched_qwen25_packed_two_layers(cuda_lib):
+    _layer_set_case(cuda_lib, "qwen2.5-0.5b", 2, 1, "packed", 4, 64)
+
+
+@pytest.mark.parametrize("bits,group", [(3, 64), (3, 0), (16, 64), (2, 64)])
+def test_batched_qwen3_runtime_one_layer(cuda_lib, bits, group):
+    _layer_set_case(cuda_lib, "qwen3-0.6b", 1, 2, "runtime", bits, group)
+
+
+def test_batched_qwen3_8b_one_layer_m16(cuda_lib):
+    _layer_set_case(cuda_lib, "qwen3-8b", 1, 4, "packed", 4, 64, M=16)
+    _layer_set_case(cuda_lib, "qwen3-8b", 1, 4, "runtime", 3, 64, M=1)
+
+
+def test_determinism_batched(cuda_lib):
+    """Enargeia: the output is identical every run (no float atomics)."""
+    mats = wl.layer_set("qwen2.5-0.5b", 1)
+    items = []
+    for m in mats:
+        W = dev(wl.weight(1, 0, m.name, m.K, m.N, 0.02))
+        s, z = cuda_lib.group_params(W, 4, 64, torch.float16)
+        items.append((dev(wl.activation(1, 0, m.x_tag, 1, m.K)),
+                      cuda_lib.pack_int4(W, s, z), s, z,
+                      torch.empty((1, m.N), device="cuda")))
+    descs = cuda_lib.make_descs(items)
+    outs = []
+    for _ in range(10):
+        cuda_lib.matmul_q_batched(descs, 1, 4, 64, cuda_lib.BC_MODE_PACKED_INT4)
+        outs.append(torch.cat([it[4].flatten() for it in items]).cpu())
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
