@@ -184,6 +184,16 @@ BC_API bc_status bc_matmul_q_batched(const bc_matmul_desc *descs, int count,
 BC_API size_t bc_workspace_size_batched(const bc_matmul_desc *descs, int count,
                                  int64_t M, bc_mode mode, bc_dtype x_dtype);
 
+/*
+ * bc_device_timeouts -- number of bounded in-kernel waits (tensor-core
+ * pipeline barriers) that ran out on the current device since the library
+ * was loaded.  A kernel whose wait runs out stops early, frees its tensor
+ * memory and leaves its outputs incomplete instead of hanging the GPU; a
+ * nonzero count means some earlier output is not valid.  Synchronises the
+ * device.  `count` is a HOST pointer.
+ */
+BC_API bc_status bc_device_timeouts(unsigned *count);
+
 /* Static description of a status code. */
 BC_API const char *bc_status_string(bc_status status);
 

@@ -29,7 +29,8 @@ GROUP_PER_CHANNEL = 0
 # Every symbol include/bc.h declares.
 EXPORTS = ("bc_group_params", "bc_quantize_codes", "bc_pack_int4",
            "bc_matmul_q", "bc_workspace_size", "bc_matmul_q_batched",
-           "bc_workspace_size_batched", "bc_status_string", "bc_version")
+           "bc_workspace_size_batched", "bc_device_timeouts",
+           "bc_status_string", "bc_version")
 
 
 class BCError(RuntimeError):
@@ -64,6 +65,8 @@ def _load() -> ctypes.CDLL:
     lib.bc_workspace_size_batched.argtypes = [ctypes.POINTER(MatmulDesc), i32,
                                               i64, i32, i32]
     lib.bc_workspace_size_batched.restype = sz
+    lib.bc_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+    lib.bc_device_timeouts.restype = i32
     lib.bc_status_string.argtypes = [i32]
     lib.bc_status_string.restype = ctypes.c_char_p
     lib.bc_version.restype = i32
@@ -188,3 +191,10 @@ def matmul_q_batched(descs, M: int, bits: int, group: int, mode: int,
     _check(lib.bc_matmul_q_batched(descs, len(descs), M, bits, group, mode,
                                    x_dtype, wsp, wsb, _stream(stream)),
            "bc_matmul_q_batched")
+
+
+def device_timeouts() -> int:
+    """Bounded in-kernel waits that ran out on this device (0 when healthy)."""
+    c = ctypes.c_uint(0)
+    _check(lib.bc_device_timeouts(ctypes.byref(c)), "bc_device_timeouts")
+    return int(c.value)

@@ -113,6 +113,15 @@ const char *bc_status_string(bc_status st) {
 
 int bc_version(void) { return 100; }
 
+bc_status bc_device_timeouts(unsigned *count) {
+    if (!count) return BC_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return BC_ERR_CUDA;
+    const unsigned v = gemm_timeouts();
+    if (v == ~0u) return BC_ERR_CUDA;
+    *count = v;
+    return BC_OK;
+}
+
 bc_status bc_group_params(const void *W, int64_t N, int64_t K, int bits,
                           int64_t group, bc_dtype out_dtype, void *scales,
                           void *zeros, bc_stream_t stream) {

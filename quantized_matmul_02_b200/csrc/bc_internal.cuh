@@ -76,5 +76,7 @@ struct GemmJob {
 };
 bc_status launch_gemm_packed(const GemmJob *jobs, int count, int64_t M,
                              cudaStream_t s);
+// Bounded waits of the GEMM that ran out on the current device since load.
+unsigned gemm_timeouts();
 
 }  // namespace bc

@@ -91,7 +91,7 @@ def test_runtime_ties_take_exact_path(cuda_lib, bits):
     L = (1 << bits) - 1
     N, K = 64, 512
     G = K // 64
-    e = rng.integers(4, 10, size=(N, G)).astype(np.float64)
+    e = rng.integers(4, 10, size=(N, G))
     z = rng.integers(1, L, size=(N, G))
     h = rng.integers(0, L, size=(N, K)) + 0.5 * rng.integers(0, 2, size=(N, K))
     h[:, 0::64] = 0
