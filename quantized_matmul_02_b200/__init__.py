@@ -185,7 +185,12 @@ def workspace_size_batched(descs, M: int, mode: int, x_dtype: int) -> int:
 def matmul_q_batched(descs, M: int, bits: int, group: int, mode: int,
                      x_dtype: int = BC_F32, workspace: Optional[torch.Tensor] = None,
                      stream=None) -> None:
-    """One grouped launch over the matrices in `descs` (from make_descs)."""
+    """One grouped launch over the matrices in `descs` (from make_descs).
+    Without `workspace`, split-K scratch (if any) is taken from torch."""
+    if workspace is None:
+        need = workspace_size_batched(descs, M, mode, x_dtype)
+        if need:
+            workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
     wsp = _ptr(workspace) if workspace is not None else None
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib.bc_matmul_q_batched(descs, len(descs), M, bits, group, mode,
