@@ -185,6 +185,35 @@ BC_API size_t bc_workspace_size_batched(const bc_matmul_desc *descs, int count,
                                  int64_t M, bc_mode mode, bc_dtype x_dtype);
 
 /*
+ * bc_matmul_q_noalloc -- the decode matmul (fp32 x, the GEMV path of
+ * bc_matmul_q) for callers that cannot allocate device memory: code that
+ * must not call cudaMalloc (a host callback, a fixed-pool allocator, a
+ * plugin that only receives its input and output pointers) and so cannot
+ * supply bc_matmul_q's workspace.  The paper has no counterpart; this is a
+ * deployment variant of the same computation.
+ *   Arguments mean what they mean for bc_matmul_q with x_dtype = BC_F32.
+ *   Scratch: instead of a caller workspace, the split-K partial sums and
+ *   tickets live in a fixed 4 MiB array inside the library (a __device__
+ *   object that every GPU loading the library holds until process exit).
+ *   Shapes whose scratch would exceed it are rejected with
+ *   BC_ERR_WORKSPACE before anything is enqueued.  The call allocates
+ *   nothing (no cudaMalloc/cudaFree, no allocating library routine).
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture on that device.
+ *   Sharing: all calls share the one array, which keeps the last call's
+ *   contents (the counters that must start at zero are cleared by each
+ *   call).  Calls that can overlap on the GPU -- on different streams, or
+ *   from different threads without ordering -- race on the array and give
+ *   wrong results; serialise them (e.g. one stream).
+ */
+BC_API bc_status bc_matmul_q_noalloc(const void *x, const void *W_or_packed,
+                                     const void *scales, const void *zeros,
+                                     int64_t M, int64_t N, int64_t K, int bits,
+                                     int64_t group, bc_mode mode, float *y,
+                                     bc_stream_t stream);
+
+/*
  * bc_device_timeouts -- number of bounded in-kernel waits (tensor-core
  * pipeline barriers) that ran out on the current device since the library
  * was loaded.  A kernel whose wait runs out stops early, frees its tensor

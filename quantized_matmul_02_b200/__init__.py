@@ -29,7 +29,8 @@ GROUP_PER_CHANNEL = 0
 # Every symbol include/bc.h declares.
 EXPORTS = ("bc_group_params", "bc_quantize_codes", "bc_pack_int4",
            "bc_matmul_q", "bc_workspace_size", "bc_matmul_q_batched",
-           "bc_workspace_size_batched", "bc_device_timeouts",
+           "bc_workspace_size_batched", "bc_matmul_q_noalloc",
+           "bc_device_timeouts",
            "bc_status_string", "bc_version")
 
 
@@ -65,6 +66,9 @@ def _load() -> ctypes.CDLL:
     lib.bc_workspace_size_batched.argtypes = [ctypes.POINTER(MatmulDesc), i32,
                                               i64, i32, i32]
     lib.bc_workspace_size_batched.restype = sz
+    lib.bc_matmul_q_noalloc.argtypes = [P, P, P, P, i64, i64, i64, i32, i64,
+                                        i32, P, P]
+    lib.bc_matmul_q_noalloc.restype = i32
     lib.bc_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     lib.bc_device_timeouts.restype = i32
     lib.bc_status_string.argtypes = [i32]
@@ -203,3 +207,18 @@ def device_timeouts() -> int:
     c = ctypes.c_uint(0)
     _check(lib.bc_device_timeouts(ctypes.byref(c)), "bc_device_timeouts")
     return int(c.value)
+
+
+def matmul_q_noalloc(x: torch.Tensor, W: torch.Tensor,
+                     scales: Optional[torch.Tensor], zeros: Optional[torch.Tensor],
+                     bits: int, group: int, mode: int, y: torch.Tensor,
+                     stream=None) -> torch.Tensor:
+    """bc_matmul_q_noalloc: the fp32-x decode matmul using the library's own
+    fixed scratch instead of a workspace (for callers that cannot allocate).
+    `y` must be supplied; nothing is allocated by this call."""
+    M, K = x.shape
+    N = W.shape[0]
+    _check(lib.bc_matmul_q_noalloc(_ptr(x), _ptr(W), _ptr(scales), _ptr(zeros),
+                                   M, N, K, bits, group, mode, _ptr(y),
+                                   _stream(stream)), "bc_matmul_q_noalloc")
+    return y
