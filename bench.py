@@ -48,7 +48,14 @@ WORKLOADS = {
     "qwen3-8b-int4-decode-m16": ("qwen3-8b", 36, "packed", 4, 64, 16, 4),
     "qwen3-8b-rtn3-decode": ("qwen3-8b", 36, "runtime", 3, 64, 1, 4),
     "qwen3-8b-rtn3-decode-m16": ("qwen3-8b", 36, "runtime", 3, 64, 16, 4),
+    # prefill: bf16 x, packed int4 W, tcgen05 tensor-core GEMM
+    "qwen2.5-0.5b-int4-prefill-m128": ("qwen2.5-0.5b", 24, "packed", 4, 64, 128, 3),
+    "qwen2.5-0.5b-int4-prefill-m2048": ("qwen2.5-0.5b", 24, "packed", 4, 64, 2048, 3),
 }
+
+
+def is_prefill(name: str) -> bool:
+    return WORKLOADS[name][5] >= 64
 DEFAULT_WORKLOAD = "qwen2.5-0.5b-int4-decode"
 
 
@@ -72,7 +79,9 @@ def measured_peaks() -> dict:
 
 def workload_bytes(name: str) -> int:
     shape_set, layers, mode, bits, group, M, _ = WORKLOADS[name]
-    return sum(wl.gemv_bytes(m.K, m.N, M, mode, bits, m.K if group == 0 else group)
+    xb = 2 if is_prefill(name) else 4
+    return sum(wl.gemv_bytes(m.K, m.N, M, mode, bits, m.K if group == 0 else group,
+                             x_bytes_per_elem=xb)
                for m in wl.layer_set(shape_set, layers))
 
 
@@ -81,11 +90,32 @@ def workload_flops(name: str) -> int:
     return sum(2 * M * m.N * m.K for m in wl.layer_set(shape_set, layers))
 
 
-def kernel_source_digest() -> str:
+def launches_per_step(name: str, count: int) -> int:
+    """Kernel launches the library makes for one grouped call (its own
+    chunking of the descriptor list: 80 matrices per tensor-core GEMM
+    launch, 400 per streaming GEMV launch, 368 x 16-row chunks of M for the
+    general GEMV)."""
+    M = WORKLOADS[name][5]
+    if is_prefill(name):
+        return -(-count // 80)
+    if M <= 4:
+        return -(-count // 400)
+    return -(-M // 16) * -(-count // 368)
+
+
+KERNEL_SOURCES = {"decode": ("bc_gemv_stream.cu", "bc_gemv.cu", "bc_internal.cuh"),
+                  "prefill": ("bc_gemm_sm100.cu", "bc_internal.cuh")}
+
+
+def kernel_source_digest(kind: str = "decode") -> str:
+    """Digest of the sources of the kernels a workload runs; a recorded DRAM
+    traffic figure is only reported while it still matches."""
     h = hashlib.sha256()
-    for f in ("bc_gemv.cu", "bc_internal.cuh"):
-        with open(os.path.join(ROOT, "quantized_matmul_02_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    for f in KERNEL_SOURCES[kind]:
+        path = os.path.join(ROOT, "quantized_matmul_02_b200", "csrc", f)
+        if os.path.exists(path):
+            with open(path, "rb") as fh:
+                h.update(fh.read())
     return h.hexdigest()[:16]
 
 
@@ -97,7 +127,8 @@ def recorded_traffic(name: str):
         fields = dict(line.split(":", 1) for line in open(path) if ":" in line)
     except OSError:
         return None
-    if fields.get("source_digest", "").strip() != kernel_source_digest():
+    kind = "prefill" if name in WORKLOADS and is_prefill(name) else "decode"
+    if fields.get("source_digest", "").strip() != kernel_source_digest(kind):
         return None
     try:
         return int(fields["dram_bytes_per_launch"].strip())
@@ -206,8 +237,13 @@ def build_workload(qmm, torch, name: str, copies: int):
         key = (m.layer, m.x_tag)
         if key not in xs_dev:
             xh = wl.activation(seed, m.layer, m.x_tag, M, m.K)
-            xs_host[key] = xh
-            xs_dev[key] = torch.from_numpy(xh).cuda()
+            if is_prefill(name):
+                xh = wl.bf16_bits(xh).view(np.int16)
+                xs_host[key] = xh
+                xs_dev[key] = torch.from_numpy(xh).cuda().view(torch.bfloat16)
+            else:
+                xs_host[key] = xh
+                xs_dev[key] = torch.from_numpy(xh).cuda()
         W = torch.from_numpy(wl.weight(seed, m.layer, m.name, m.K, m.N, sigma)).cuda()
         if mode == "packed":
             s, z = qmm.group_params(W, 4, 64, torch.float16)
@@ -235,6 +271,15 @@ def build_workload(qmm, torch, name: str, copies: int):
             "group": group, "M": M}
 
 
+def _oracle_x(name: str, seed: int, m) -> np.ndarray:
+    """The activation exactly as the GPU path sees it, as fp64."""
+    M = WORKLOADS[name][5]
+    x = wl.activation(seed, m.layer, m.x_tag, M, m.K)
+    if is_prefill(name):
+        x = wl.bf16_to_f32(wl.bf16_bits(x))
+    return x.astype(np.float64)
+
+
 def cpu_baseline_sample(name: str, target_s: float = 12.0):
     """The oracle (as it stands) on a bounded sample of the workload: for
     whole matrices of the first layers, dequantize the codes and multiply
@@ -243,11 +288,11 @@ def cpu_baseline_sample(name: str, target_s: float = 12.0):
     shape_set, layers, mode, bits, group, M, seed = WORKLOADS[name]
     mats = wl.layer_set(shape_set, layers)
     sigma = wl.SIGMA[shape_set]
-    done_bytes, spent = 0, 0.0
+    done_bytes, done_flops, spent = 0, 0, 0.0
     done = 0
     for m in mats:
         W = wl.weight(seed, m.layer, m.name, m.K, m.N, sigma)
-        x = wl.activation(seed, m.layer, m.x_tag, M, m.K).astype(np.float64)
+        x = _oracle_x(name, seed, m)
         g = m.K if group == 0 else group
         if mode == "runtime" and bits == 16:
             t0 = time.perf_counter()
@@ -262,11 +307,17 @@ def cpu_baseline_sample(name: str, target_s: float = 12.0):
                 q = oracle.codes(W, s, z, bits, g)
             oracle.matmul(x, oracle.dequant(q, s, z, g))
             spent += time.perf_counter() - t0
-        done_bytes += wl.gemv_bytes(m.K, m.N, M, mode, bits, g)
+        done_bytes += wl.gemv_bytes(m.K, m.N, M, mode, bits, g,
+                                    x_bytes_per_elem=2 if is_prefill(name) else 4)
+        done_flops += 2 * M * m.N * m.K
         done += 1
         if spent >= target_s:
             break
-    return {"value": done_bytes / spent / 1e9, "unit": "GB/s",
+    if is_prefill(name):
+        value, unit = done_flops / spent / 1e12, "TFLOP/s"
+    else:
+        value, unit = done_bytes / spent / 1e9, "GB/s"
+    return {"value": value, "unit": unit,
             "cores": oracle.threads(), "kind": "oracle",
             "sample": f"{done} of {len(mats)} matrices of {name} (first layers), "
                       f"fp64 dequant + matmul, {spent:.1f} s"}
@@ -285,7 +336,7 @@ def _reference_sample(name: str, rows: int):
     for m in wl.layer_set(shape_set, 1):
         n = min(rows, m.N)
         W = wl.weight(seed, m.layer, m.name, m.K, m.N, wl.SIGMA[shape_set])[:n]
-        x = wl.activation(seed, m.layer, m.x_tag, M, m.K).astype(np.float64)
+        x = _oracle_x(name, seed, m)
         g = m.K if group == 0 else group
         item = {"W": W, "x": x, "g": g,
                 "bytes": wl.gemv_bytes(m.K, n, M, mode, bits, g)}
@@ -371,13 +422,15 @@ def run_ours(args, rank, world, local_rank):
     copies = min(copies, 8)
     W = build_workload(qmm, torch, name, copies)
     mode_id = qmm.BC_MODE_PACKED_INT4 if mode == "packed" else qmm.BC_MODE_RUNTIME
-    ws_bytes = max(qmm.workspace_size_batched(d, M, mode_id, qmm.BC_F32) for d in W["descs"])
+    prefill = is_prefill(name)
+    x_dtype = qmm.BC_BF16 if prefill else qmm.BC_F32
+    ws_bytes = max(qmm.workspace_size_batched(d, M, mode_id, x_dtype) for d in W["descs"])
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step(i):
         qmm.matmul_q_batched(W["descs"][i % copies], M, bits, group, mode_id,
-                             workspace=ws)
+                             x_dtype=x_dtype, workspace=ws)
 
     for i in range(args.warmup):
         step(i)
@@ -413,13 +466,19 @@ def run_ours(args, rank, world, local_rank):
         t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         times = [float(t.item())]
-    agg = aggregate_times(times, world, step_bytes * args.steps / 1e9)
+    step_flops = workload_flops(name)
+    # units of the metric per step: GB (decode GEMV) or TFLOP (prefill GEMM)
+    step_units = step_flops / 1e12 if prefill else step_bytes / 1e9
+    unit = "TFLOP/s" if prefill else "GB/s"
+    agg = aggregate_times(times, world, step_units * args.steps)
     ms_per_step = agg["ms"] / args.steps
 
     # ---- end to end through the public API: pinned host x in, y out ----
     xs_pinned = {k: torch.from_numpy(v).pin_memory() for k, v in W["xs_host"].items()}
+    if prefill:
+        xs_pinned = {k: v.view(torch.bfloat16) for k, v in xs_pinned.items()}
     ys_pinned = [torch.empty(y.shape, dtype=torch.float32).pin_memory() for y in W["ys"]]
-    h2d = sum(v.numel() * 4 for v in xs_pinned.values())
+    h2d = sum(v.numel() * v.element_size() for v in xs_pinned.values())
     d2h = sum(y.numel() * 4 for y in ys_pinned)
 
     def e2e_step(i):
@@ -447,7 +506,7 @@ def run_ours(args, rank, world, local_rank):
         t = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e_ms = float(t.item())
-    e2e_value = step_bytes * e_steps * world / (e_ms / 1e3) / 1e9
+    e2e_value = step_units * e_steps * world / (e_ms / 1e3)
 
     if dist:
         dist.barrier()
@@ -457,34 +516,52 @@ def run_ours(args, rank, world, local_rank):
 
     peaks = measured_peaks()
     avg_launch_ms = float(np.mean(launch_ms))
-    achieved = step_bytes / (avg_launch_ms / 1e3) / 1e9
     traffic = recorded_traffic(name)
+    if prefill:
+        achieved = step_flops / (avg_launch_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops_sustained"],
+                "traffic": traffic,
+                "peak_source": f"{peaks['source']} dense bf16, sustained "
+                               "(MEASURED_PEAKS.json bf16_tflops_sustained); "
+                               f"burst {peaks['bf16_tflops']}",
+                "frac_of_burst": achieved / peaks["bf16_tflops"],
+                "hbm_gbs_achieved": step_bytes / (avg_launch_ms / 1e3) / 1e9,
+                "kernel": "gemm_packed_kernel (bc_gemm_sm100.cu)",
+                "avg_step_us": avg_launch_ms * 1e3}
+    else:
+        achieved = step_bytes / (avg_launch_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "traffic": traffic,
+                "peak_source": f"{peaks['source']} copy bandwidth "
+                               "(MEASURED_PEAKS.json hbm_gbs)",
+                "kernel": "gemv_stream_kernel (bc_gemv_stream.cu)" if M <= 4
+                          else "gemv_kernel (bc_gemv.cu)",
+                "avg_step_us": avg_launch_ms * 1e3}
     line = {
-        "metric": METRIC, "value": agg["value"], "unit": "GB/s",
+        "metric": METRIC, "value": agg["value"], "unit": unit,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16" if prefill else "f32",
+        "data": "synthetic",
         "config": {"workload": name, "shape_set": shape_set, "layers": layers,
                    "matrices": len(W["mats"]), "mode": mode, "bits": bits,
                    "group": group if group else "per-channel", "M": M,
                    "weights": "int4 packed, fp16 scale/zero per 64-block"
                    if mode == "packed" else "fp16, runtime RTN",
-                   "x": "fp32", "bytes_per_step": step_bytes,
+                   "x": "bf16" if prefill else "fp32", "bytes_per_step": step_bytes,
+                   "flops_per_step": step_flops,
                    "l2": f"inputs larger than L2: {copies} weight copies "
                          f"({copies * step_bytes / 1e6:.0f} MB) rotated between "
                          f"steps, L2 {l2 / 1e6:.0f} MB",
                    "launch": "one grouped launch per step"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": traffic,
-                     "peak_source": f"{peaks['source']} copy bandwidth "
-                                    "(MEASURED_PEAKS.json hbm_gbs)",
-                     "kernel": "gemv_kernel (bc_gemv.cu)",
-                     "avg_launch_us": avg_launch_ms * 1e3},
-        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": e_ms / e_steps, "steps": e_steps},
-        "gpu_launches": args.steps * ((M + 15) // 16) * ((len(W["mats"]) + 367) // 368),
+        "gpu_launches": args.steps * launches_per_step(name, len(W["mats"])),
         "clocks": sampler.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -116,9 +116,9 @@ int bc_version(void) { return 100; }
 bc_status bc_device_timeouts(unsigned *count) {
     if (!count) return BC_ERR_INVALID_ARG;
     if (cudaDeviceSynchronize() != cudaSuccess) return BC_ERR_CUDA;
-    const unsigned v = gemm_timeouts();
-    if (v == ~0u) return BC_ERR_CUDA;
-    *count = v;
+    const unsigned a = gemm_timeouts(), b = gemv_timeouts();
+    if (a == ~0u || b == ~0u) return BC_ERR_CUDA;
+    *count = a + b;
     return BC_OK;
 }
 

@@ -73,7 +73,7 @@ template <int BNX> struct Cfg {
     static constexpr int kStageBytes = kABytes + kBBytes + kCBytes;
     static constexpr int kStages = BNX == 256 ? 4 : 6;
     static constexpr int kTmemCols = 2 * BNX;
-    static constexpr int kBarBytes = 1024;
+    static constexpr int kBarBytes = 4096;     // barriers + job table copy
     static constexpr int kSmem = kStages * kStageBytes + kBarBytes + 1024;
     // instruction descriptor: D f32, A/B bf16, K-major both, N, M = 128
     static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
@@ -216,14 +216,66 @@ __device__ __noinline__ uint4 dequant8_wide(uint32_t w, float z, float s) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-__device__ __forceinline__ int find_job(const GemmParams &P, int tile) {
-    int lo = 0, hi = P.count - 1;
+// Job descriptors are read from a shared-memory copy (sjobs): dynamically
+// indexed reads of the parameter block miss the constant cache.
+__device__ __forceinline__ int find_job(const GemmJobDev *jobs, int count, int tile) {
+    int lo = 0, hi = count - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (P.jobs[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
+        if (jobs[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
     }
     return lo;
 }
+
+constexpr int kLook = 4;     // scale/zero look-ahead, in 64-blocks of K
+
+// Walks the (tile, 64-block) sequence a dequant thread consumes and loads
+// the scale/zero of its weight row for each position.
+struct SzCursor {
+    int tile, kb, kblocks;
+    const __half *srow, *zrow;
+    const GemmJobDev *jobs;
+    __device__ __forceinline__ void bind(const GemmParams &P, int r) {
+        if (tile >= P.total_tiles) {
+            srow = zrow = nullptr;
+            kblocks = 1;
+            return;
+        }
+        const GemmJobDev &J = jobs[find_job(jobs, P.count, tile)];
+        const int nb = (tile - J.tile_begin) / J.xblocks;
+        const int row = nb * kBM + r;
+        kblocks = J.K / kBK;
+        if (row < J.N) {
+            srow = J.s + (int64_t)row * kblocks;
+            zrow = J.z + (int64_t)row * kblocks;
+        } else {
+            srow = zrow = nullptr;
+        }
+    }
+    __device__ __forceinline__ void init(const GemmParams &P, const GemmJobDev *sj,
+                                         int first, int, int r) {
+        jobs = sj;
+        tile = first;
+        kb = 0;
+        bind(P, r);
+    }
+    __device__ __forceinline__ void advance(const GemmParams &P, int stride, int r) {
+        if (++kb == kblocks) {
+            kb = 0;
+            tile += stride;
+            bind(P, r);
+        }
+    }
+    __device__ __forceinline__ void load(float &s, float &z) const {
+        if (srow) {
+            s = __half2float(__ldg(srow + kb));
+            z = __half2float(__ldg(zrow + kb));
+        } else {
+            s = 0.0f;
+            z = 0.0f;
+        }
+    }
+};
 
 template <int BNX>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -241,6 +293,13 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
     uint64_t *mma_done = acc_empty + 2;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(mma_done + 1);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1) + 1;
+    GemmJobDev *sjobs = reinterpret_cast<GemmJobDev *>(mma_done + 2);
+    {
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(P.jobs);
+        uint32_t *dst = reinterpret_cast<uint32_t *>(sjobs);
+        const int words = P.count * (int)(sizeof(GemmJobDev) / 4);
+        for (int i = threadIdx.x; i < words; i += kThreads) dst[i] = src[i];
+    }
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -276,8 +335,8 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
             uint32_t armed = 0;                   // stages with a load issued
             for (int tile = blockIdx.x; tile < P.total_tiles && !*abort_flag;
                  tile += gridDim.x) {
-                const int j = find_job(P, tile);
-                const GemmJobDev &J = P.jobs[j];
+                const int j = find_job(sjobs, P.count, tile);
+                const GemmJobDev &J = sjobs[j];
                 const int local = tile - J.tile_begin;
                 const int nb = local / J.xblocks, xb = local % J.xblocks;
                 const int kblocks = J.K / kBK;
@@ -316,8 +375,8 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
             int lt = 0;
             for (int tile = blockIdx.x; tile < P.total_tiles && !*abort_flag;
                  tile += gridDim.x, ++lt) {
-                const int j = find_job(P, tile);
-                const int kblocks = P.jobs[j].K / kBK;
+                const int j = find_job(sjobs, P.count, tile);
+                const int kblocks = sjobs[j].K / kBK;
                 const int buf = lt & 1;
                 const uint32_t aph = (lt >> 1) & 1;
                 if (!mbar_wait(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag)) break;
@@ -353,27 +412,42 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
             }
         }
     } else if (warp < kDqWarp0 + kDqWarps) {
-        // dequant: thread -> (row r, half h) of the 128 x 64 weight tile
+        // dequant: thread -> (row r, half h) of the 128 x 64 weight tile.
+        // Scale/zero come from global memory.  They are fetched kLook blocks
+        // ahead into a window of kLook register slots indexed at compile
+        // time (slot j serves blocks g with g % kLook == j), so no register
+        // copy waits on a load that is still in flight.
         const int t = threadIdx.x - 32 * kDqWarp0;
         const int r = t & (kBM - 1), h = t >> 7;
+        SzCursor la;                        // look-ahead cursor
+        la.init(P, sjobs, blockIdx.x, gridDim.x, r);
+        float sq[kLook], zq[kLook];
+#pragma unroll
+        for (int i = 0; i < kLook; ++i) {
+            la.load(sq[i], zq[i]);
+            la.advance(P, gridDim.x, r);
+        }
+        int tile = blockIdx.x, kb = 0, kblocks = 1;
+        bool valid = false;
+        auto bind = [&]() {
+            if (tile >= P.total_tiles) return;
+            const GemmJobDev &J = sjobs[find_job(sjobs, P.count, tile)];
+            const int nb = (tile - J.tile_begin) / J.xblocks;
+            kblocks = J.K / kBK;
+            valid = nb * kBM + r < J.N;
+        };
+        bind();
         uint32_t g = 0;
-        for (int tile = blockIdx.x; tile < P.total_tiles && !*abort_flag;
-             tile += gridDim.x) {
-            const int j = find_job(P, tile);
-            const GemmJobDev &J = P.jobs[j];
-            const int local = tile - J.tile_begin;
-            const int nb = local / J.xblocks;
-            const int row = nb * kBM + r;
-            const int kblocks = J.K / kBK;
-            const bool valid = row < J.N;
-            const __half *srow = J.s + (int64_t)(valid ? row : 0) * kblocks;
-            const __half *zrow = J.z + (int64_t)(valid ? row : 0) * kblocks;
-            bool ok = true;
-            for (int kb = 0; kb < kblocks; ++kb, ++g) {
+        bool ok = true;
+        while (ok && tile < P.total_tiles && !*abort_flag) {
+#pragma unroll
+            for (int j = 0; j < kLook; ++j) {
+                if (tile >= P.total_tiles) break;
+                const float sf = sq[j], zf = zq[j];
+                la.load(sq[j], zq[j]);             // refill slot j, kLook ahead
+                la.advance(P, gridDim.x, r);
                 const int s = g % C::kStages;
                 const uint32_t ph = (g / C::kStages) & 1;
-                const float sf = __half2float(__ldg(srow + kb));
-                const float zf = __half2float(__ldg(zrow + kb));
                 if (!mbar_wait(smem_u32(&full_tma[s]), ph, abort_flag)) {
                     ok = false;
                     break;
@@ -412,8 +486,13 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&full_dq[s]));
+                ++g;
+                if (++kb == kblocks) {
+                    kb = 0;
+                    tile += gridDim.x;
+                    bind();
+                }
             }
-            if (!ok) break;
         }
     } else {
         // epilogue: warp quarter q reads TMEM lanes 32q..32q+31 (weight rows)
@@ -421,8 +500,8 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
         int lt = 0;
         for (int tile = blockIdx.x; tile < P.total_tiles && !*abort_flag;
              tile += gridDim.x, ++lt) {
-            const int j = find_job(P, tile);
-            const GemmJobDev &J = P.jobs[j];
+            const int j = find_job(sjobs, P.count, tile);
+            const GemmJobDev &J = sjobs[j];
             const int local = tile - J.tile_begin;
             const int nb = local / J.xblocks, xb = local % J.xblocks;
             const int buf = lt & 1;

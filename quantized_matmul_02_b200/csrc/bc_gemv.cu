@@ -361,10 +361,23 @@ bc_status launch_mt(const GemvParams &P, int mt, int grid, cudaStream_t s) {
     return cuda_status();
 }
 
+// Whole launches with at least half an SM's worth of 128-row units per SM
+// go to the streaming kernel; lone small matrices keep the split-K GEMV.
+bool use_stream(const GemvJob *jobs, int count, int M, bool packed,
+                const DeviceInfo &di) {
+    if (M > 4) return false;
+    int64_t units = 0;
+    for (int i = 0; i < count; ++i) units += (jobs[i].N + 127) / 128;
+    if (units < di.sm_count / 2) return false;
+    return gemv_stream_supported(jobs, count, M, packed, di.max_smem_optin);
+}
+
 }  // namespace
 
 size_t gemv_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed,
                             int sm_count) {
+    DeviceInfo di;
+    if (device_info(&di) && use_stream(jobs, count, M, packed, di)) return 0;
     size_t worst = 0;
     for (int b = 0; b < count; b += kMaxJobs) {
         const int n = std::min(kMaxJobs, count - b);
@@ -379,6 +392,8 @@ bc_status launch_gemv(const GemvJob *jobs, int count, int M, int bits,
                       cudaStream_t s) {
     DeviceInfo di;
     if (!device_info(&di)) return BC_ERR_CUDA;
+    if (use_stream(jobs, count, M, packed, di))
+        return launch_gemv_stream(jobs, count, M, bits, packed, s);
     // ~32 KB of kernel parameters, kept off the stack; the launch copies it.
     thread_local GemvParams *Pp = nullptr;
     if (!Pp) Pp = new GemvParams();

@@ -56,6 +56,13 @@ struct GemvJob {             // one matrix of a launch
     int64_t N, K;
     int64_t group;           // 64 or K
 };
+// Streaming GEMV (bc_gemv_stream.cu): M <= 4, bulk-copy ring, mma.sync
+// unpack for packed codes.  Used for launches large enough to fill the GPU.
+bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed,
+                           int max_smem);
+bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
+                             bool packed, cudaStream_t s);
+unsigned gemv_timeouts();
 // Bytes of split-K scratch a launch over these jobs needs.
 size_t gemv_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed,
                             int sm_count);

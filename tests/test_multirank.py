@@ -84,10 +84,11 @@ def test_traffic_needs_matching_digest(tmp_path, monkeypatch):
     csrc = tmp_path / "quantized_matmul_02_b200" / "csrc"
     os.makedirs(csrc)
     (csrc / "bc_gemv.cu").write_text("a")
+    (csrc / "bc_gemv_stream.cu").write_text("c")
     (csrc / "bc_internal.cuh").write_text("b")
     d = bench.kernel_source_digest()
     f = tmp_path / "profiles" / "traffic_w.txt"
     f.write_text(f"source_digest: {d}\ndram_bytes_per_launch: 123\n")
     assert bench.recorded_traffic("w") == 123
-    (csrc / "bc_gemv.cu").write_text("changed")
+    (csrc / "bc_gemv_stream.cu").write_text("changed")
     assert bench.recorded_traffic("w") is None

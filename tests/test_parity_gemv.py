@@ -209,3 +209,48 @@ def test_determinism_batched(cuda_lib):
         outs.append(torch.cat([it[4].flatten() for it in items]).cpu())
     for o in outs[1:]:
         assert torch.equal(o, outs[0])
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("mode,bits,group", [("packed", 4, 64), ("runtime", 5, 64),
+                                             ("runtime", 3, 0), ("runtime", 16, 64)])
+def test_batched_mixed_shapes_stream(cuda_lib, M, mode, bits, group):
+    """A grouped launch large enough for the streaming kernel, with ragged
+    row blocks (N not a multiple of 128) and K tails (K not a multiple of
+    the 256-byte stage chunk), several matrices sharing one x."""
+    rng = np.random.default_rng(M * 10 + bits)
+    shapes = [(37, 192), (200, 896), (896, 1024), (130, 64), (256, 4864),
+              (1000, 320)]
+    items, refs = [], []
+    xs = {}
+    for i in range(36):
+        N, K = shapes[i % len(shapes)]
+        key = (K, i // 12)
+        if key not in xs:
+            xs[key] = wl.activation(50 + i // 12, K, "x", M, K)
+        x = xs[key]
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+        g = K if group == 0 else group
+        Wd = dev(W)
+        if mode == "packed":
+            s, z = cuda_lib.group_params(Wd, 4, 64, torch.float16)
+            Wk = cuda_lib.pack_int4(Wd, s, z)
+            ref = oracle.matmul_q(x, W, 4, 64, "packed")
+        elif bits == 16:
+            s = z = None
+            Wk = Wd
+            ref = oracle.matmul_q(x, W, 16, g, "runtime")
+        else:
+            s, z = cuda_lib.group_params(Wd, bits, group, torch.float32)
+            Wk = Wd
+            ref = oracle.matmul_q(x, W, bits, g, "runtime")
+        y = torch.full((M, N), float("nan"), device="cuda")
+        items.append((dev(x), Wk, s, z, y))
+        refs.append(ref)
+    descs = cuda_lib.make_descs(items)
+    mid = cuda_lib.BC_MODE_PACKED_INT4 if mode == "packed" else cuda_lib.BC_MODE_RUNTIME
+    cuda_lib.matmul_q_batched(descs, M, bits, group, mid)
+    torch.cuda.synchronize()
+    for i, (ref, it) in enumerate(zip(refs, items)):
+        assert_close(host(it[4]), ref["y"], ref["A"], TOL_FP32, f"matrix {i}")
+    assert cuda_lib.device_timeouts() == 0

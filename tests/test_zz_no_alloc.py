@@ -45,7 +45,7 @@ def _noalloc_vs_workspace(qmm, c):
 
 
 def test_noalloc_matches_workspace_entry_two_calls_in_a_row(cuda_lib):
-    a = _case(cuda_lib, "packed", 1, 128, 4864, 4, 64, 0)
+    a = _case(cuda_lib, "packed", 8, 128, 4864, 4, 64, 0)
     b = _case(cuda_lib, "runtime", 5, 256, 3072, 3, 64, 1)
     _noalloc_vs_workspace(cuda_lib, a)     # first call: sets the scratch up
     _noalloc_vs_workspace(cuda_lib, b)     # second call reuses the scratch
