@@ -2,34 +2,41 @@
 //
 // Decode "reads every weight in the model to write one word" (Enargeia):
 // the matmul is one pass over HBM.  The kernel is a TMA pipeline that keeps
-// ~160 KB per SM in flight, with the arithmetic kept well under the SM's
-// issue budget so that the stream, not the ALUs, sets the pace.
+// ~130-200 KB per SM in flight, with the arithmetic per weight cut down until
+// the stream, not the issue slots, sets the pace.
 //
 // One CTA per SM, persistent over a byte-balanced contiguous range of
 // "units" (128 weight rows of one matrix) that spans every matrix of a
 // grouped launch (Enargeia, "One decode step": hundreds of passes per token
 // are one launch here).  Warp roles:
-//   warp 0      TMA producer: each stage is a 256-byte column chunk of the
-//               unit's 128 rows, loaded as two 2D boxes of 128 rows x 128
-//               bytes with the 128-byte swizzle (ring of up to 6 stages,
-//               full/empty mbarriers);
+//   warp 0      loader: lane 0 issues the TMA of each stage (a 256-byte column
+//               chunk of the unit's 128 rows as two 2D boxes of 128 rows x
+//               128 bytes, 128-byte swizzle) into a ring of up to 6 stages with
+//               full/empty mbarriers.
 //   warp 1      activation stager: the x of each new matrix goes into one of
-//               two smem slots -- fp32 rows (runtime mode), or fp16 hi + lo
-//               pieces (x = hi + lo to 2^-22) in mma.sync fragment order
-//               plus per-64-group sums of the even-k and odd-k pieces
-//               (packed mode);
+//               two smem slots (see below); the first slot is filled by every
+//               warp but the loader together before streaming starts.
 //   warps 2-17  consumers: warp (window w, row group g) handles 16 rows and
 //               the w-th 128-byte window of every stage; the two windows'
-//               partial row sums meet in smem at the end of each unit.
+//               partial row sums meet in smem at the end of each unit.  Each
+//               lane loads its own fp16 scales and zeros from global memory two
+//               stages ahead (small scattered copies cost the loader more issue
+//               time than the stage itself).
 //
-// Packed int4 (Enargeia, "Four bits per weight": codes unpacked in
-// registers, never written back).  Two shifts and four LOP3 turn 8 nibbles
-// into exact fp16 pairs (256 + q) for even k and (16 + q) for odd k, which
-// feed mma.sync.m16n8k16 A fragments straight from registers.  B holds the
-// x pieces of the window's four 64-groups block-diagonally (8 columns = 4
-// groups x {hi, lo}), so every group's dot product lands in its own column:
-//     sum_k x_k (q_k - z) = C_hi + C_lo - (256 + z) X_even - (16 + z) X_odd
-// then one multiply by the group's scale.  About one instruction per weight.
+// Packed int4 (Enargeia, "Four bits per weight": codes unpacked in registers,
+// never written back) runs on the int8 tensor cores (mma.sync m16n8k32
+// u8 x s8 -> s32).  ldmatrix brings the swizzled stage into A fragments; one
+// AND per register gives the even-k codes (q) and one the odd-k codes (16 q)
+// as unsigned bytes.  The activations are staged as integers per 64-group,
+//     x_k ~= X_k * 2^(E_g - 27),  X_k = rint(x_k 2^(27 - E_g)) (even k),
+//                                 X_k = 16 rint(x_k 2^(23 - E_g)) (odd k),
+// with max|x| < 2^E_g over the group, each split into four balanced int8
+// digits (X = d0 + 2^8 d1 + 2^16 d2 + 2^24 d3) that fill the 8 columns of B.
+// With one x row the columns hold 2 groups x 4 digits, the k slots of each
+// mma split between the two groups (block diagonal); with several x rows
+// they hold 2 rows x 4 digits.  The integer dot products are exact, so
+//     y = sum_g s_g ( 2^(E_g-27) sum_d 2^(8d) C_gd - z_g sum_k x_k~ )
+// carries only the rounding of x to 23-27 bits and of the fp32 epilogue.
 //
 // Runtime RTN (BITCRUSH BC-06, "Under the hood": codes computed inline as
 // weights are read) runs on the CUDA cores, four threads per row, with the
@@ -57,11 +64,12 @@ constexpr int kChunk = 256;             // bytes of a row per stage
 constexpr int kBoxBytes = kRows * 128;  // one TMA box: 128 rows x 128 bytes, SW128
 constexpr int kStageBytes = 2 * kBoxBytes;
 constexpr int kConsumers = 16;
+constexpr int kStagers = 1 + kConsumers;   // warps that fill the first x slot
 constexpr int kThreads = 32 * (2 + kConsumers);
 constexpr int kMaxJobs = 168;
 constexpr int kMaxCtas = 160;
 constexpr int kMaxM = 4;
-constexpr int kPiecePad = 32;           // bytes between the hi and lo pieces
+constexpr int kXP = 23;                 // bits of the odd-k activation integers
 constexpr long long kWaitCycles = 4000000000LL;
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
 
@@ -93,11 +101,14 @@ template <bool PACKED> __host__ __device__ __forceinline__ int kchunks_of(int K)
 template <bool PACKED> __host__ __device__ __forceinline__ int kpad_of(int K) {
     return kchunks_of<PACKED>(K) * (PACKED ? 2 * kChunk : kChunk / 2);
 }
-// Bytes of one x row in a slot.  Packed: hi[kp] f16, pad, lo[kp] f16,
-// sums[kp/64] x {even, odd} f32.  Runtime: x[kp] f32.
+// Packed x row: digit words [digit d][lane t][unit U][parity] with a row
+// stride of dig_rs words (= 4 mod 32, so the 8 rows a quarter-warp reads sit
+// in distinct banks), then [parity][group] float2 (f, X~) tables.
+__host__ __device__ __forceinline__ int dig_rs(int kchunks) { return 32 * kchunks + 4; }
+// Bytes of one x row in a slot.  Runtime: x[kp] f32.
 template <bool PACKED> __host__ __device__ __forceinline__ int xrow_bytes(int K) {
-    const int kp = kpad_of<PACKED>(K);
-    return PACKED ? 4 * kp + kPiecePad + (kp / 64) * 8 : 4 * kp;
+    const int kc = kchunks_of<PACKED>(K);
+    return PACKED ? 64 * dig_rs(kc) + 16 * (8 * kc) : 4 * kpad_of<false>(K);
 }
 
 // ---- PTX helpers -------------------------------------------------------------
@@ -137,45 +148,46 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
         }
     }
 }
+// Weights are read once: their lines go first when L2 needs room, which keeps
+// the activations, scales and zeros (read by many CTAs or stages) resident.
+__device__ __forceinline__ uint64_t evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map,
-                                            int x, int y, uint32_t bar) {
+                                            int x, int y, uint32_t bar, uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
         : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 __device__ __forceinline__ void named_bar(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
-// Byte offset of 16-byte unit `u` of row `r` inside a 128B-swizzled box.
-__device__ __forceinline__ int sw_off(int r, int u) {
-    return r * 128 + ((u ^ (r & 7)) << 4);
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
 }
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1,
-                                         uint32_t a2, uint32_t a3, uint32_t b0,
-                                         uint32_t b1) {
+// C (16x8 s32) += A (16x32 u8) * B (32x8 s8)
+__device__ __forceinline__ void mma_i8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                       uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// (t & mask) | bias: fp16 pairs built from nibbles already at mantissa bits.
-template <uint32_t MASK, uint32_t BIAS>
-__device__ __forceinline__ uint32_t lop_or(uint32_t t) {
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(t), "n"(MASK), "n"(BIAS));
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
     return r;
-}
-// 8 packed codes (nibble j = k_j) -> fp16 pairs R_j = (k_j, k_{j+4}):
-// even j as 256 + q (mantissa bits 2-5), odd j as 16 + q (bits 6-9).
-__device__ __forceinline__ void unpack8(uint32_t w, uint32_t (&R)[4]) {
-    const uint32_t t0 = w << 2, t1 = w >> 6;
-    R[0] = lop_or<0x003C003Cu, 0x5C005C00u>(t0);
-    R[1] = lop_or<0x03C003C0u, 0x4C004C00u>(t0);
-    R[2] = lop_or<0x003C003Cu, 0x5C005C00u>(t1);
-    R[3] = lop_or<0x03C003C0u, 0x4C004C00u>(t1);
 }
 __device__ __forceinline__ float rcp_approx(float s) {
     float r;
@@ -187,6 +199,11 @@ __device__ __noinline__ float centered_code_exact(float w, float s, float z,
     double q = rint((double)w / (double)s) + (double)z;
     q = fmin(fmax(q, 0.0), (double)L);
     return (float)(q - (double)z);
+}
+__device__ __forceinline__ float2 half2_bits_to_float2(uint32_t v) {
+    __half2 h;
+    *reinterpret_cast<uint32_t *>(&h) = v;
+    return __half22float2(h);
 }
 
 // The job table is copied into shared memory at kernel start: dynamically
@@ -203,6 +220,129 @@ __device__ __forceinline__ int find_job(const StreamJob *jobs, int count, int un
 __device__ __forceinline__ int next_job(const StreamJob *jobs, int count, int j, int unit) {
     while (j + 1 < count && jobs[j + 1].unit_begin <= unit) ++j;
     return j;
+}
+
+// ---- activation staging ------------------------------------------------------
+// Four balanced int8 digits of v (|v| < 2^31 - 2^23) as the bytes of one word:
+// adding 0x80 to each low byte turns the digits into unsigned bytes.
+__device__ __forceinline__ uint32_t digits4(int v) {
+    return ((uint32_t)v + 0x00808080u) ^ 0x00808080u;
+}
+// Byte transpose: out[d] = byte d of w[0..3].
+__device__ __forceinline__ void transpose4(const uint32_t (&w)[4], uint32_t (&o)[4]) {
+    const uint32_t t0 = prmt(w[0], w[1], 0x5140), t1 = prmt(w[0], w[1], 0x7362);
+    const uint32_t t2 = prmt(w[2], w[3], 0x5140), t3 = prmt(w[2], w[3], 0x7362);
+    o[0] = prmt(t0, t2, 0x5410);
+    o[1] = prmt(t0, t2, 0x7632);
+    o[2] = prmt(t1, t3, 0x5410);
+    o[3] = prmt(t1, t3, 0x7632);
+}
+
+// One x row of a packed-mode slot, by warp `widx` of `nw` working together.
+// Eight lanes per 64-group, each with 8 consecutive k (one 32-k unit half).
+__device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
+                               int widx, int nw, int lane) {
+    const int kch = kchunks_of<true>(K);
+    const int rs = dig_rs(kch);
+    const int gpad = 8 * kch, G = K >> 6;
+    uint32_t *dig = reinterpret_cast<uint32_t *>(xm);
+    float2 *tab = reinterpret_cast<float2 *>(xm + 64 * rs);
+    const int j = lane & 7;
+    const int nq = gpad / 4;
+    constexpr int kBatch = 4;
+    for (int q0 = widx; q0 < nq; q0 += nw * kBatch) {
+        float4 va[kBatch][2];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int g = 4 * (q0 + b * nw) + (lane >> 3);
+            va[b][0] = va[b][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (q0 + b * nw < nq && g < G) {
+                const float4 *p = reinterpret_cast<const float4 *>(xr + 64 * g + 8 * j);
+                va[b][0] = __ldg(p);
+                va[b][1] = __ldg(p + 1);
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            if (q0 + b * nw >= nq) break;
+            const int g = 4 * (q0 + b * nw) + (lane >> 3);
+            const float v[8] = {va[b][0].x, va[b][0].y, va[b][0].z, va[b][0].w,
+                                va[b][1].x, va[b][1].y, va[b][1].z, va[b][1].w};
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+            // max|x| < 2^E; E >= -96 keeps every scale below a normal float
+            int E = amax > 0.0f ? (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126 : 0;
+            E = max(E, -96);
+            const float sc_e = __uint_as_float((uint32_t)(127 + kXP + 4 - E) << 23);
+            const float sc_o = __uint_as_float((uint32_t)(127 + kXP - E) << 23);
+            uint32_t de[4], dq[4];
+            int sum = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int xe = __float2int_rn(v[2 * i] * sc_e);      // |xe| <= 2^27
+                const int xo = __float2int_rn(v[2 * i + 1] * sc_o);  // |xo| <= 2^23
+                sum += xe + 16 * xo;
+                de[i] = digits4(xe);
+                dq[i] = digits4(xo);
+            }
+            uint32_t te[4], to[4];
+            transpose4(de, te);
+            transpose4(dq, to);
+            const int U = 2 * g + (j >> 2), tt = j & 3;
+#pragma unroll
+            for (int d = 0; d < 4; ++d)
+                *reinterpret_cast<uint2 *>(dig + (d * 4 + tt) * rs + 2 * U) =
+                    make_uint2(te[d], to[d]);
+            float fs = (float)sum;
+            fs += __shfl_xor_sync(0xffffffffu, fs, 1);
+            fs += __shfl_xor_sync(0xffffffffu, fs, 2);
+            fs += __shfl_xor_sync(0xffffffffu, fs, 4);
+            if (j == 0) {
+                const float f = __uint_as_float((uint32_t)(127 + E - kXP - 4) << 23);
+                tab[g] = make_float2(f, f * fs);
+                tab[gpad + g] = make_float2(f * 65536.0f, 0.0f);
+            }
+        }
+    }
+}
+
+// One x row of a runtime-mode slot: fp32, zero past K.
+__device__ void stage_x_runtime(const float *__restrict__ xr, int K, uint8_t *xm,
+                                int widx, int nw, int lane) {
+    float *xf = reinterpret_cast<float *>(xm);
+    const int kp = kpad_of<false>(K);
+    constexpr int kBatch = 8;
+    const int step = 128 * nw;
+    for (int k0 = 128 * widx + 4 * lane; k0 < kp; k0 += step * kBatch) {
+        float4 v[kBatch];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int k = k0 + step * q;
+            v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (k < K) v[q] = __ldg(reinterpret_cast<const float4 *>(xr + k));
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int k = k0 + step * q;
+            if (k < kp) *reinterpret_cast<float4 *>(xf + k) = v[q];
+        }
+    }
+}
+
+template <bool PACKED>
+__device__ __forceinline__ void stage_x(const StreamJob &J, int M, uint8_t *xs,
+                                        int widx, int nw, int lane) {
+    const int mb = xrow_bytes<PACKED>(J.K);
+    for (int m = 0; m < M; ++m) {
+        if constexpr (PACKED)
+            stage_x_packed(J.x + (int64_t)m * J.K, J.K, xs + m * mb, widx, nw, lane);
+        else
+            stage_x_runtime(J.x + (int64_t)m * J.K, J.K, xs + m * mb, widx, nw, lane);
+    }
 }
 
 // The consumer's activation slot; it moves on at a unit whose matrix reads
@@ -229,188 +369,425 @@ __device__ __forceinline__ bool x_enter(XCursor &c, const StreamJob &J, bool fir
 }
 
 // Cross-window sums: the window-1 warp of a row group hands its 16 row
-// partials to the window-0 warp through smem (double-buffered by unit).
+// partials to the window-0 warp through smem, double-buffered by unit, with
+// an mbarrier pair per buffer (bounded waits, so a warp that stops early on
+// an abort leaves no partner blocked).
 struct Xchg {
     float *base;       // [8 row groups][2 parity][16 rows][kMaxM]
+    uint64_t *bars;    // [8 row groups][2 parity] {full, empty}
     __device__ __forceinline__ float *slot(int rg, int parity, int r16) const {
         return base + ((rg * 2 + parity) * 16 + r16) * kMaxM;
     }
+    __device__ __forceinline__ uint32_t bar(int rg, int parity, int which) const {
+        return smem_u32(&bars[(rg * 2 + parity) * 2 + which]);
+    }
+    // window 1, unit n of this warp: wait until slot n&1 was read two units ago
+    __device__ __forceinline__ bool put_begin(int rg, uint32_t n, volatile int *ab) const {
+        return mbar_wait(bar(rg, n & 1, 1), ((n >> 1) & 1) ^ 1, ab);
+    }
+    __device__ __forceinline__ void put_end(int rg, uint32_t n, int lane) const {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(rg, n & 1, 0));
+    }
+    // window 0: wait for the partials of unit n, then hand the slot back
+    __device__ __forceinline__ bool get_begin(int rg, uint32_t n, volatile int *ab) const {
+        return mbar_wait(bar(rg, n & 1, 0), (n >> 1) & 1, ab);
+    }
+    __device__ __forceinline__ void get_end(int rg, uint32_t n, int lane) const {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(rg, n & 1, 1));
+    }
 };
 
-// ---- packed consumer -----------------------------------------------------------
-// Scale / zero of one group for this lane's rows ra, rb.
-struct SzP {
-    float sa, za, sb, zb;
+// Stage / unit walk shared by the consumers.
+struct Walk {
+    int u, kc, jidx, sidx;
+    uint32_t sph;
 };
-__device__ __forceinline__ void load_sz_packed(const StreamJob &J, int ra, int rb,
-                                               int grp, SzP &o) {
-    const __half *S16 = reinterpret_cast<const __half *>(J.s);
-    const __half *Z16 = reinterpret_cast<const __half *>(J.z);
-    const int G = J.K >> 6;
-    const bool gv = grp < G;
-    const bool va = gv && ra < J.N, vb = gv && rb < J.N;
-    const int64_t ia = (int64_t)ra * G + grp, ib = (int64_t)rb * G + grp;
-    o.sa = va ? __half2float(__ldg(S16 + ia)) : 0.f;
-    o.za = va ? __half2float(__ldg(Z16 + ia)) : 0.f;
-    o.sb = vb ? __half2float(__ldg(S16 + ib)) : 0.f;
-    o.zb = vb ? __half2float(__ldg(Z16 + ib)) : 0.f;
+// A second walk, two stages ahead, tells which scales and zeros to prefetch
+// (it stays on the last stage of the range once it gets there).  It keeps
+// this lane's two scale rows and two zero rows as pointers, renewed once per
+// unit, so a fetch is four loads.  Rows past N are clamped to the last row:
+// they only feed outputs that are never stored.
+struct Ahead {
+    int u, kc, j, G;
+    const unsigned short *s0, *s1, *z0, *z1;
+    __device__ __forceinline__ void rows(const StreamJob *jobs, int ra) {
+        const StreamJob &J = jobs[j];
+        G = J.K >> 6;
+        const int r = (u - J.unit_begin) * kRows + ra;
+        const int64_t b0 = (int64_t)min(r, J.N - 1) * G, b1 = (int64_t)min(r + 8, J.N - 1) * G;
+        s0 = reinterpret_cast<const unsigned short *>(J.s) + b0;
+        s1 = reinterpret_cast<const unsigned short *>(J.s) + b1;
+        z0 = reinterpret_cast<const unsigned short *>(J.z) + b0;
+        z1 = reinterpret_cast<const unsigned short *>(J.z) + b1;
+    }
+    __device__ __forceinline__ void start(const StreamJob *jobs, int u0, int j0, int ra) {
+        u = u0;
+        kc = 0;
+        j = j0;
+        rows(jobs, ra);
+    }
+    __device__ __forceinline__ void advance(const StreamJob *jobs, int count, int u1, int ra) {
+        if (++kc == kchunks_of<true>(jobs[j].K)) {
+            if (u + 1 >= u1) {
+                --kc;
+                return;
+            }
+            kc = 0;
+            ++u;
+            j = next_job(jobs, count, j, u);
+            rows(jobs, ra);
+        }
+    }
+};
+
+// This lane's fp16 scales and zeros for one stage: rows ra and ra+8 of the
+// unit, NG consecutive groups from 8*kc + gw, packed in pairs (g, g+1).
+// Issued two stages before use so the loads are in flight while the stages
+// in between are consumed.  Groups are clamped into the row instead of
+// predicated, so the loads go straight into the registers read two stages
+// later; a group past K/64 multiplies an exactly zero code sum and
+// activation sum.
+template <int NG>
+struct SzRegs {
+    uint32_t s[2][NG / 2], z[2][NG / 2];
+};
+template <int NG>
+__device__ __forceinline__ void fetch_sz(const Ahead &a, int gw, SzRegs<NG> &o) {
+    const int g = 8 * a.kc + gw;
+#pragma unroll
+    for (int p = 0; p < NG / 2; ++p) {
+        if ((a.G & 1) == 0) {         // pair (gg, gg+1) is 4-byte aligned
+            const int gg = min(g + 2 * p, a.G - 2);
+            o.s[0][p] = __ldg(reinterpret_cast<const uint32_t *>(a.s0 + gg));
+            o.s[1][p] = __ldg(reinterpret_cast<const uint32_t *>(a.s1 + gg));
+            o.z[0][p] = __ldg(reinterpret_cast<const uint32_t *>(a.z0 + gg));
+            o.z[1][p] = __ldg(reinterpret_cast<const uint32_t *>(a.z1 + gg));
+        } else {
+            const int g0 = min(g + 2 * p, a.G - 1), g1 = min(g + 2 * p + 1, a.G - 1);
+            o.s[0][p] = (uint32_t)__ldg(a.s0 + g0) | ((uint32_t)__ldg(a.s0 + g1) << 16);
+            o.s[1][p] = (uint32_t)__ldg(a.s1 + g0) | ((uint32_t)__ldg(a.s1 + g1) << 16);
+            o.z[0][p] = (uint32_t)__ldg(a.z0 + g0) | ((uint32_t)__ldg(a.z0 + g1) << 16);
+            o.z[1][p] = (uint32_t)__ldg(a.z1 + g0) | ((uint32_t)__ldg(a.z1 + g1) << 16);
+        }
+    }
 }
 
-template <int MT>
-__device__ __forceinline__ void consume_packed(
+// Window 0 folds window 1's partial row sums of a unit into y one unit
+// later, when they are long written, instead of waiting at the unit's end.
+struct PendingY {
+    bool on = false;
+    uint32_t n = 0;            // unit index (this warp's count) it belongs to
+    float *ya = nullptr;       // y + row of this lane's first row (or null)
+    float *yb = nullptr;       // ... second row (or null)
+    float va[kMaxM / 2 + 1], vb[kMaxM / 2 + 1];
+};
+
+// ---- packed consumer, one x row: block-diagonal groups ---------------------------
+// mma p of a step pairs window units (p, p+4): slots 0-15 take unit p's codes
+// and B columns 0-3, slots 16-31 unit p+4's and columns 4-7.  Units (0,4) and
+// (1,5) belong to groups (0,2), units (2,6) and (3,7) to groups (1,3).
+__device__ __forceinline__ void consume_packed_m1(
     const StreamParams &P, const StreamJob *jobs, uint8_t *smem, uint8_t *xslots,
     uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
     volatile int *abort_flag, const Xchg &xg, int u0, int u1, int cw, int lane) {
     const int S = P.stages;
-    const int rg = cw & 7, w = cw >> 3;               // row group, window
-    const int gq = lane >> 2, t = lane & 3;          // A/C fragment role
-    // mma row gq <-> unit row 16*rg + perm(gq): rows 4 apart share a 16-byte
-    // load phase, so their swizzled units land in different banks
-    const int ra_l = 16 * rg + ((gq >> 1) | ((gq & 1) << 2));
-    const int rb_l = ra_l + 8;
-    const int piece = (lane >> 2) & 1, gsb = lane >> 3;    // B role: column lane>>2
-    const bool act0 = gsb == (t >> 1), act1 = gsb == 2 + (t >> 1);
+    const int rg = cw & 7, w = cw >> 3;
+    const int gq = lane >> 2, t = lane & 3;
+    // ldmatrix: this lane gives the address of row lrow of unit (j + 4*(lane>>4))
+    const int lrow = 16 * rg + (lane & 7) + ((lane >> 3) & 1) * 8;
+    uint32_t a_off[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        a_off[j] = lrow * 128 + ((((lane >> 4) * 4 + j) ^ (lrow & 7)) << 4);
+    // B role: column gq = 4*bh + digit bd
+    const int bh = gq >> 2, bd = gq & 3;
+    const uint32_t m0 = bh ? 0u : 0xffffffffu, m1 = ~m0;
+    // epilogue role: groups 2*eh (+1), digit pair ep
+    const int eh = t >> 1, ep = t & 1;
+    const int ra = 16 * rg + gq;
     XCursor xc;
-    int u = u0, kc = 0, jidx = find_job(jobs, P.count, u);
-    int sidx = 0;              // stage slot and its mbarrier phase
-    uint32_t sph = 0;
-    SzP cur, nxt;
-    {
-        const StreamJob &J = jobs[jidx];
-        const int r0 = (u - J.unit_begin) * kRows;
-        load_sz_packed(J, r0 + ra_l, r0 + rb_l, w * 4 + t, cur);
-    }
-    float yacc[MT][2];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) yacc[m][0] = yacc[m][1] = 0.0f;
+    Walk k{u0, 0, find_job(jobs, P.count, u0), 0, 0u};
+    Ahead ah;
+    ah.start(jobs, u0, k.jidx, ra);
+    SzRegs<2> sz0, sz1, sz2;
+    fetch_sz<2>(ah, 4 * w + 2 * eh, sz0);
+    ah.advance(jobs, P.count, u1, ra);
+    fetch_sz<2>(ah, 4 * w + 2 * eh, sz1);
+    ah.advance(jobs, P.count, u1, ra);
+    float ya = 0.0f, yb = 0.0f;
     int parity = 0;
-    // One stage.  `use` holds this stage's scale/zero (loaded a stage ago);
-    // `fill` receives the next stage's.  The two sets swap roles every call,
-    // so no register copy ever waits on an outstanding load.  Returns true
-    // when this warp is done.
-    auto step = [&](const SzP &use, SzP &fill) -> bool {
-        const StreamJob &J = jobs[jidx];
-        const int r0 = (u - J.unit_begin) * kRows;
-        if (kc == 0 && !x_enter(xc, J, u == u0, xslots, P.xslot_bytes, xfull,
-                                xempty, abort_flag, lane))
+    uint32_t nunit = 0;
+    PendingY pend;
+    // window 0: add window 1's partials of the pending unit and store
+    auto flush = [&]() -> bool {
+        if (!pend.on) return true;
+        if (!xg.get_begin(rg, pend.n, abort_flag)) return false;
+        if (t == 0) {
+            if (pend.ya) *pend.ya = pend.va[0] + xg.slot(rg, pend.n & 1, gq)[0];
+            if (pend.yb) *pend.yb = pend.vb[0] + xg.slot(rg, pend.n & 1, gq + 8)[0];
+        }
+        xg.get_end(rg, pend.n, lane);
+        pend.on = false;
+        return true;
+    };
+    // One stage; `use` holds its scales/zeros, `fill` receives those of the
+    // stage two ahead.  Returns true when this warp is done.
+    auto step = [&](const SzRegs<2> &use, SzRegs<2> &fill) -> bool {
+        fetch_sz<2>(ah, 4 * w + 2 * eh, fill);
+        ah.advance(jobs, P.count, u1, ra);
+        const StreamJob &J = jobs[k.jidx];
+        if (k.kc == 0 && !x_enter(xc, J, k.u == u0, xslots, P.xslot_bytes, xfull, xempty,
+                                  abort_flag, lane))
             return true;
-        const int kchunks = kchunks_of<true>(J.K);
-        int nu = u, nkc = kc + 1, nj = jidx;
-        if (nkc == kchunks) {
-            nu = u + 1;
-            nkc = 0;
-            if (nu < u1) nj = next_job(jobs, P.count, jidx, nu);
-        }
-        if (nu < u1) {          // next stage's scale / zero, fetched early
-            const StreamJob &Jn = jobs[nj];
-            const int nr0 = (nu - Jn.unit_begin) * kRows;
-            load_sz_packed(Jn, nr0 + ra_l, nr0 + rb_l, nkc * 8 + w * 4 + t, fill);
-        }
-        const int s = sidx;
-        if (!mbar_wait(smem_u32(&full[s]), sph, abort_flag)) return true;
-        const int kp = kpad_of<true>(J.K);
-        const int mb = xrow_bytes<true>(J.K);
-        const uint8_t *box = smem + s * kStageBytes + w * kBoxBytes;
-        // independent accumulator chains hide the MMA latency (fewer when
-        // several x rows already give independent work)
-        constexpr int NCH = MT == 1 ? 4 : 2;
-        float acc[MT][NCH][4];
+        const int kch = kchunks_of<true>(J.K);
+        const int rs = dig_rs(kch);
+        const int s = k.sidx;
+        if (!mbar_wait(smem_u32(&full[s]), k.sph, abort_flag)) return true;
+        const uint32_t box = smem_u32(smem + s * kStageBytes + w * kBoxBytes);
+        uint32_t R[4][4];
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
+        for (int j = 0; j < 4; ++j) ldsm_x4(box + a_off[j], R[j]);
+        const uint32_t *xd = reinterpret_cast<const uint32_t *>(xc.xs) + (bd * 4 + t) * rs +
+                             2 * (16 * k.kc + 8 * w + 4 * bh);
+        const uint4 Q0 = *reinterpret_cast<const uint4 *>(xd);
+        const uint4 Q1 = *reinterpret_cast<const uint4 *>(xd + 4);
+        const float4 tb = *reinterpret_cast<const float4 *>(
+            xc.xs + 64 * rs + 8 * (ep * 8 * kch + 8 * k.kc + 4 * w + 2 * eh));
+        uint32_t lo[4][4], hi[4][4];
 #pragma unroll
-            for (int a = 0; a < NCH; ++a)
-                acc[m][a][0] = acc[m][a][1] = acc[m][a][2] = acc[m][a][3] = 0.0f;
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-            const uint4 qa = *reinterpret_cast<const uint4 *>(box + sw_off(ra_l, ch * 4 + t));
-            const uint4 qb = *reinterpret_cast<const uint4 *>(box + sw_off(rb_l, ch * 4 + t));
-            const bool act = ch == 0 ? act0 : act1;
-            const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
-            const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                uint32_t A[4], B[4];
-                unpack8(wa[i], A);
-                unpack8(wb[i], B);
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    // x pieces at k = kc*512 + w*256 + ch*128 + 32*t + 8*i
-                    const uint8_t *bp = xc.xs + m * mb + piece * (2 * kp + kPiecePad) +
-                                        (kc * 512 + w * 256 + ch * 128 + 32 * t + 8 * i) * 2;
-                    uint4 bv = make_uint4(0u, 0u, 0u, 0u);
-                    if (act) bv = *reinterpret_cast<const uint4 *>(bp);
-                    constexpr int base = 0;
-                    const int c0 = NCH == 4 ? ch * 2 : base, c1 = c0 + 1;
-                    mma16816(acc[m][c0], A[0], B[0], A[1], B[1], bv.x, bv.y);
-                    mma16816(acc[m][c1], A[2], B[2], A[3], B[3], bv.z, bv.w);
-                }
+                lo[j][i] = R[j][i] & 0x0F0F0F0Fu;
+                hi[j][i] = R[j][i] & 0xF0F0F0F0u;
             }
-        }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[s]));   // stage consumed
-        const int grp = kc * 8 + w * 4 + t;
-        if (grp < (J.K >> 6)) {
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                float c[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    c[q] = acc[m][0][q] + acc[m][1][q];
-                    if constexpr (NCH == 4) c[q] += acc[m][2][q] + acc[m][3][q];
-                }
-                const float2 xsum = reinterpret_cast<const float2 *>(
-                    xc.xs + m * mb + 4 * kp + kPiecePad)[grp];
-                const float v0 = (c[0] + c[1]) - (256.0f + use.za) * xsum.x -
-                                 (16.0f + use.za) * xsum.y;
-                const float v1 = (c[2] + c[3]) - (256.0f + use.zb) * xsum.x -
-                                 (16.0f + use.zb) * xsum.y;
-                yacc[m][0] = fmaf(use.sa, v0, yacc[m][0]);
-                yacc[m][1] = fmaf(use.sb, v1, yacc[m][1]);
-            }
+        int CA[4] = {0, 0, 0, 0}, CB[4] = {0, 0, 0, 0};
+        mma_i8(CA, lo[0][0], lo[0][1], lo[0][2], lo[0][3], Q0.x & m0, Q0.x & m1);
+        mma_i8(CB, lo[2][0], lo[2][1], lo[2][2], lo[2][3], Q1.x & m0, Q1.x & m1);
+        mma_i8(CA, hi[0][0], hi[0][1], hi[0][2], hi[0][3], Q0.y & m0, Q0.y & m1);
+        mma_i8(CB, hi[2][0], hi[2][1], hi[2][2], hi[2][3], Q1.y & m0, Q1.y & m1);
+        mma_i8(CA, lo[1][0], lo[1][1], lo[1][2], lo[1][3], Q0.z & m0, Q0.z & m1);
+        mma_i8(CB, lo[3][0], lo[3][1], lo[3][2], lo[3][3], Q1.z & m0, Q1.z & m1);
+        mma_i8(CA, hi[1][0], hi[1][1], hi[1][2], hi[1][3], Q0.w & m0, Q0.w & m1);
+        mma_i8(CB, hi[3][0], hi[3][1], hi[3][2], hi[3][3], Q1.w & m0, Q1.w & m1);
+        // this lane: digits (2ep, 2ep+1) of rows ra, ra+8 for groups 2eh (A), 2eh+1 (B)
+        const float2 sa = half2_bits_to_float2(use.s[0][0]), sb = half2_bits_to_float2(use.s[1][0]);
+        const float2 za = half2_bits_to_float2(use.z[0][0]), zb = half2_bits_to_float2(use.z[1][0]);
+        const float vAa = (float)(CA[0] + 256 * CA[1]), vAb = (float)(CA[2] + 256 * CA[3]);
+        const float vBa = (float)(CB[0] + 256 * CB[1]), vBb = (float)(CB[2] + 256 * CB[3]);
+        ya = fmaf(sa.x, fmaf(tb.x, vAa, -za.x * tb.y), ya);
+        yb = fmaf(sb.x, fmaf(tb.x, vAb, -zb.x * tb.y), yb);
+        ya = fmaf(sa.y, fmaf(tb.z, vBa, -za.y * tb.w), ya);
+        yb = fmaf(sb.y, fmaf(tb.z, vBb, -zb.y * tb.w), yb);
+
+        int nu = k.u, nkc = k.kc + 1, nj = k.jidx;
+        if (nkc == kch) {
+            nu = k.u + 1;
+            nkc = 0;
+            if (nu < u1) nj = next_job(jobs, P.count, k.jidx, nu);
         }
-        if (nkc == 0) {       // unit done: four group lanes, then two windows
-#pragma unroll
-            for (int m = 0; m < MT; ++m)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    float v = yacc[m][h];
-                    v += __shfl_xor_sync(0xffffffffu, v, 1);
-                    v += __shfl_xor_sync(0xffffffffu, v, 2);
-                    yacc[m][h] = v;
+        if (nkc == 0) {       // unit done: four lanes per row, then two windows
+            ya += __shfl_xor_sync(0xffffffffu, ya, 1);
+            ya += __shfl_xor_sync(0xffffffffu, ya, 2);
+            yb += __shfl_xor_sync(0xffffffffu, yb, 1);
+            yb += __shfl_xor_sync(0xffffffffu, yb, 2);
+            if (w == 1) {
+                if (!xg.put_begin(rg, nunit, abort_flag)) return true;
+                if (t == 0) {
+                    xg.slot(rg, parity, gq)[0] = ya;
+                    xg.slot(rg, parity, gq + 8)[0] = yb;
                 }
-            if (w == 1 && t == 0) {
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    xg.slot(rg, parity, 2 * gq)[m] = yacc[m][0];
-                    xg.slot(rg, parity, 2 * gq + 1)[m] = yacc[m][1];
-                }
+                xg.put_end(rg, nunit, lane);
+            } else {
+                if (!flush()) return true;
+                const int r0 = (k.u - J.unit_begin) * kRows;
+                pend.on = true;
+                pend.n = nunit;
+                pend.ya = r0 + ra < J.N ? J.y + r0 + ra : nullptr;
+                pend.yb = r0 + ra + 8 < J.N ? J.y + r0 + ra + 8 : nullptr;
+                pend.va[0] = ya;
+                pend.vb[0] = yb;
             }
-            named_bar(1 + rg, 64);
-            if (w == 0 && t == 0) {
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    if (m >= P.M) break;
-                    const float ya = yacc[m][0] + xg.slot(rg, parity, 2 * gq)[m];
-                    const float yb = yacc[m][1] + xg.slot(rg, parity, 2 * gq + 1)[m];
-                    if (r0 + ra_l < J.N) J.y[(int64_t)m * J.N + r0 + ra_l] = ya;
-                    if (r0 + rb_l < J.N) J.y[(int64_t)m * J.N + r0 + rb_l] = yb;
-                }
-            }
-#pragma unroll
-            for (int m = 0; m < MT; ++m) yacc[m][0] = yacc[m][1] = 0.0f;
+            ya = yb = 0.0f;
             parity ^= 1;
+            ++nunit;
         }
         if (nu >= u1) return true;
-        u = nu;
-        kc = nkc;
-        jidx = nj;
-        if (++sidx == S) {      // ring position of the next stage
-            sidx = 0;
-            sph ^= 1;
+        k.u = nu;
+        k.kc = nkc;
+        k.jidx = nj;
+        if (++k.sidx == S) {      // ring position of the next stage
+            k.sidx = 0;
+            k.sph ^= 1;
         }
         return false;
     };
-    while (!step(cur, nxt) && !step(nxt, cur)) {
+    while (!step(sz0, sz2) && !step(sz1, sz0) && !step(sz2, sz1)) {
+    }
+    if (w == 0) flush();
+}
+
+// ---- packed consumer, 2 or 4 x rows ------------------------------------------------
+// Each mma takes one 32-k unit (slots 0-15 even k, 16-31 odd k) and a pair of
+// x rows as B columns (row 2*mp + h in columns 4h..4h+3).
+template <int MT>
+__device__ __forceinline__ void consume_packed_mx(
+    const StreamParams &P, const StreamJob *jobs, uint8_t *smem, uint8_t *xslots,
+    uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
+    volatile int *abort_flag, const Xchg &xg, int u0, int u1, int cw, int lane) {
+    constexpr int MP = MT / 2;
+    const int S = P.stages;
+    const int rg = cw & 7, w = cw >> 3;
+    const int gq = lane >> 2, t = lane & 3;
+    // ldmatrix: this lane gives the address of row lrow of unit (2j + (lane>>4))
+    const int lrow = 16 * rg + (lane & 7) + ((lane >> 3) & 1) * 8;
+    uint32_t a_off[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        a_off[j] = lrow * 128 + (((2 * j + (lane >> 4)) ^ (lrow & 7)) << 4);
+    const int bh = gq >> 2, bd = gq & 3;
+    const int eh = t >> 1, ep = t & 1;
+    const int ra = 16 * rg + gq;
+    XCursor xc;
+    Walk k{u0, 0, find_job(jobs, P.count, u0), 0, 0u};
+    Ahead ah;
+    ah.start(jobs, u0, k.jidx, ra);
+    SzRegs<4> sz0, sz1, sz2;
+    fetch_sz<4>(ah, 4 * w, sz0);
+    ah.advance(jobs, P.count, u1, ra);
+    fetch_sz<4>(ah, 4 * w, sz1);
+    ah.advance(jobs, P.count, u1, ra);
+    float ya[MP], yb[MP];
+#pragma unroll
+    for (int p = 0; p < MP; ++p) ya[p] = yb[p] = 0.0f;
+    int parity = 0;
+    uint32_t nunit = 0;
+    auto step = [&](const SzRegs<4> &use, SzRegs<4> &fill) -> bool {
+        fetch_sz<4>(ah, 4 * w, fill);
+        ah.advance(jobs, P.count, u1, ra);
+        const StreamJob &J = jobs[k.jidx];
+        if (k.kc == 0 && !x_enter(xc, J, k.u == u0, xslots, P.xslot_bytes, xfull, xempty,
+                                  abort_flag, lane))
+            return true;
+        const int kch = kchunks_of<true>(J.K);
+        const int rs = dig_rs(kch);
+        const int mb = xrow_bytes<true>(J.K);
+        const int s = k.sidx;
+        if (!mbar_wait(smem_u32(&full[s]), k.sph, abort_flag)) return true;
+        const uint32_t box = smem_u32(smem + s * kStageBytes + w * kBoxBytes);
+        uint32_t R[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ldsm_x4(box + a_off[j], R[j]);
+        uint32_t lo[4][4], hi[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                lo[j][i] = R[j][i] & 0x0F0F0F0Fu;
+                hi[j][i] = R[j][i] & 0xF0F0F0F0u;
+            }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty[s]));   // stage consumed
+        float sa[4], sb[4], za[4], zb[4];
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const float2 a2 = half2_bits_to_float2(use.s[0][p]), b2 = half2_bits_to_float2(use.s[1][p]);
+            const float2 c2 = half2_bits_to_float2(use.z[0][p]), d2 = half2_bits_to_float2(use.z[1][p]);
+            sa[2 * p] = a2.x; sa[2 * p + 1] = a2.y;
+            sb[2 * p] = b2.x; sb[2 * p + 1] = b2.y;
+            za[2 * p] = c2.x; za[2 * p + 1] = c2.y;
+            zb[2 * p] = d2.x; zb[2 * p + 1] = d2.y;
+        }
+#pragma unroll
+        for (int mp = 0; mp < MP; ++mp) {
+            // B: this lane's words for units 0..7 of the window, both parities
+            const uint32_t *xd = reinterpret_cast<const uint32_t *>(xc.xs + (2 * mp + bh) * mb) +
+                                 (bd * 4 + t) * rs + 2 * (16 * k.kc + 8 * w);
+            uint4 Q[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) Q[j] = reinterpret_cast<const uint4 *>(xd)[j];
+            int C[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                C[j][0] = C[j][1] = C[j][2] = C[j][3] = 0;
+                mma_i8(C[j], lo[j][0], lo[j][1], hi[j][0], hi[j][1], Q[j].x, Q[j].y);
+                mma_i8(C[j], lo[j][2], lo[j][3], hi[j][2], hi[j][3], Q[j].z, Q[j].w);
+            }
+            const float *tb = reinterpret_cast<const float *>(
+                xc.xs + (2 * mp + eh) * mb + 64 * rs + 8 * (ep * 8 * kch + 8 * k.kc + 4 * w));
+            const float4 t01 = reinterpret_cast<const float4 *>(tb)[0];
+            const float4 t23 = reinterpret_cast<const float4 *>(tb)[1];
+            const float f[4] = {t01.x, t01.z, t23.x, t23.z};
+            const float X[4] = {t01.y, t01.w, t23.y, t23.w};
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const float va = (float)(C[g][0] + 256 * C[g][1]);
+                const float vb = (float)(C[g][2] + 256 * C[g][3]);
+                ya[mp] = fmaf(sa[g], fmaf(f[g], va, -za[g] * X[g]), ya[mp]);
+                yb[mp] = fmaf(sb[g], fmaf(f[g], vb, -zb[g] * X[g]), yb[mp]);
+            }
+        }
+
+        int nu = k.u, nkc = k.kc + 1, nj = k.jidx;
+        if (nkc == kch) {
+            nu = k.u + 1;
+            nkc = 0;
+            if (nu < u1) nj = next_job(jobs, P.count, k.jidx, nu);
+        }
+        if (nkc == 0) {       // unit done: two lanes per row and x row, then two windows
+#pragma unroll
+            for (int mp = 0; mp < MP; ++mp) {
+                ya[mp] += __shfl_xor_sync(0xffffffffu, ya[mp], 1);
+                yb[mp] += __shfl_xor_sync(0xffffffffu, yb[mp], 1);
+            }
+            if (w == 1) {
+                if (!xg.put_begin(rg, nunit, abort_flag)) return true;
+                if (ep == 0) {
+#pragma unroll
+                    for (int mp = 0; mp < MP; ++mp) {
+                        xg.slot(rg, parity, gq)[2 * mp + eh] = ya[mp];
+                        xg.slot(rg, parity, gq + 8)[2 * mp + eh] = yb[mp];
+                    }
+                }
+                xg.put_end(rg, nunit, lane);
+            } else {
+                if (!xg.get_begin(rg, nunit, abort_flag)) return true;
+                if (ep == 0) {
+                    const int r0 = (k.u - J.unit_begin) * kRows;
+#pragma unroll
+                    for (int mp = 0; mp < MP; ++mp) {
+                        const int m = 2 * mp + eh;
+                        if (m >= P.M) continue;
+                        if (r0 + ra < J.N)
+                            J.y[(int64_t)m * J.N + r0 + ra] =
+                                ya[mp] + xg.slot(rg, parity, gq)[m];
+                        if (r0 + ra + 8 < J.N)
+                            J.y[(int64_t)m * J.N + r0 + ra + 8] =
+                                yb[mp] + xg.slot(rg, parity, gq + 8)[m];
+                    }
+                }
+                xg.get_end(rg, nunit, lane);
+            }
+#pragma unroll
+            for (int mp = 0; mp < MP; ++mp) ya[mp] = yb[mp] = 0.0f;
+            parity ^= 1;
+            ++nunit;
+        }
+        if (nu >= u1) return true;
+        k.u = nu;
+        k.kc = nkc;
+        k.jidx = nj;
+        if (++k.sidx == S) {
+            k.sidx = 0;
+            k.sph ^= 1;
+        }
+        return false;
+    };
+    while (!step(sz0, sz2) && !step(sz1, sz0) && !step(sz2, sz1)) {
     }
 }
 
@@ -447,6 +824,7 @@ __device__ __forceinline__ void consume_runtime(
 #pragma unroll
     for (int m = 0; m < MT; ++m) yacc[m] = 0.0f;
     int parity = 0;
+    uint32_t nunit = 0;
     auto step = [&](const float2 use, float2 &fill) -> bool {
         const float s_cur = use.x, z_cur = use.y;
         const StreamJob &J = jobs[jidx];
@@ -477,8 +855,9 @@ __device__ __forceinline__ void consume_runtime(
                                          4.76837158203125e-07f;   // 2^-21
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
-                const uint4 raw =
-                    *reinterpret_cast<const uint4 *>(box + sw_off(rr, part * 4 + c8));
+                const int u16 = part * 4 + c8;
+                const uint4 raw = *reinterpret_cast<const uint4 *>(
+                    box + rr * 128 + ((u16 ^ (rr & 7)) << 4));
                 const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
                 float wv[8];
 #pragma unroll
@@ -534,21 +913,28 @@ __device__ __forceinline__ void consume_runtime(
 #pragma unroll
             for (int m = 0; m < MT; ++m)
                 yacc[m] += __shfl_xor_sync(0xffffffffu, yacc[m], 1);
-            if (w == 1 && part == 0) {
+            if (w == 1) {
+                if (!xg.put_begin(rg, nunit, abort_flag)) return true;
+                if (part == 0) {
 #pragma unroll
-                for (int m = 0; m < MT; ++m) xg.slot(rg, parity, r16)[m] = yacc[m];
-            }
-            named_bar(1 + rg, 64);
-            if (w == 0 && part == 0 && row < J.N) {
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    if (m >= P.M) break;
-                    J.y[(int64_t)m * J.N + row] = yacc[m] + xg.slot(rg, parity, r16)[m];
+                    for (int m = 0; m < MT; ++m) xg.slot(rg, parity, r16)[m] = yacc[m];
                 }
+                xg.put_end(rg, nunit, lane);
+            } else {
+                if (!xg.get_begin(rg, nunit, abort_flag)) return true;
+                if (part == 0 && row < J.N) {
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        if (m >= P.M) break;
+                        J.y[(int64_t)m * J.N + row] = yacc[m] + xg.slot(rg, parity, r16)[m];
+                    }
+                }
+                xg.get_end(rg, nunit, lane);
             }
 #pragma unroll
             for (int m = 0; m < MT; ++m) yacc[m] = 0.0f;
             parity ^= 1;
+            ++nunit;
         }
         if (nu >= u1) return true;
         u = nu;
@@ -577,10 +963,23 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     uint64_t *full = bars, *empty = bars + S;
     uint64_t *xfull = bars + 2 * S, *xempty = xfull + 2;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(xempty + 2);
-    StreamJob *jobs = reinterpret_cast<StreamJob *>(bars + 2 * S + 8);
+    uint64_t *xbars = bars + 2 * S + 8;                 // 8 row groups x 2 x {full, empty}
+    StreamJob *jobs = reinterpret_cast<StreamJob *>(bars + 2 * S + 8 + 32);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u0 = P.cta_begin[blockIdx.x], u1 = P.cta_begin[blockIdx.x + 1];
+    // The activations of this CTA's matrices go to L2 ahead of the weight
+    // stream: queued behind the first ring fill they would hold up the start.
+    if (warp >= 1 && u0 < u1) {
+        const int jf = find_job(P.jobs, P.count, u0), jl = find_job(P.jobs, P.count, u1 - 1);
+        for (int j = jf; j <= jl; ++j) {
+            const StreamJob &J = P.jobs[j];
+            if (j > jf && P.jobs[j - 1].x == J.x) continue;
+            const int lines = (int)(((int64_t)P.M * J.K * 4 + 127) / 128);
+            for (int l = 32 * (warp - 1) + lane; l < lines; l += 32 * kStagers)
+                prefetch_l2(reinterpret_cast<const char *>(J.x) + (int64_t)l * 128);
+        }
+    }
     {
         const uint32_t *src = reinterpret_cast<const uint32_t *>(P.jobs);
         uint32_t *dst = reinterpret_cast<uint32_t *>(jobs);
@@ -597,28 +996,50 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
             mbar_init(smem_u32(&xfull[b]), 32);
             mbar_init(smem_u32(&xempty[b]), kConsumers);
         }
+        for (int b = 0; b < 32; ++b) mbar_init(smem_u32(&xbars[b]), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
 
     if (warp == 0) {
-        // ---------------- weight producer (one thread) ----------------
+        // ---------------- loader ----------------
+        const uint64_t policy = evict_first_policy();
         uint32_t g = 0, armed = 0;
         int jw = u0 < u1 ? find_job(jobs, P.count, u0) : 0;
         int pidx = 0;
         uint32_t pph = 0;
-        for (int u = u0; u < u1 && lane == 0 && !*abort_flag; ++u) {
+        bool ok = true;
+        for (int u = u0; u < u1 && ok; ++u) {
             jw = next_job(jobs, P.count, jw, u);
             const int j = jw;
             const StreamJob &J = jobs[j];
             const int r0 = (u - J.unit_begin) * kRows;
             const int rbytes = row_bytes_of<PACKED>(J.K);
             const int kchunks = kchunks_of<PACKED>(J.K);
-            bool ok = true;
+            if constexpr (PACKED) {
+                // the unit's scales and zeros (one contiguous block each) go to
+                // L2 with its weights; consumers read them a few stages later
+                const int G = J.K >> 6;
+                const int64_t b0 = (int64_t)r0 * G * 2;
+                const int64_t b1 = (int64_t)min(r0 + kRows, J.N) * G * 2;
+                const int lines = (int)((b1 - b0 + 127) >> 7) + 1;
+                const char *sb = reinterpret_cast<const char *>(J.s) + (b0 & ~(int64_t)127);
+                const char *zb = reinterpret_cast<const char *>(J.z) + (b0 & ~(int64_t)127);
+                const int64_t limit = (int64_t)J.N * G * 2 - (b0 & ~(int64_t)127);
+                for (int l = lane; l < lines; l += 32) {
+                    if ((int64_t)l * 128 >= limit) break;
+                    prefetch_l2(sb + (int64_t)l * 128);
+                    prefetch_l2(zb + (int64_t)l * 128);
+                }
+            }
             for (int kc = 0; kc < kchunks; ++kc, ++g) {
                 const int s = pidx;
-                if (!mbar_wait(smem_u32(&empty[s]), pph ^ 1, abort_flag)) {
+                bool got = true;
+                if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), pph ^ 1, abort_flag);
+                got = __shfl_sync(0xffffffffu, got, 0);
+                __syncwarp();
+                if (!got) {
                     ok = false;
                     break;
                 }
@@ -626,19 +1047,21 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
                     pidx = 0;
                     pph ^= 1;
                 }
-                // a window wholly past the row end is not loaded: its weights
-                // meet zero activations (packed) or are skipped (runtime)
-                const int nbox = (rbytes - kc * kChunk) > 128 ? 2 : 1;
                 const uint32_t fb = smem_u32(&full[s]);
-                mbar_expect_tx(fb, (uint32_t)(nbox * kBoxBytes));
-                const uint32_t st = smem_u32(smem + s * kStageBytes);
-                for (int b = 0; b < nbox; ++b)
-                    tma_load_2d(st + b * kBoxBytes, &P.wmap[j], kc * kChunk + b * 128, r0, fb);
+                if (lane == 0) {
+                    // a window wholly past the row end is not loaded: its codes
+                    // meet zero activation digits (packed) or are skipped (runtime)
+                    const int nbox = (rbytes - kc * kChunk) > 128 ? 2 : 1;
+                    mbar_expect_tx(fb, (uint32_t)(nbox * kBoxBytes));
+                    const uint32_t st = smem_u32(smem + s * kStageBytes);
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d(st + b * kBoxBytes, &P.wmap[j], kc * kChunk + b * 128, r0, fb,
+                                    policy);
+                }
                 armed |= 1u << s;
             }
-            if (!ok) break;
         }
-        // drain: loads in flight land before the CTA exits
+        // drain: copies in flight land before the CTA exits
         if (lane == 0 && g > 0) {
             for (int q = 0; q < S; ++q) {
                 if (!(armed & (1u << q))) continue;
@@ -650,118 +1073,51 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ---------------- activation stager ----------------
-        const float *cur = nullptr;
-        uint32_t e = 0;
-        int js = u0 < u1 ? find_job(jobs, P.count, u0) : 0;
-        for (int u = u0; u < u1 && !*abort_flag; ++u) {
-            js = next_job(jobs, P.count, js, u);
-            const StreamJob &J = jobs[js];
-            if (u != u0 && J.x == cur) continue;
-            cur = J.x;
-            const int slot = e & 1;
-            if (!mbar_wait(smem_u32(&xempty[slot]), ((e >> 1) & 1) ^ 1, abort_flag)) break;
-            uint8_t *xs = xslots + slot * P.xslot_bytes;
-            const int K = J.K;
-            const int kp = kpad_of<PACKED>(K);
-            const int mb = xrow_bytes<PACKED>(K);
-            for (int m = 0; m < P.M; ++m) {
-                const float *xr = J.x + (int64_t)m * K;
-                uint8_t *xm = xs + m * mb;
+    } else {
+        // the first x slot, by every warp but the loader
+        if (u0 < u1) {
+            const StreamJob &J0 = jobs[find_job(jobs, P.count, u0)];
+            stage_x<PACKED>(J0, P.M, xslots, warp - 1, kStagers, lane);
+            named_bar(9, 32 * kStagers);
+            if (warp == 1) mbar_arrive(smem_u32(&xfull[0]));
+        }
+        if (warp == 1) {
+            // ---------------- activation stager ----------------
+            const float *cur = nullptr;
+            uint32_t e = 0;
+            int js = u0 < u1 ? find_job(jobs, P.count, u0) : 0;
+            for (int u = u0; u < u1 && !*abort_flag; ++u) {
+                js = next_job(jobs, P.count, js, u);
+                const StreamJob &J = jobs[js];
+                if (u != u0 && J.x == cur) continue;
+                cur = J.x;
+                if (u == u0) {     // filled above
+                    e = 1;
+                    continue;
+                }
+                const int slot = e & 1;
+                if (!mbar_wait(smem_u32(&xempty[slot]), ((e >> 1) & 1) ^ 1, abort_flag)) break;
+                stage_x<PACKED>(J, P.M, xslots + slot * P.xslot_bytes, 0, 1, lane);
+                mbar_arrive(smem_u32(&xfull[slot]));     // every lane, after its writes
+                ++e;
+            }
+        } else {
+            // ---------------- consumers ----------------
+            const int cw = warp - 2;
+            const Xchg xg{xchg, xbars};
+            if (u0 < u1) {
                 if constexpr (PACKED) {
-                    __half *hi = reinterpret_cast<__half *>(xm);
-                    __half *lo = reinterpret_cast<__half *>(xm + 2 * kp + kPiecePad);
-                    float2 *sums = reinterpret_cast<float2 *>(xm + 4 * kp + kPiecePad);
-                    // 8-blocks; lanes 8q..8q+7 hold one 64-group.  Loads are
-                    // issued kBatch blocks ahead so the stager pays one memory
-                    // round trip per batch, not per block.
-                    constexpr int kBatch = 4;
-                    for (int b00 = 0; b00 < kp / 8; b00 += 32 * kBatch) {
-                      float4 pre[kBatch][2];
-#pragma unroll
-                      for (int q = 0; q < kBatch; ++q) {
-                          const int b = b00 + 32 * q + lane;
-                          pre[q][0] = pre[q][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-                          if (8 * b < K) {
-                              pre[q][0] = __ldg(reinterpret_cast<const float4 *>(xr + 8 * b));
-                              pre[q][1] = __ldg(reinterpret_cast<const float4 *>(xr + 8 * b + 4));
-                          }
-                      }
-#pragma unroll
-                      for (int q = 0; q < kBatch; ++q) {
-                        const int b = b00 + 32 * q + lane;
-                        if (b00 + 32 * q >= kp / 8) break;
-                        float v[8];
-                        v[0] = pre[q][0].x; v[1] = pre[q][0].y; v[2] = pre[q][0].z; v[3] = pre[q][0].w;
-                        v[4] = pre[q][1].x; v[5] = pre[q][1].y; v[6] = pre[q][1].z; v[7] = pre[q][1].w;
-                        __half h[8], l[8];
-                        float se = 0.0f, so = 0.0f;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            h[i] = __float2half_rn(v[i]);
-                            const float hf = __half2float(h[i]);
-                            l[i] = __float2half_rn(v[i] - hf);
-                            const float xt = hf + __half2float(l[i]);
-                            if (i & 1) so += xt; else se += xt;
-                        }
-                        // fragment order of an 8-block: k0 k4 k1 k5 k2 k6 k3 k7
-                        const __half2 H0 = __halves2half2(h[0], h[4]), H1 = __halves2half2(h[1], h[5]);
-                        const __half2 H2 = __halves2half2(h[2], h[6]), H3 = __halves2half2(h[3], h[7]);
-                        const __half2 L0 = __halves2half2(l[0], l[4]), L1 = __halves2half2(l[1], l[5]);
-                        const __half2 L2 = __halves2half2(l[2], l[6]), L3 = __halves2half2(l[3], l[7]);
-                        uint4 hv, lv;
-                        hv.x = *reinterpret_cast<const uint32_t *>(&H0);
-                        hv.y = *reinterpret_cast<const uint32_t *>(&H1);
-                        hv.z = *reinterpret_cast<const uint32_t *>(&H2);
-                        hv.w = *reinterpret_cast<const uint32_t *>(&H3);
-                        lv.x = *reinterpret_cast<const uint32_t *>(&L0);
-                        lv.y = *reinterpret_cast<const uint32_t *>(&L1);
-                        lv.z = *reinterpret_cast<const uint32_t *>(&L2);
-                        lv.w = *reinterpret_cast<const uint32_t *>(&L3);
-                        *reinterpret_cast<uint4 *>(hi + 8 * b) = hv;
-                        *reinterpret_cast<uint4 *>(lo + 8 * b) = lv;
-#pragma unroll
-                        for (int off = 1; off < 8; off <<= 1) {
-                            se += __shfl_xor_sync(0xffffffffu, se, off);
-                            so += __shfl_xor_sync(0xffffffffu, so, off);
-                        }
-                        if ((lane & 7) == 0) sums[b / 8] = make_float2(se, so);
-                      }
-                    }
+                    if constexpr (MT == 1)
+                        consume_packed_m1(P, jobs, smem, xslots, full, empty, xfull, xempty,
+                                          abort_flag, xg, u0, u1, cw, lane);
+                    else
+                        consume_packed_mx<MT>(P, jobs, smem, xslots, full, empty, xfull,
+                                              xempty, abort_flag, xg, u0, u1, cw, lane);
                 } else {
-                    float *xf = reinterpret_cast<float *>(xm);
-                    constexpr int kBatch = 8;
-                    for (int k0 = 4 * lane; k0 < kp; k0 += 128 * kBatch) {
-                        float4 v[kBatch];
-#pragma unroll
-                        for (int q = 0; q < kBatch; ++q) {
-                            const int k = k0 + 128 * q;
-                            v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-                            if (k < K) v[q] = __ldg(reinterpret_cast<const float4 *>(xr + k));
-                        }
-#pragma unroll
-                        for (int q = 0; q < kBatch; ++q) {
-                            const int k = k0 + 128 * q;
-                            if (k < kp) *reinterpret_cast<float4 *>(xf + k) = v[q];
-                        }
-                    }
+                    consume_runtime<MT>(P, jobs, smem, xslots, full, empty, xfull, xempty,
+                                        abort_flag, xg, u0, u1, cw, lane);
                 }
             }
-            mbar_arrive(smem_u32(&xfull[slot]));     // every lane, after its writes
-            ++e;
-        }
-    } else {
-        // ---------------- consumers ----------------
-        const int cw = warp - 2;
-        const Xchg xg{xchg};
-        if (u0 < u1) {
-            if constexpr (PACKED)
-                consume_packed<MT>(P, jobs, smem, xslots, full, empty, xfull, xempty,
-                                   abort_flag, xg, u0, u1, cw, lane);
-            else
-                consume_runtime<MT>(P, jobs, smem, xslots, full, empty, xfull, xempty,
-                                    abort_flag, xg, u0, u1, cw, lane);
         }
     }
     __syncthreads();
@@ -771,7 +1127,7 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
 // host side
 // ---------------------------------------------------------------------------
 constexpr int kXchgBytes = 8 * 2 * 16 * kMaxM * 4;
-constexpr int kBarBytes = 256 + kMaxJobs * (int)sizeof(StreamJob);
+constexpr int kBarBytes = 512 + kMaxJobs * (int)sizeof(StreamJob);
 
 template <bool PACKED, int MT>
 bc_status launch_one(const StreamParams &P, int grid, int smem, cudaStream_t s) {
@@ -820,7 +1176,10 @@ bool encode_weights(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Slots hold MT x rows (M rounded up to the kernel's 1, 2 or 4): the
+// consumers of M = 3 read a fourth row whose results are never stored.
 size_t xslot_bytes_for(const GemvJob *jobs, int count, int M, bool packed) {
+    M = M <= 1 ? 1 : M <= 2 ? 2 : 4;
     size_t xmax = 0;
     for (int i = 0; i < count; ++i) {
         const int K = (int)jobs[i].K;
@@ -897,13 +1256,13 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
         P.xslot_bytes = (int)xs;
         P.stages = stages;
         const int smem = stages * kStageBytes + fixed;
-        const int mt = M <= 1 ? 1 : M <= 2 ? 2 : 4;
         bc_status st;
         if (packed) {
-            st = mt == 1 ? launch_one<true, 1>(P, grid, smem, s)
-               : mt == 2 ? launch_one<true, 2>(P, grid, smem, s)
-                         : launch_one<true, 4>(P, grid, smem, s);
+            st = M <= 1 ? launch_one<true, 1>(P, grid, smem, s)
+               : M <= 2 ? launch_one<true, 2>(P, grid, smem, s)
+                        : launch_one<true, 4>(P, grid, smem, s);
         } else {
+            const int mt = M <= 1 ? 1 : M <= 2 ? 2 : 4;
             st = mt == 1 ? launch_one<false, 1>(P, grid, smem, s)
                : mt == 2 ? launch_one<false, 2>(P, grid, smem, s)
                          : launch_one<false, 4>(P, grid, smem, s);
