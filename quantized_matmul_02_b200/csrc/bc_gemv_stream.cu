@@ -16,12 +16,12 @@
 //   warp 1      activation stager: the x of each new matrix goes into one of
 //               two smem slots (see below); the first slot is filled by every
 //               warp but the loader together before streaming starts.
-//   warps 2-17  consumers: warp (window w, row group g) handles 16 rows and
-//               the w-th 128-byte window of every stage; the two windows'
-//               partial row sums meet in smem at the end of each unit.  Each
-//               lane loads its own fp16 scales and zeros from global memory two
-//               stages ahead (small scattered copies cost the loader more issue
-//               time than the stage itself).
+//   warp 2      scale/zero stager (packed): the fp16 scales and zeros of each
+//               stage (128 rows x 8 groups) into a ring slot beside it, with
+//               coalesced loads a stage ahead of the stores; its arrival is
+//               the second one each full barrier counts.
+//   warps 3-10  consumers: warp g handles rows 16g..16g+15 of each unit over
+//               both 128-byte windows of every stage.
 //
 // Packed int4 (Enargeia, "Four bits per weight": codes unpacked in registers,
 // never written back) runs on the int8 tensor cores (mma.sync m16n8k32
@@ -63,9 +63,12 @@ constexpr int kRows = 128;              // weight rows per unit
 constexpr int kChunk = 256;             // bytes of a row per stage
 constexpr int kBoxBytes = kRows * 128;  // one TMA box: 128 rows x 128 bytes, SW128
 constexpr int kStageBytes = 2 * kBoxBytes;
-constexpr int kConsumers = 16;
+constexpr int kConsumers = 8;
 constexpr int kStagers = 1 + kConsumers;   // warps that fill the first x slot
-constexpr int kThreads = 32 * (2 + kConsumers);
+constexpr int kSzWarps = 2;                // scale/zero stagers, 64 rows each
+constexpr int kFirstConsumer = 2 + kSzWarps;  // warps: loader, x stager, scale/zero stagers
+constexpr int kThreads = 32 * (kFirstConsumer + kConsumers);
+constexpr int kSzBytes = 2 * kRows * 16;   // packed: fp16 scales + zeros of a stage
 constexpr int kMaxJobs = 168;
 constexpr int kMaxCtas = 160;
 constexpr int kMaxM = 4;
@@ -165,9 +168,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
 }
 __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-__device__ __forceinline__ void named_bar(int id, int threads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -368,132 +368,115 @@ __device__ __forceinline__ bool x_enter(XCursor &c, const StreamJob &J, bool fir
     return true;
 }
 
-// Cross-window sums: the window-1 warp of a row group hands its 16 row
-// partials to the window-0 warp through smem, double-buffered by unit, with
-// an mbarrier pair per buffer (bounded waits, so a warp that stops early on
-// an abort leaves no partner blocked).
-struct Xchg {
-    float *base;       // [8 row groups][2 parity][16 rows][kMaxM]
-    uint64_t *bars;    // [8 row groups][2 parity] {full, empty}
-    __device__ __forceinline__ float *slot(int rg, int parity, int r16) const {
-        return base + ((rg * 2 + parity) * 16 + r16) * kMaxM;
-    }
-    __device__ __forceinline__ uint32_t bar(int rg, int parity, int which) const {
-        return smem_u32(&bars[(rg * 2 + parity) * 2 + which]);
-    }
-    // window 1, unit n of this warp: wait until slot n&1 was read two units ago
-    __device__ __forceinline__ bool put_begin(int rg, uint32_t n, volatile int *ab) const {
-        return mbar_wait(bar(rg, n & 1, 1), ((n >> 1) & 1) ^ 1, ab);
-    }
-    __device__ __forceinline__ void put_end(int rg, uint32_t n, int lane) const {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(rg, n & 1, 0));
-    }
-    // window 0: wait for the partials of unit n, then hand the slot back
-    __device__ __forceinline__ bool get_begin(int rg, uint32_t n, volatile int *ab) const {
-        return mbar_wait(bar(rg, n & 1, 0), (n >> 1) & 1, ab);
-    }
-    __device__ __forceinline__ void get_end(int rg, uint32_t n, int lane) const {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(rg, n & 1, 1));
-    }
-};
-
 // Stage / unit walk shared by the consumers.
 struct Walk {
     int u, kc, jidx, sidx;
     uint32_t sph;
-};
-// A second walk, two stages ahead, tells which scales and zeros to prefetch
-// (it stays on the last stage of the range once it gets there).  It keeps
-// this lane's two scale rows and two zero rows as pointers, renewed once per
-// unit, so a fetch is four loads.  Rows past N are clamped to the last row:
-// they only feed outputs that are never stored.
-struct Ahead {
-    int u, kc, j, G;
-    const unsigned short *s0, *s1, *z0, *z1;
-    __device__ __forceinline__ void rows(const StreamJob *jobs, int ra) {
-        const StreamJob &J = jobs[j];
-        G = J.K >> 6;
-        const int r = (u - J.unit_begin) * kRows + ra;
-        const int64_t b0 = (int64_t)min(r, J.N - 1) * G, b1 = (int64_t)min(r + 8, J.N - 1) * G;
-        s0 = reinterpret_cast<const unsigned short *>(J.s) + b0;
-        s1 = reinterpret_cast<const unsigned short *>(J.s) + b1;
-        z0 = reinterpret_cast<const unsigned short *>(J.z) + b0;
-        z1 = reinterpret_cast<const unsigned short *>(J.z) + b1;
-    }
-    __device__ __forceinline__ void start(const StreamJob *jobs, int u0, int j0, int ra) {
-        u = u0;
-        kc = 0;
-        j = j0;
-        rows(jobs, ra);
-    }
-    __device__ __forceinline__ void advance(const StreamJob *jobs, int count, int u1, int ra) {
-        if (++kc == kchunks_of<true>(jobs[j].K)) {
-            if (u + 1 >= u1) {
-                --kc;
-                return;
-            }
-            kc = 0;
-            ++u;
-            j = next_job(jobs, count, j, u);
-            rows(jobs, ra);
+    // the stage after this one; false at the end of the range
+    __device__ __forceinline__ bool next(const StreamJob *jobs, int count, int u1, int kch,
+                                         int S, Walk &n) const {
+        n = *this;
+        if (++n.kc == kch) {
+            n.kc = 0;
+            if (++n.u >= u1) return false;
+            n.jidx = next_job(jobs, count, jidx, n.u);
         }
+        if (++n.sidx == S) {
+            n.sidx = 0;
+            n.sph ^= 1;
+        }
+        return true;
     }
 };
-
-// This lane's fp16 scales and zeros for one stage: rows ra and ra+8 of the
-// unit, NG consecutive groups from 8*kc + gw, packed in pairs (g, g+1).
-// Issued two stages before use so the loads are in flight while the stages
-// in between are consumed.  Groups are clamped into the row instead of
-// predicated, so the loads go straight into the registers read two stages
-// later; a group past K/64 multiplies an exactly zero code sum and
-// activation sum.
-template <int NG>
-struct SzRegs {
-    uint32_t s[2][NG / 2], z[2][NG / 2];
+// ---- packed: scales and zeros through shared memory ----------------------------
+// Warp 2 copies the fp16 scales and zeros of each stage (rows r0..r0+127,
+// groups 8kc..8kc+7) into a ring slot beside the weight stage: s[128][8] then
+// z[128][8].  Lane l takes 16-byte row slice word l&3 of rows l/4 + 8i, so a
+// load instruction reads eight whole 16-byte slices.  Loads run one stage
+// ahead of the stores (two register sets), their indices clamped into the
+// matrix so no load waits on a predicate; positions past N or K/64 are stored
+// as zero once the values are in.  The warp runs ahead of the consumers by
+// the ring depth, and the loader has prefetched each unit's scale/zero block
+// into L2, so one stage of load look-ahead suffices.
+struct SzSet {
+    uint32_t s[8], z[8];
 };
-template <int NG>
-__device__ __forceinline__ void fetch_sz(const Ahead &a, int gw, SzRegs<NG> &o) {
-    const int g = 8 * a.kc + gw;
+struct SzWalk {
+    int u, kc, j;
+    __device__ __forceinline__ bool next(const StreamJob *jobs, int count, int u1) {
+        if (++kc == kchunks_of<true>(jobs[j].K)) {
+            kc = 0;
+            if (++u >= u1) return false;
+            j = next_job(jobs, count, j, u);
+        }
+        return true;
+    }
+};
+__device__ __forceinline__ void sz_issue(const StreamJob *jobs, const SzWalk &a, int half,
+                                         int lane, SzSet &o) {
+    const StreamJob &J = jobs[a.j];
+    const int G = J.K >> 6;
+    const int r0 = (a.u - J.unit_begin) * kRows + 64 * half + (lane >> 2);
+    const int c = lane & 3;
+    const unsigned short *S16 = reinterpret_cast<const unsigned short *>(J.s);
+    const unsigned short *Z16 = reinterpret_cast<const unsigned short *>(J.z);
+    if ((G & 1) == 0) {
+        const int g = min(8 * a.kc + 2 * c, G - 2);
 #pragma unroll
-    for (int p = 0; p < NG / 2; ++p) {
-        if ((a.G & 1) == 0) {         // pair (gg, gg+1) is 4-byte aligned
-            const int gg = min(g + 2 * p, a.G - 2);
-            o.s[0][p] = __ldg(reinterpret_cast<const uint32_t *>(a.s0 + gg));
-            o.s[1][p] = __ldg(reinterpret_cast<const uint32_t *>(a.s1 + gg));
-            o.z[0][p] = __ldg(reinterpret_cast<const uint32_t *>(a.z0 + gg));
-            o.z[1][p] = __ldg(reinterpret_cast<const uint32_t *>(a.z1 + gg));
-        } else {
-            const int g0 = min(g + 2 * p, a.G - 1), g1 = min(g + 2 * p + 1, a.G - 1);
-            o.s[0][p] = (uint32_t)__ldg(a.s0 + g0) | ((uint32_t)__ldg(a.s0 + g1) << 16);
-            o.s[1][p] = (uint32_t)__ldg(a.s1 + g0) | ((uint32_t)__ldg(a.s1 + g1) << 16);
-            o.z[0][p] = (uint32_t)__ldg(a.z0 + g0) | ((uint32_t)__ldg(a.z0 + g1) << 16);
-            o.z[1][p] = (uint32_t)__ldg(a.z1 + g0) | ((uint32_t)__ldg(a.z1 + g1) << 16);
+        for (int i = 0; i < 8; ++i) {
+            const int64_t off = (int64_t)min(r0 + 8 * i, J.N - 1) * G + g;
+            o.s[i] = __ldg(reinterpret_cast<const uint32_t *>(S16 + off));
+            o.z[i] = __ldg(reinterpret_cast<const uint32_t *>(Z16 + off));
+        }
+    } else {        // rows only 2-byte aligned: two halves per word
+        const int g0 = min(8 * a.kc + 2 * c, G - 1), g1 = min(8 * a.kc + 2 * c + 1, G - 1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int64_t off = (int64_t)min(r0 + 8 * i, J.N - 1) * G;
+            o.s[i] = (uint32_t)__ldg(S16 + off + g0) | ((uint32_t)__ldg(S16 + off + g1) << 16);
+            o.z[i] = (uint32_t)__ldg(Z16 + off + g0) | ((uint32_t)__ldg(Z16 + off + g1) << 16);
         }
     }
 }
-
-// Window 0 folds window 1's partial row sums of a unit into y one unit
-// later, when they are long written, instead of waiting at the unit's end.
-struct PendingY {
-    bool on = false;
-    uint32_t n = 0;            // unit index (this warp's count) it belongs to
-    float *ya = nullptr;       // y + row of this lane's first row (or null)
-    float *yb = nullptr;       // ... second row (or null)
-    float va[kMaxM / 2 + 1], vb[kMaxM / 2 + 1];
-};
+__device__ __forceinline__ void sz_store(const StreamJob *jobs, const SzWalk &a, int half,
+                                         int lane, const SzSet &v, uint8_t *slot) {
+    const StreamJob &J = jobs[a.j];
+    const int G = J.K >> 6;
+    const int rl = 64 * half + (lane >> 2), c = lane & 3;
+    const int r0 = (a.u - J.unit_begin) * kRows + rl;
+    const int g = 8 * a.kc + 2 * c;
+    const uint32_t gmask = g + 1 < G ? 0xffffffffu : (g < G ? 0x0000ffffu : 0u);
+    uint32_t *ss = reinterpret_cast<uint32_t *>(slot) + rl * 4 + c;
+    uint32_t *zz = reinterpret_cast<uint32_t *>(slot + kSzBytes / 2) + rl * 4 + c;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t m = r0 + 8 * i < J.N ? gmask : 0u;
+        ss[32 * i] = v.s[i] & m;
+        zz[32 * i] = v.z[i] & m;
+    }
+}
 
 // ---- packed consumer, one x row: block-diagonal groups ---------------------------
-// mma p of a step pairs window units (p, p+4): slots 0-15 take unit p's codes
-// and B columns 0-3, slots 16-31 unit p+4's and columns 4-7.  Units (0,4) and
-// (1,5) belong to groups (0,2), units (2,6) and (3,7) to groups (1,3).
+// Warp rg owns rows 16rg..16rg+15 of each unit and both 128-byte windows of a
+// stage.  In window w, mma p pairs units (p, p+4): slots 0-15 take unit p's
+// codes and B columns 0-3, slots 16-31 unit p+4's and columns 4-7.  Units
+// (0,4) and (1,5) belong to groups (0,2), units (2,6) and (3,7) to groups
+// (1,3).
+//
+// The loop is software-pipelined by one stage: a step releases stage n, waits
+// for stage n+1 and issues its ldmatrix loads, and only then runs stage n's
+// tensor-core math and epilogue, so the wait and load latency of one stage
+// hide behind the arithmetic of the other.  A step reads the activation slot
+// only for its own stage, before the next stage may move to another slot.
+struct StageA {
+    uint32_t R[2][4][4];   // [window][j] ldmatrix fragments
+    uint32_t s[2][2], z[2][2];   // [row ra / ra+8][window] fp16 pair (2eh, 2eh+1)
+};
 __device__ __forceinline__ void consume_packed_m1(
-    const StreamParams &P, const StreamJob *jobs, uint8_t *smem, uint8_t *xslots,
-    uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
-    volatile int *abort_flag, const Xchg &xg, int u0, int u1, int cw, int lane) {
+    const StreamParams &P, const StreamJob *jobs, uint8_t *smem, const uint8_t *szring,
+    uint8_t *xslots, uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
+    volatile int *abort_flag, int u0, int u1, int rg, int lane) {
     const int S = P.stages;
-    const int rg = cw & 7, w = cw >> 3;
     const int gq = lane >> 2, t = lane & 3;
     // ldmatrix: this lane gives the address of row lrow of unit (j + 4*(lane>>4))
     const int lrow = 16 * rg + (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -504,131 +487,100 @@ __device__ __forceinline__ void consume_packed_m1(
     // B role: column gq = 4*bh + digit bd
     const int bh = gq >> 2, bd = gq & 3;
     const uint32_t m0 = bh ? 0u : 0xffffffffu, m1 = ~m0;
-    // epilogue role: groups 2*eh (+1), digit pair ep
+    // epilogue role: groups 2*eh (+1) of each window, digit pair ep
     const int eh = t >> 1, ep = t & 1;
     const int ra = 16 * rg + gq;
     XCursor xc;
     Walk k{u0, 0, find_job(jobs, P.count, u0), 0, 0u};
-    Ahead ah;
-    ah.start(jobs, u0, k.jidx, ra);
-    SzRegs<2> sz0, sz1, sz2;
-    fetch_sz<2>(ah, 4 * w + 2 * eh, sz0);
-    ah.advance(jobs, P.count, u1, ra);
-    fetch_sz<2>(ah, 4 * w + 2 * eh, sz1);
-    ah.advance(jobs, P.count, u1, ra);
     float ya = 0.0f, yb = 0.0f;
-    int parity = 0;
-    uint32_t nunit = 0;
-    PendingY pend;
-    // window 0: add window 1's partials of the pending unit and store
-    auto flush = [&]() -> bool {
-        if (!pend.on) return true;
-        if (!xg.get_begin(rg, pend.n, abort_flag)) return false;
-        if (t == 0) {
-            if (pend.ya) *pend.ya = pend.va[0] + xg.slot(rg, pend.n & 1, gq)[0];
-            if (pend.yb) *pend.yb = pend.vb[0] + xg.slot(rg, pend.n & 1, gq + 8)[0];
+    auto load = [&](StageA &r, int s, uint32_t ph) -> bool {
+        if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) return false;
+        const uint32_t box = smem_u32(smem + s * kStageBytes);
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) ldsm_x4(box + w * kBoxBytes + a_off[j], r.R[w][j]);
+        const uint8_t *sz = szring + s * kSzBytes + ra * 16 + 4 * eh;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            r.s[0][w] = *reinterpret_cast<const uint32_t *>(sz + 8 * w);
+            r.s[1][w] = *reinterpret_cast<const uint32_t *>(sz + 128 + 8 * w);
+            r.z[0][w] = *reinterpret_cast<const uint32_t *>(sz + kSzBytes / 2 + 8 * w);
+            r.z[1][w] = *reinterpret_cast<const uint32_t *>(sz + kSzBytes / 2 + 128 + 8 * w);
         }
-        xg.get_end(rg, pend.n, lane);
-        pend.on = false;
         return true;
     };
-    // One stage; `use` holds its scales/zeros, `fill` receives those of the
-    // stage two ahead.  Returns true when this warp is done.
-    auto step = [&](const SzRegs<2> &use, SzRegs<2> &fill) -> bool {
-        fetch_sz<2>(ah, 4 * w + 2 * eh, fill);
-        ah.advance(jobs, P.count, u1, ra);
+    if (!x_enter(xc, jobs[k.jidx], true, xslots, P.xslot_bytes, xfull, xempty, abort_flag, lane))
+        return;
+    StageA stA, stB;
+    if (!load(stA, 0, 0u)) return;
+    // One step on `cur` (loaded); `nxt` receives the next stage's fragments.
+    // Returns true when this warp is done.
+    auto step = [&](StageA &cur, StageA &nxt) -> bool {
         const StreamJob &J = jobs[k.jidx];
-        if (k.kc == 0 && !x_enter(xc, J, k.u == u0, xslots, P.xslot_bytes, xfull, xempty,
-                                  abort_flag, lane))
-            return true;
         const int kch = kchunks_of<true>(J.K);
-        const int rs = dig_rs(kch);
-        const int s = k.sidx;
-        if (!mbar_wait(smem_u32(&full[s]), k.sph, abort_flag)) return true;
-        const uint32_t box = smem_u32(smem + s * kStageBytes + w * kBoxBytes);
-        uint32_t R[4][4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) ldsm_x4(box + a_off[j], R[j]);
-        const uint32_t *xd = reinterpret_cast<const uint32_t *>(xc.xs) + (bd * 4 + t) * rs +
-                             2 * (16 * k.kc + 8 * w + 4 * bh);
-        const uint4 Q0 = *reinterpret_cast<const uint4 *>(xd);
-        const uint4 Q1 = *reinterpret_cast<const uint4 *>(xd + 4);
-        const float4 tb = *reinterpret_cast<const float4 *>(
-            xc.xs + 64 * rs + 8 * (ep * 8 * kch + 8 * k.kc + 4 * w + 2 * eh));
-        uint32_t lo[4][4], hi[4][4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                lo[j][i] = R[j][i] & 0x0F0F0F0Fu;
-                hi[j][i] = R[j][i] & 0xF0F0F0F0u;
-            }
+        // stage released: the arrive's release semantics order this warp's
+        // ldmatrix reads (made visible to lane 0 by the warp sync) before it
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty[s]));   // stage consumed
-        int CA[4] = {0, 0, 0, 0}, CB[4] = {0, 0, 0, 0};
-        mma_i8(CA, lo[0][0], lo[0][1], lo[0][2], lo[0][3], Q0.x & m0, Q0.x & m1);
-        mma_i8(CB, lo[2][0], lo[2][1], lo[2][2], lo[2][3], Q1.x & m0, Q1.x & m1);
-        mma_i8(CA, hi[0][0], hi[0][1], hi[0][2], hi[0][3], Q0.y & m0, Q0.y & m1);
-        mma_i8(CB, hi[2][0], hi[2][1], hi[2][2], hi[2][3], Q1.y & m0, Q1.y & m1);
-        mma_i8(CA, lo[1][0], lo[1][1], lo[1][2], lo[1][3], Q0.z & m0, Q0.z & m1);
-        mma_i8(CB, lo[3][0], lo[3][1], lo[3][2], lo[3][3], Q1.z & m0, Q1.z & m1);
-        mma_i8(CA, hi[1][0], hi[1][1], hi[1][2], hi[1][3], Q0.w & m0, Q0.w & m1);
-        mma_i8(CB, hi[3][0], hi[3][1], hi[3][2], hi[3][3], Q1.w & m0, Q1.w & m1);
-        // this lane: digits (2ep, 2ep+1) of rows ra, ra+8 for groups 2eh (A), 2eh+1 (B)
-        const float2 sa = half2_bits_to_float2(use.s[0][0]), sb = half2_bits_to_float2(use.s[1][0]);
-        const float2 za = half2_bits_to_float2(use.z[0][0]), zb = half2_bits_to_float2(use.z[1][0]);
-        const float vAa = (float)(CA[0] + 256 * CA[1]), vAb = (float)(CA[2] + 256 * CA[3]);
-        const float vBa = (float)(CB[0] + 256 * CB[1]), vBb = (float)(CB[2] + 256 * CB[3]);
-        ya = fmaf(sa.x, fmaf(tb.x, vAa, -za.x * tb.y), ya);
-        yb = fmaf(sb.x, fmaf(tb.x, vAb, -zb.x * tb.y), yb);
-        ya = fmaf(sa.y, fmaf(tb.z, vBa, -za.y * tb.w), ya);
-        yb = fmaf(sb.y, fmaf(tb.z, vBb, -zb.y * tb.w), yb);
-
-        int nu = k.u, nkc = k.kc + 1, nj = k.jidx;
-        if (nkc == kch) {
-            nu = k.u + 1;
-            nkc = 0;
-            if (nu < u1) nj = next_job(jobs, P.count, k.jidx, nu);
+        if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));
+        Walk n;
+        const bool more = k.next(jobs, P.count, u1, kch, S, n);
+        if (more && !load(nxt, n.sidx, n.sph)) return true;
+        const int rs = dig_rs(kch);
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            // activation digits and (f, X~) of this window
+            const uint32_t *xd = reinterpret_cast<const uint32_t *>(xc.xs) + (bd * 4 + t) * rs +
+                                 2 * (16 * k.kc + 8 * w + 4 * bh);
+            const uint4 Q0 = *reinterpret_cast<const uint4 *>(xd);
+            const uint4 Q1 = *reinterpret_cast<const uint4 *>(xd + 4);
+            const float4 tb = *reinterpret_cast<const float4 *>(
+                xc.xs + 64 * rs + 8 * (ep * 8 * kch + 8 * k.kc + 4 * w + 2 * eh));
+            int CA[4] = {0, 0, 0, 0}, CB[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                int (&C)[4] = j < 2 ? CA : CB;
+                const uint4 &Q = j < 2 ? Q0 : Q1;
+                const uint32_t bl = (j & 1) ? Q.z : Q.x, bu = (j & 1) ? Q.w : Q.y;
+                const uint32_t(&R)[4] = cur.R[w][j];
+                mma_i8(C, R[0] & 0x0F0F0F0Fu, R[1] & 0x0F0F0F0Fu, R[2] & 0x0F0F0F0Fu,
+                       R[3] & 0x0F0F0F0Fu, bl & m0, bl & m1);
+                mma_i8(C, R[0] & 0xF0F0F0F0u, R[1] & 0xF0F0F0F0u, R[2] & 0xF0F0F0F0u,
+                       R[3] & 0xF0F0F0F0u, bu & m0, bu & m1);
+            }
+            // digits (2ep, 2ep+1) of rows ra, ra+8 for groups 4w+2eh (A) and +1 (B)
+            const float2 sa = half2_bits_to_float2(cur.s[0][w]);
+            const float2 sb = half2_bits_to_float2(cur.s[1][w]);
+            const float2 za = half2_bits_to_float2(cur.z[0][w]);
+            const float2 zb = half2_bits_to_float2(cur.z[1][w]);
+            const float vAa = (float)(CA[0] + 256 * CA[1]), vAb = (float)(CA[2] + 256 * CA[3]);
+            const float vBa = (float)(CB[0] + 256 * CB[1]), vBb = (float)(CB[2] + 256 * CB[3]);
+            ya = fmaf(sa.x, fmaf(tb.x, vAa, -za.x * tb.y), ya);
+            yb = fmaf(sb.x, fmaf(tb.x, vAb, -zb.x * tb.y), yb);
+            ya = fmaf(sa.y, fmaf(tb.z, vBa, -za.y * tb.w), ya);
+            yb = fmaf(sb.y, fmaf(tb.z, vBb, -zb.y * tb.w), yb);
         }
-        if (nkc == 0) {       // unit done: four lanes per row, then two windows
+        if (n.kc == 0 || !more) {      // unit done: four lanes per row
             ya += __shfl_xor_sync(0xffffffffu, ya, 1);
             ya += __shfl_xor_sync(0xffffffffu, ya, 2);
             yb += __shfl_xor_sync(0xffffffffu, yb, 1);
             yb += __shfl_xor_sync(0xffffffffu, yb, 2);
-            if (w == 1) {
-                if (!xg.put_begin(rg, nunit, abort_flag)) return true;
-                if (t == 0) {
-                    xg.slot(rg, parity, gq)[0] = ya;
-                    xg.slot(rg, parity, gq + 8)[0] = yb;
-                }
-                xg.put_end(rg, nunit, lane);
-            } else {
-                if (!flush()) return true;
+            if (t == 0) {
                 const int r0 = (k.u - J.unit_begin) * kRows;
-                pend.on = true;
-                pend.n = nunit;
-                pend.ya = r0 + ra < J.N ? J.y + r0 + ra : nullptr;
-                pend.yb = r0 + ra + 8 < J.N ? J.y + r0 + ra + 8 : nullptr;
-                pend.va[0] = ya;
-                pend.vb[0] = yb;
+                if (r0 + ra < J.N) J.y[r0 + ra] = ya;
+                if (r0 + ra + 8 < J.N) J.y[r0 + ra + 8] = yb;
             }
             ya = yb = 0.0f;
-            parity ^= 1;
-            ++nunit;
         }
-        if (nu >= u1) return true;
-        k.u = nu;
-        k.kc = nkc;
-        k.jidx = nj;
-        if (++k.sidx == S) {      // ring position of the next stage
-            k.sidx = 0;
-            k.sph ^= 1;
-        }
+        if (!more) return true;
+        if (n.kc == 0 && !x_enter(xc, jobs[n.jidx], false, xslots, P.xslot_bytes, xfull,
+                                  xempty, abort_flag, lane))
+            return true;
+        k = n;
         return false;
     };
-    while (!step(sz0, sz2) && !step(sz1, sz0) && !step(sz2, sz1)) {
+    while (!step(stA, stB) && !step(stB, stA)) {
     }
-    if (w == 0) flush();
 }
 
 // ---- packed consumer, 2 or 4 x rows ------------------------------------------------
@@ -636,12 +588,11 @@ __device__ __forceinline__ void consume_packed_m1(
 // x rows as B columns (row 2*mp + h in columns 4h..4h+3).
 template <int MT>
 __device__ __forceinline__ void consume_packed_mx(
-    const StreamParams &P, const StreamJob *jobs, uint8_t *smem, uint8_t *xslots,
-    uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
-    volatile int *abort_flag, const Xchg &xg, int u0, int u1, int cw, int lane) {
+    const StreamParams &P, const StreamJob *jobs, uint8_t *smem, const uint8_t *szring,
+    uint8_t *xslots, uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
+    volatile int *abort_flag, int u0, int u1, int rg, int lane) {
     constexpr int MP = MT / 2;
     const int S = P.stages;
-    const int rg = cw & 7, w = cw >> 3;
     const int gq = lane >> 2, t = lane & 3;
     // ldmatrix: this lane gives the address of row lrow of unit (2j + (lane>>4))
     const int lrow = 16 * rg + (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -654,299 +605,298 @@ __device__ __forceinline__ void consume_packed_mx(
     const int ra = 16 * rg + gq;
     XCursor xc;
     Walk k{u0, 0, find_job(jobs, P.count, u0), 0, 0u};
-    Ahead ah;
-    ah.start(jobs, u0, k.jidx, ra);
-    SzRegs<4> sz0, sz1, sz2;
-    fetch_sz<4>(ah, 4 * w, sz0);
-    ah.advance(jobs, P.count, u1, ra);
-    fetch_sz<4>(ah, 4 * w, sz1);
-    ah.advance(jobs, P.count, u1, ra);
     float ya[MP], yb[MP];
 #pragma unroll
     for (int p = 0; p < MP; ++p) ya[p] = yb[p] = 0.0f;
-    int parity = 0;
-    uint32_t nunit = 0;
-    auto step = [&](const SzRegs<4> &use, SzRegs<4> &fill) -> bool {
-        fetch_sz<4>(ah, 4 * w, fill);
-        ah.advance(jobs, P.count, u1, ra);
+    if (!x_enter(xc, jobs[k.jidx], true, xslots, P.xslot_bytes, xfull, xempty, abort_flag, lane))
+        return;
+    auto step = [&]() -> bool {
         const StreamJob &J = jobs[k.jidx];
-        if (k.kc == 0 && !x_enter(xc, J, k.u == u0, xslots, P.xslot_bytes, xfull, xempty,
-                                  abort_flag, lane))
-            return true;
         const int kch = kchunks_of<true>(J.K);
         const int rs = dig_rs(kch);
         const int mb = xrow_bytes<true>(J.K);
-        const int s = k.sidx;
-        if (!mbar_wait(smem_u32(&full[s]), k.sph, abort_flag)) return true;
-        const uint32_t box = smem_u32(smem + s * kStageBytes + w * kBoxBytes);
-        uint32_t R[4][4];
+        if (!mbar_wait(smem_u32(&full[k.sidx]), k.sph, abort_flag)) return true;
+        const uint32_t box0 = smem_u32(smem + k.sidx * kStageBytes);
+        // scales / zeros of rows ra, ra+8, groups 4w..4w+3 of both windows
+        uint2 su[2][2], zu[2][2];
+        {
+            const uint8_t *sz = szring + k.sidx * kSzBytes + ra * 16;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) ldsm_x4(box + a_off[j], R[j]);
-        uint32_t lo[4][4], hi[4][4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                lo[j][i] = R[j][i] & 0x0F0F0F0Fu;
-                hi[j][i] = R[j][i] & 0xF0F0F0F0u;
-            }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty[s]));   // stage consumed
-        float sa[4], sb[4], za[4], zb[4];
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const float2 a2 = half2_bits_to_float2(use.s[0][p]), b2 = half2_bits_to_float2(use.s[1][p]);
-            const float2 c2 = half2_bits_to_float2(use.z[0][p]), d2 = half2_bits_to_float2(use.z[1][p]);
-            sa[2 * p] = a2.x; sa[2 * p + 1] = a2.y;
-            sb[2 * p] = b2.x; sb[2 * p + 1] = b2.y;
-            za[2 * p] = c2.x; za[2 * p + 1] = c2.y;
-            zb[2 * p] = d2.x; zb[2 * p + 1] = d2.y;
-        }
-#pragma unroll
-        for (int mp = 0; mp < MP; ++mp) {
-            // B: this lane's words for units 0..7 of the window, both parities
-            const uint32_t *xd = reinterpret_cast<const uint32_t *>(xc.xs + (2 * mp + bh) * mb) +
-                                 (bd * 4 + t) * rs + 2 * (16 * k.kc + 8 * w);
-            uint4 Q[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) Q[j] = reinterpret_cast<const uint4 *>(xd)[j];
-            int C[4][4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                C[j][0] = C[j][1] = C[j][2] = C[j][3] = 0;
-                mma_i8(C[j], lo[j][0], lo[j][1], hi[j][0], hi[j][1], Q[j].x, Q[j].y);
-                mma_i8(C[j], lo[j][2], lo[j][3], hi[j][2], hi[j][3], Q[j].z, Q[j].w);
-            }
-            const float *tb = reinterpret_cast<const float *>(
-                xc.xs + (2 * mp + eh) * mb + 64 * rs + 8 * (ep * 8 * kch + 8 * k.kc + 4 * w));
-            const float4 t01 = reinterpret_cast<const float4 *>(tb)[0];
-            const float4 t23 = reinterpret_cast<const float4 *>(tb)[1];
-            const float f[4] = {t01.x, t01.z, t23.x, t23.z};
-            const float X[4] = {t01.y, t01.w, t23.y, t23.w};
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                const float va = (float)(C[g][0] + 256 * C[g][1]);
-                const float vb = (float)(C[g][2] + 256 * C[g][3]);
-                ya[mp] = fmaf(sa[g], fmaf(f[g], va, -za[g] * X[g]), ya[mp]);
-                yb[mp] = fmaf(sb[g], fmaf(f[g], vb, -zb[g] * X[g]), yb[mp]);
+            for (int w = 0; w < 2; ++w) {
+                su[0][w] = *reinterpret_cast<const uint2 *>(sz + 8 * w);
+                su[1][w] = *reinterpret_cast<const uint2 *>(sz + 128 + 8 * w);
+                zu[0][w] = *reinterpret_cast<const uint2 *>(sz + kSzBytes / 2 + 8 * w);
+                zu[1][w] = *reinterpret_cast<const uint2 *>(sz + kSzBytes / 2 + 128 + 8 * w);
             }
         }
-
-        int nu = k.u, nkc = k.kc + 1, nj = k.jidx;
-        if (nkc == kch) {
-            nu = k.u + 1;
-            nkc = 0;
-            if (nu < u1) nj = next_job(jobs, P.count, k.jidx, nu);
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            uint32_t R[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) ldsm_x4(box0 + w * kBoxBytes + a_off[j], R[j]);
+            uint32_t lo[4][4], hi[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    lo[j][i] = R[j][i] & 0x0F0F0F0Fu;
+                    hi[j][i] = R[j][i] & 0xF0F0F0F0u;
+                }
+            if (w == 1) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));   // stage consumed
+            }
+            float sa[4], sb[4], za[4], zb[4];
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const float2 a2 = half2_bits_to_float2(p ? su[0][w].y : su[0][w].x);
+                const float2 b2 = half2_bits_to_float2(p ? su[1][w].y : su[1][w].x);
+                const float2 c2 = half2_bits_to_float2(p ? zu[0][w].y : zu[0][w].x);
+                const float2 d2 = half2_bits_to_float2(p ? zu[1][w].y : zu[1][w].x);
+                sa[2 * p] = a2.x; sa[2 * p + 1] = a2.y;
+                sb[2 * p] = b2.x; sb[2 * p + 1] = b2.y;
+                za[2 * p] = c2.x; za[2 * p + 1] = c2.y;
+                zb[2 * p] = d2.x; zb[2 * p + 1] = d2.y;
+            }
+#pragma unroll
+            for (int mp = 0; mp < MP; ++mp) {
+                // B: this lane's words for units 0..7 of the window, both parities
+                const uint32_t *xd =
+                    reinterpret_cast<const uint32_t *>(xc.xs + (2 * mp + bh) * mb) +
+                    (bd * 4 + t) * rs + 2 * (16 * k.kc + 8 * w);
+                uint4 Q[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) Q[j] = reinterpret_cast<const uint4 *>(xd)[j];
+                int C[4][4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    C[j][0] = C[j][1] = C[j][2] = C[j][3] = 0;
+                    mma_i8(C[j], lo[j][0], lo[j][1], hi[j][0], hi[j][1], Q[j].x, Q[j].y);
+                    mma_i8(C[j], lo[j][2], lo[j][3], hi[j][2], hi[j][3], Q[j].z, Q[j].w);
+                }
+                const float *tb = reinterpret_cast<const float *>(
+                    xc.xs + (2 * mp + eh) * mb + 64 * rs + 8 * (ep * 8 * kch + 8 * k.kc + 4 * w));
+                const float4 t01 = reinterpret_cast<const float4 *>(tb)[0];
+                const float4 t23 = reinterpret_cast<const float4 *>(tb)[1];
+                const float f[4] = {t01.x, t01.z, t23.x, t23.z};
+                const float X[4] = {t01.y, t01.w, t23.y, t23.w};
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const float va = (float)(C[g][0] + 256 * C[g][1]);
+                    const float vb = (float)(C[g][2] + 256 * C[g][3]);
+                    ya[mp] = fmaf(sa[g], fmaf(f[g], va, -za[g] * X[g]), ya[mp]);
+                    yb[mp] = fmaf(sb[g], fmaf(f[g], vb, -zb[g] * X[g]), yb[mp]);
+                }
+            }
         }
-        if (nkc == 0) {       // unit done: two lanes per row and x row, then two windows
+        Walk n;
+        const bool more = k.next(jobs, P.count, u1, kch, S, n);
+        if (n.kc == 0 || !more) {      // unit done: two lanes per row and x row
+            const int r0 = (k.u - J.unit_begin) * kRows;
 #pragma unroll
             for (int mp = 0; mp < MP; ++mp) {
                 ya[mp] += __shfl_xor_sync(0xffffffffu, ya[mp], 1);
                 yb[mp] += __shfl_xor_sync(0xffffffffu, yb[mp], 1);
-            }
-            if (w == 1) {
-                if (!xg.put_begin(rg, nunit, abort_flag)) return true;
-                if (ep == 0) {
-#pragma unroll
-                    for (int mp = 0; mp < MP; ++mp) {
-                        xg.slot(rg, parity, gq)[2 * mp + eh] = ya[mp];
-                        xg.slot(rg, parity, gq + 8)[2 * mp + eh] = yb[mp];
-                    }
+                const int m = 2 * mp + eh;
+                if (ep == 0 && m < P.M) {
+                    if (r0 + ra < J.N) J.y[(int64_t)m * J.N + r0 + ra] = ya[mp];
+                    if (r0 + ra + 8 < J.N) J.y[(int64_t)m * J.N + r0 + ra + 8] = yb[mp];
                 }
-                xg.put_end(rg, nunit, lane);
-            } else {
-                if (!xg.get_begin(rg, nunit, abort_flag)) return true;
-                if (ep == 0) {
-                    const int r0 = (k.u - J.unit_begin) * kRows;
-#pragma unroll
-                    for (int mp = 0; mp < MP; ++mp) {
-                        const int m = 2 * mp + eh;
-                        if (m >= P.M) continue;
-                        if (r0 + ra < J.N)
-                            J.y[(int64_t)m * J.N + r0 + ra] =
-                                ya[mp] + xg.slot(rg, parity, gq)[m];
-                        if (r0 + ra + 8 < J.N)
-                            J.y[(int64_t)m * J.N + r0 + ra + 8] =
-                                yb[mp] + xg.slot(rg, parity, gq + 8)[m];
-                    }
-                }
-                xg.get_end(rg, nunit, lane);
+                ya[mp] = yb[mp] = 0.0f;
             }
-#pragma unroll
-            for (int mp = 0; mp < MP; ++mp) ya[mp] = yb[mp] = 0.0f;
-            parity ^= 1;
-            ++nunit;
         }
-        if (nu >= u1) return true;
-        k.u = nu;
-        k.kc = nkc;
-        k.jidx = nj;
-        if (++k.sidx == S) {
-            k.sidx = 0;
-            k.sph ^= 1;
-        }
+        if (!more) return true;
+        if (n.kc == 0 && !x_enter(xc, jobs[n.jidx], false, xslots, P.xslot_bytes, xfull,
+                                  xempty, abort_flag, lane))
+            return true;
+        k = n;
         return false;
     };
-    while (!step(sz0, sz2) && !step(sz1, sz0) && !step(sz2, sz1)) {
+    while (!step()) {
     }
 }
 
 // ---- runtime (RTN) consumer --------------------------------------------------
+// Warp rg owns rows 16rg..16rg+15; lane (row r16, half part) takes 32 of the
+// 64 k of each window, so a row's dot product is spread over two lanes.
 template <int MT>
 __device__ __forceinline__ void consume_runtime(
     const StreamParams &P, const StreamJob *jobs, uint8_t *smem, uint8_t *xslots,
     uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
-    volatile int *abort_flag, const Xchg &xg, int u0, int u1, int cw, int lane) {
+    volatile int *abort_flag, int u0, int u1, int rg, int lane) {
     const int S = P.stages;
-    const int rg = cw & 7, w = cw >> 3;
     const int r16 = lane >> 1, part = lane & 1;       // row in group, 32-k half
     const int rr = 16 * rg + r16;
     const float L = (float)((1 << P.bits) - 1);
     const bool pass = P.bits == 16;
     XCursor xc;
-    int u = u0, kc = 0, jidx = find_job(jobs, P.count, u);
-    int sidx = 0;              // stage slot and its mbarrier phase
-    uint32_t sph = 0;
-    auto load_sz = [&](const StreamJob &J, int uu, int kk, float &sv, float &zv) {
-        const int row = (uu - J.unit_begin) * kRows + rr;
-        const int k0 = kk * 128 + w * 64;
-        sv = 1.0f;
-        zv = 0.0f;
-        if (!pass && row < J.N && k0 < J.K) {
-            const int64_t gi = (int64_t)row * (J.K / J.group) + k0 / J.group;
-            sv = __ldg(reinterpret_cast<const float *>(J.s) + gi);
-            zv = __ldg(reinterpret_cast<const float *>(J.z) + gi);
+    Walk k{u0, 0, find_job(jobs, P.count, u0), 0, 0u};
+    // (scale, zero) of this lane's two windows for the current and next stage
+    auto load_sz = [&](const Walk &q, float4 &o) {
+        const StreamJob &J = jobs[q.jidx];
+        const int row = (q.u - J.unit_begin) * kRows + rr;
+        o = make_float4(1.0f, 0.0f, 1.0f, 0.0f);
+        if (pass || row >= J.N) return;
+        const float *Sf = reinterpret_cast<const float *>(J.s);
+        const float *Zf = reinterpret_cast<const float *>(J.z);
+        const int64_t gr = (int64_t)row * (J.K / J.group);
+        const int k0 = q.kc * 128;
+        if (k0 < J.K) {
+            o.x = __ldg(Sf + gr + k0 / J.group);
+            o.y = __ldg(Zf + gr + k0 / J.group);
+        }
+        if (k0 + 64 < J.K) {
+            o.z = __ldg(Sf + gr + (k0 + 64) / J.group);
+            o.w = __ldg(Zf + gr + (k0 + 64) / J.group);
         }
     };
-    float2 sz_a, sz_b = make_float2(1.0f, 0.0f);     // (scale, zero) ping-pong
-    load_sz(jobs[jidx], u, 0, sz_a.x, sz_a.y);
+    float4 sz_a, sz_b = make_float4(1.0f, 0.0f, 1.0f, 0.0f);
+    load_sz(k, sz_a);
     float yacc[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) yacc[m] = 0.0f;
-    int parity = 0;
-    uint32_t nunit = 0;
-    auto step = [&](const float2 use, float2 &fill) -> bool {
-        const float s_cur = use.x, z_cur = use.y;
-        const StreamJob &J = jobs[jidx];
-        const int row = (u - J.unit_begin) * kRows + rr;
-        if (kc == 0 && !x_enter(xc, J, u == u0, xslots, P.xslot_bytes, xfull,
-                                xempty, abort_flag, lane))
-            return true;
+    if (!x_enter(xc, jobs[k.jidx], true, xslots, P.xslot_bytes, xfull, xempty, abort_flag, lane))
+        return;
+    auto step = [&](const float4 use, float4 &fill) -> bool {
+        const StreamJob &J = jobs[k.jidx];
+        const int row = (k.u - J.unit_begin) * kRows + rr;
         const int kchunks = kchunks_of<false>(J.K);
-        int nu = u, nkc = kc + 1, nj = jidx;
-        if (nkc == kchunks) {
-            nu = u + 1;
-            nkc = 0;
-            if (nu < u1) nj = next_job(jobs, P.count, jidx, nu);
-        }
-        if (nu < u1) load_sz(jobs[nj], nu, nkc, fill.x, fill.y);
-        const int s = sidx;
-        if (!mbar_wait(smem_u32(&full[s]), sph, abort_flag)) return true;
-        const int k0 = kc * 128 + w * 64 + part * 32;     // this thread's 32 k
-        float part_acc[MT];
+        Walk n;
+        const bool more = k.next(jobs, P.count, u1, kchunks, S, n);
+        if (more) load_sz(n, fill);
+        if (!mbar_wait(smem_u32(&full[k.sidx]), k.sph, abort_flag)) return true;
+        const uint8_t *stage = smem + k.sidx * kStageBytes;
+        const int kp = kpad_of<false>(J.K);
 #pragma unroll
-        for (int m = 0; m < MT; ++m) part_acc[m] = 0.0f;
-        if (row < J.N && k0 < J.K) {
-            const int kp = kpad_of<false>(J.K);
-            const uint8_t *box = smem + s * kStageBytes + w * kBoxBytes;
-            const float inv = rcp_approx(s_cur);
-            const float lo_c = -z_cur, hi_c = L - z_cur;
-            const float thr = 0.5f - (fmaxf(fabsf(lo_c), fabsf(hi_c)) + 2.0f) *
-                                         4.76837158203125e-07f;   // 2^-21
+        for (int w = 0; w < 2; ++w) {
+            const float s_cur = w ? use.z : use.x, z_cur = w ? use.w : use.y;
+            const int k0 = k.kc * 128 + w * 64 + part * 32;     // this thread's 32 k
+            float part_acc[MT];
 #pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) {
-                const int u16 = part * 4 + c8;
-                const uint4 raw = *reinterpret_cast<const uint4 *>(
-                    box + rr * 128 + ((u16 ^ (rr & 7)) << 4));
-                const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
-                float wv[8];
+            for (int m = 0; m < MT; ++m) part_acc[m] = 0.0f;
+            if (row < J.N && k0 < J.K) {
+                const uint8_t *box = stage + w * kBoxBytes;
+                const float inv = rcp_approx(s_cur);
+                const float lo_c = -z_cur, hi_c = L - z_cur;
+                const float thr = 0.5f - (fmaxf(fabsf(lo_c), fabsf(hi_c)) + 2.0f) *
+                                             4.76837158203125e-07f;   // 2^-21
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f2 = __half22float2(h2[i]);
-                    wv[2 * i] = f2.x;
-                    wv[2 * i + 1] = f2.y;
-                }
-                float cq[8];
-                if (pass) {
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    const int u16 = part * 4 + c8;
+                    const uint4 raw = *reinterpret_cast<const uint4 *>(
+                        box + rr * 128 + ((u16 ^ (rr & 7)) << 4));
+                    const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
+                    float wv[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) cq[i] = wv[i];
-                } else {
-                    float emax = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float v = fmaf(wv[i], inv, kMagic);
-                        const float r = v - kMagic;
-                        const float ee = fmaf(wv[i], inv, -r);
-                        emax = fmaxf(emax, fabsf(ee));
-                        cq[i] = fminf(fmaxf(r, lo_c), hi_c);
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 f2 = __half22float2(h2[i]);
+                        wv[2 * i] = f2.x;
+                        wv[2 * i + 1] = f2.y;
                     }
-                    if (emax > thr) {
+                    float cq[8];
+                    if (pass) {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            cq[i] = centered_code_exact(wv[i], s_cur, z_cur, L);
+                        for (int i = 0; i < 8; ++i) cq[i] = wv[i];
+                    } else {
+                        float emax = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float v = fmaf(wv[i], inv, kMagic);
+                            const float r = v - kMagic;
+                            const float ee = fmaf(wv[i], inv, -r);
+                            emax = fmaxf(emax, fabsf(ee));
+                            cq[i] = fminf(fmaxf(r, lo_c), hi_c);
+                        }
+                        if (emax > thr) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                cq[i] = centered_code_exact(wv[i], s_cur, z_cur, L);
+                        }
                     }
-                }
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    const float *xr = reinterpret_cast<const float *>(xc.xs) +
-                                      (int64_t)m * kp + k0 + c8 * 8;
-                    const float4 xa = *reinterpret_cast<const float4 *>(xr);
-                    const float4 xb = *reinterpret_cast<const float4 *>(xr + 4);
-                    float p = part_acc[m];
-                    p = fmaf(xa.x, cq[0], p);
-                    p = fmaf(xa.y, cq[1], p);
-                    p = fmaf(xa.z, cq[2], p);
-                    p = fmaf(xa.w, cq[3], p);
-                    p = fmaf(xb.x, cq[4], p);
-                    p = fmaf(xb.y, cq[5], p);
-                    p = fmaf(xb.z, cq[6], p);
-                    p = fmaf(xb.w, cq[7], p);
-                    part_acc[m] = p;
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
-#pragma unroll
-        for (int m = 0; m < MT; ++m) yacc[m] = fmaf(part_acc[m], s_cur, yacc[m]);
-        if (nkc == 0) {
-#pragma unroll
-            for (int m = 0; m < MT; ++m)
-                yacc[m] += __shfl_xor_sync(0xffffffffu, yacc[m], 1);
-            if (w == 1) {
-                if (!xg.put_begin(rg, nunit, abort_flag)) return true;
-                if (part == 0) {
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) xg.slot(rg, parity, r16)[m] = yacc[m];
-                }
-                xg.put_end(rg, nunit, lane);
-            } else {
-                if (!xg.get_begin(rg, nunit, abort_flag)) return true;
-                if (part == 0 && row < J.N) {
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
-                        if (m >= P.M) break;
-                        J.y[(int64_t)m * J.N + row] = yacc[m] + xg.slot(rg, parity, r16)[m];
+                        const float *xr = reinterpret_cast<const float *>(xc.xs) +
+                                          (int64_t)m * kp + k0 + c8 * 8;
+                        const float4 xa = *reinterpret_cast<const float4 *>(xr);
+                        const float4 xb = *reinterpret_cast<const float4 *>(xr + 4);
+                        float p = part_acc[m];
+                        p = fmaf(xa.x, cq[0], p);
+                        p = fmaf(xa.y, cq[1], p);
+                        p = fmaf(xa.z, cq[2], p);
+                        p = fmaf(xa.w, cq[3], p);
+                        p = fmaf(xb.x, cq[4], p);
+                        p = fmaf(xb.y, cq[5], p);
+                        p = fmaf(xb.z, cq[6], p);
+                        p = fmaf(xb.w, cq[7], p);
+                        part_acc[m] = p;
                     }
                 }
-                xg.get_end(rg, nunit, lane);
             }
 #pragma unroll
-            for (int m = 0; m < MT; ++m) yacc[m] = 0.0f;
-            parity ^= 1;
-            ++nunit;
+            for (int m = 0; m < MT; ++m) yacc[m] = fmaf(part_acc[m], s_cur, yacc[m]);
         }
-        if (nu >= u1) return true;
-        u = nu;
-        kc = nkc;
-        jidx = nj;
-        if (++sidx == S) {      // ring position of the next stage
-            sidx = 0;
-            sph ^= 1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));
+        if (n.kc == 0 || !more) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                yacc[m] += __shfl_xor_sync(0xffffffffu, yacc[m], 1);
+                if (part == 0 && row < J.N && m < P.M) J.y[(int64_t)m * J.N + row] = yacc[m];
+                yacc[m] = 0.0f;
+            }
         }
+        if (!more) return true;
+        if (n.kc == 0 && !x_enter(xc, jobs[n.jidx], false, xslots, P.xslot_bytes, xfull,
+                                  xempty, abort_flag, lane))
+            return true;
+        k = n;
         return false;
     };
     while (!step(sz_a, sz_b) && !step(sz_b, sz_a)) {
+    }
+}
+
+// Warp 2 of a packed launch: the scale / zero slice of every stage of the
+// CTA's range, in ring order, gated by the same empty barriers as the loader
+// and counted as a second arrival on each full barrier.
+__device__ __forceinline__ void sz_stager(const StreamParams &P, const StreamJob *jobs,
+                                       uint8_t *szring, uint64_t *full, uint64_t *empty,
+                                       volatile int *abort_flag, int u0, int u1, int half,
+                                       int lane) {
+    const int S = P.stages;
+    SzWalk st{u0, 0, find_job(jobs, P.count, u0)};   // stage stored next
+    SzWalk ld = st;                                     // stage loaded next
+    bool ld_ok = true;
+    SzSet A, B, C;
+    sz_issue(jobs, ld, half, lane, A);
+    ld_ok = ld.next(jobs, P.count, u1);
+    if (ld_ok) {
+        sz_issue(jobs, ld, half, lane, B);
+        ld_ok = ld.next(jobs, P.count, u1);
+    }
+    int sidx = 0;
+    uint32_t sph = 0;
+    // start the loads of the stage two later, then store `cur` (stage st)
+    auto step = [&](const SzSet &cur, SzSet &fill) -> bool {
+        if (ld_ok) {
+            sz_issue(jobs, ld, half, lane, fill);
+            ld_ok = ld.next(jobs, P.count, u1);
+        }
+        bool got = true;
+        if (lane == 0) got = mbar_wait(smem_u32(&empty[sidx]), sph ^ 1, abort_flag);
+        got = __shfl_sync(0xffffffffu, got, 0);
+        __syncwarp();
+        if (!got) return true;
+        sz_store(jobs, st, half, lane, cur, szring + sidx * kSzBytes);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&full[sidx]));
+        if (++sidx == S) {
+            sidx = 0;
+            sph ^= 1;
+        }
+        return !st.next(jobs, P.count, u1);
+    };
+    while (!step(A, C) && !step(B, A) && !step(C, B)) {
     }
 }
 
@@ -957,20 +907,20 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int S = P.stages;
-    uint8_t *xslots = smem + S * kStageBytes;
-    float *xchg = reinterpret_cast<float *>(xslots + 2 * P.xslot_bytes);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(xchg + 8 * 2 * 16 * kMaxM);
+    uint8_t *szring = smem + S * kStageBytes;
+    uint8_t *xslots = szring + (PACKED ? S * kSzBytes : 0);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(xslots + 2 * P.xslot_bytes);
     uint64_t *full = bars, *empty = bars + S;
     uint64_t *xfull = bars + 2 * S, *xempty = xfull + 2;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(xempty + 2);
-    uint64_t *xbars = bars + 2 * S + 8;                 // 8 row groups x 2 x {full, empty}
-    StreamJob *jobs = reinterpret_cast<StreamJob *>(bars + 2 * S + 8 + 32);
+    uint64_t *xfirst = xempty + 3;      // the first x slot is complete
+    StreamJob *jobs = reinterpret_cast<StreamJob *>(bars + 2 * S + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u0 = P.cta_begin[blockIdx.x], u1 = P.cta_begin[blockIdx.x + 1];
     // The activations of this CTA's matrices go to L2 ahead of the weight
     // stream: queued behind the first ring fill they would hold up the start.
-    if (warp >= 1 && u0 < u1) {
+    if (warp >= 1 && warp < 1 + kStagers && u0 < u1) {
         const int jf = find_job(P.jobs, P.count, u0), jl = find_job(P.jobs, P.count, u1 - 1);
         for (int j = jf; j <= jl; ++j) {
             const StreamJob &J = P.jobs[j];
@@ -989,14 +939,14 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&full[s]), PACKED ? 1 + kSzWarps : 1);
             mbar_init(smem_u32(&empty[s]), kConsumers);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&xfull[b]), 32);
             mbar_init(smem_u32(&xempty[b]), kConsumers);
         }
-        for (int b = 0; b < 32; ++b) mbar_init(smem_u32(&xbars[b]), 1);
+        mbar_init(smem_u32(xfirst), kStagers);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -1073,20 +1023,33 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
             }
         }
         __syncwarp();
+    } else if (warp >= 2 && warp < kFirstConsumer) {
+        // ---------------- scale / zero stagers (packed) ----------------
+        if constexpr (PACKED) {
+            if (u0 < u1) sz_stager(P, jobs, szring, full, empty, abort_flag, u0, u1, warp - 2, lane);
+        }
     } else {
-        // the first x slot, by every warp but the loader
+        // the first x slot, by the x stager and the consumers together; each
+        // warp reports on `xfirst`, and the stager turns that into the slot's
+        // first xfull phase once all have
+        bool first_ok = true;
         if (u0 < u1) {
             const StreamJob &J0 = jobs[find_job(jobs, P.count, u0)];
-            stage_x<PACKED>(J0, P.M, xslots, warp - 1, kStagers, lane);
-            named_bar(9, 32 * kStagers);
-            if (warp == 1) mbar_arrive(smem_u32(&xfull[0]));
+            stage_x<PACKED>(J0, P.M, xslots, warp == 1 ? 0 : warp - kFirstConsumer + 1,
+                            kStagers, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(xfirst));
+            if (warp == 1) {
+                first_ok = mbar_wait(smem_u32(xfirst), 0, abort_flag);
+                if (first_ok) mbar_arrive(smem_u32(&xfull[0]));
+            }
         }
         if (warp == 1) {
             // ---------------- activation stager ----------------
             const float *cur = nullptr;
             uint32_t e = 0;
             int js = u0 < u1 ? find_job(jobs, P.count, u0) : 0;
-            for (int u = u0; u < u1 && !*abort_flag; ++u) {
+            for (int u = u0; u < u1 && first_ok && !*abort_flag; ++u) {
                 js = next_job(jobs, P.count, js, u);
                 const StreamJob &J = jobs[js];
                 if (u != u0 && J.x == cur) continue;
@@ -1103,19 +1066,18 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
             }
         } else {
             // ---------------- consumers ----------------
-            const int cw = warp - 2;
-            const Xchg xg{xchg, xbars};
+            const int rg = warp - kFirstConsumer;
             if (u0 < u1) {
                 if constexpr (PACKED) {
                     if constexpr (MT == 1)
-                        consume_packed_m1(P, jobs, smem, xslots, full, empty, xfull, xempty,
-                                          abort_flag, xg, u0, u1, cw, lane);
+                        consume_packed_m1(P, jobs, smem, szring, xslots, full, empty, xfull,
+                                          xempty, abort_flag, u0, u1, rg, lane);
                     else
-                        consume_packed_mx<MT>(P, jobs, smem, xslots, full, empty, xfull,
-                                              xempty, abort_flag, xg, u0, u1, cw, lane);
+                        consume_packed_mx<MT>(P, jobs, smem, szring, xslots, full, empty,
+                                              xfull, xempty, abort_flag, u0, u1, rg, lane);
                 } else {
                     consume_runtime<MT>(P, jobs, smem, xslots, full, empty, xfull, xempty,
-                                        abort_flag, xg, u0, u1, cw, lane);
+                                        abort_flag, u0, u1, rg, lane);
                 }
             }
         }
@@ -1126,8 +1088,7 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-constexpr int kXchgBytes = 8 * 2 * 16 * kMaxM * 4;
-constexpr int kBarBytes = 512 + kMaxJobs * (int)sizeof(StreamJob);
+constexpr int kBarBytes = 256 + kMaxJobs * (int)sizeof(StreamJob);
 
 template <bool PACKED, int MT>
 bc_status launch_one(const StreamParams &P, int grid, int smem, cudaStream_t s) {
@@ -1197,8 +1158,9 @@ bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed,
     for (int i = 0; i < count; ++i)
         if (jobs[i].N >= (1 << 30) || jobs[i].K >= (1 << 24)) return false;
     const size_t xs = xslot_bytes_for(jobs, count, M, packed);
-    const size_t fixed = 2 * xs + kXchgBytes + kBarBytes + 1024;
-    if (fixed + 2 * (size_t)kStageBytes > (size_t)max_smem) return false;
+    const size_t fixed = 2 * xs + kBarBytes + 1024;
+    const size_t per_stage = kStageBytes + (packed ? kSzBytes : 0);
+    if (fixed + 2 * per_stage > (size_t)max_smem) return false;
     return tensor_map_encoder() != nullptr;
 }
 
@@ -1227,8 +1189,9 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
             jbytes[i] = (double)J.N * rbytes;
         }
         const size_t xs = xslot_bytes_for(jobs + b0, n, M, packed);
-        const int fixed = (int)(2 * xs) + kXchgBytes + kBarBytes + 1024;
-        int stages = (di.max_smem_optin - fixed) / kStageBytes;
+        const int fixed = (int)(2 * xs) + kBarBytes + 1024;
+        const int per_stage = kStageBytes + (packed ? kSzBytes : 0);
+        int stages = (di.max_smem_optin - fixed) / per_stage;
         stages = std::min(stages, 6);
         if (stages < 2) return BC_ERR_UNSUPPORTED;
         const int grid = std::max(1, std::min({units, di.sm_count, kMaxCtas}));
@@ -1255,7 +1218,7 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
         P.bits = bits;
         P.xslot_bytes = (int)xs;
         P.stages = stages;
-        const int smem = stages * kStageBytes + fixed;
+        const int smem = stages * per_stage + fixed;
         bc_status st;
         if (packed) {
             st = M <= 1 ? launch_one<true, 1>(P, grid, smem, s)
