@@ -1150,6 +1150,63 @@ size_t xslot_bytes_for(const GemvJob *jobs, int count, int M, bool packed) {
     return (xmax + 127) / 128 * 128;
 }
 
+// Contiguous unit ranges, one per CTA, that minimise the largest range's cost
+// (the classic linear partition: binary search on the bound, greedy fill).
+// A unit costs its weight bytes plus a fixed share for its end-of-unit work,
+// and a matrix whose x differs from the previous one adds the cost of staging
+// it.  Units of one matrix cost the same, so the greedy fill works matrix by
+// matrix: O(matrices + CTAs) per probe of the bound.
+constexpr double kUnitOverheadBytes = 4096.0;
+constexpr double kXSwitchBytes = 16384.0;
+
+void partition_units(StreamParams &P, int n, bool packed, int grid) {
+    std::vector<double> ucost(n), jextra(n);
+    std::vector<int> nunits(n);
+    double total = 0, umax = 0;
+    for (int i = 0; i < n; ++i) {
+        const StreamJob &J = P.jobs[i];
+        ucost[i] = (double)kRows * (packed ? J.K / 2 : J.K * 2) + kUnitOverheadBytes;
+        jextra[i] = (i == 0 || P.jobs[i - 1].x != J.x) ? kXSwitchBytes : 0.0;
+        nunits[i] = (J.N + kRows - 1) / kRows;
+        total += ucost[i] * nunits[i] + jextra[i];
+        umax = std::max(umax, ucost[i] + jextra[i]);
+    }
+    // CTAs a bound needs; fills cta_begin when `out` is set
+    auto fill = [&](double T, bool out) -> int {
+        int ctas = 1, unit = 0;
+        double cur = 0;
+        if (out) P.cta_begin[0] = 0;
+        for (int i = 0; i < n; ++i) {
+            int left = nunits[i];
+            double extra = jextra[i];
+            while (left > 0) {
+                const double room = T - cur - extra;
+                int fit = room >= ucost[i] ? (int)std::min<double>(left, room / ucost[i]) : 0;
+                if (fit == 0 && cur == 0) fit = 1;       // a unit above T still goes somewhere
+                cur += extra + fit * ucost[i];
+                extra = 0;
+                left -= fit;
+                unit += fit;
+                if (left > 0) {                          // next CTA starts here
+                    if (out && ctas < grid) P.cta_begin[ctas] = unit;
+                    ++ctas;
+                    cur = 0;
+                    extra = kXSwitchBytes;               // it stages this x itself
+                }
+            }
+        }
+        return ctas;
+    };
+    double lo = std::max(umax, total / grid), hi = total + umax;
+    for (int it = 0; it < 48 && hi - lo > 1.0; ++it) {
+        const double mid = 0.5 * (lo + hi);
+        if (fill(mid, false) <= grid) hi = mid; else lo = mid;
+    }
+    const int used = fill(hi, true);
+    // CTAs past the last range get empty ranges
+    for (int c = std::min(used, grid); c < grid; ++c) P.cta_begin[c] = P.total_units;
+}
+
 }  // namespace
 
 bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed,
@@ -1176,7 +1233,6 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
     for (int b0 = 0; b0 < count; b0 += kMaxJobs) {
         const int n = std::min(kMaxJobs, count - b0);
         int units = 0;
-        std::vector<double> jbytes(n);
         for (int i = 0; i < n; ++i) {
             const GemvJob &G0 = jobs[b0 + i];
             StreamJob &J = P.jobs[i];
@@ -1186,7 +1242,6 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
             J.unit_begin = units;
             units += (J.N + kRows - 1) / kRows;
             if (!encode_weights(enc, &P.wmap[i], G0.w, J.N, rbytes)) return BC_ERR_CUDA;
-            jbytes[i] = (double)J.N * rbytes;
         }
         const size_t xs = xslot_bytes_for(jobs + b0, n, M, packed);
         const int fixed = (int)(2 * xs) + kBarBytes + 1024;
@@ -1195,25 +1250,10 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
         stages = std::min(stages, 6);
         if (stages < 2) return BC_ERR_UNSUPPORTED;
         const int grid = std::max(1, std::min({units, di.sm_count, kMaxCtas}));
-        // byte-balanced contiguous unit ranges
-        double total = 0;
-        for (int i = 0; i < n; ++i) total += jbytes[i];
-        P.cta_begin[0] = 0;
-        int j = 0;
-        double before = 0;     // bytes of jobs < j
-        for (int c = 1; c < grid; ++c) {
-            const double target = total * c / grid;
-            while (j < n - 1 && before + jbytes[j] <= target) before += jbytes[j++];
-            const StreamJob &J = P.jobs[j];
-            const double ub = (double)kRows * (packed ? J.K / 2 : J.K * 2);
-            int lu = (int)((target - before) / ub + 0.5);
-            const int nu = (J.N + kRows - 1) / kRows;
-            lu = std::min(std::max(lu, 0), nu);
-            P.cta_begin[c] = std::max(P.cta_begin[c - 1], J.unit_begin + lu);
-        }
+        P.total_units = units;
+        partition_units(P, n, packed, grid);
         P.cta_begin[grid] = units;
         P.count = n;
-        P.total_units = units;
         P.M = M;
         P.bits = bits;
         P.xslot_bytes = (int)xs;
