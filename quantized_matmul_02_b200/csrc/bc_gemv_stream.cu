@@ -89,8 +89,9 @@ struct __align__(64) StreamParams {
     CUtensorMap wmap[kMaxJobs];   // weights as bytes [N][row_bytes], box 128x128, SW128
     StreamJob jobs[kMaxJobs];
     int cta_begin[kMaxCtas + 1];
+    int cta_job[kMaxCtas + 1];    // job of each CTA's first unit (count-1 past the end)
     int count, total_units, M, bits;
-    int xslot_bytes, stages;
+    int xslot_bytes, stages, max_cta_jobs;
 };
 static_assert(sizeof(StreamParams) <= 32000, "kernel parameter space");
 
@@ -206,16 +207,6 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t v) {
     return __half22float2(h);
 }
 
-// The job table is copied into shared memory at kernel start: dynamically
-// indexed reads of a ~30 KB parameter block miss the constant cache.
-__device__ __forceinline__ int find_job(const StreamJob *jobs, int count, int unit) {
-    int lo = 0, hi = count - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (jobs[mid].unit_begin <= unit) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
 // Units are visited in increasing order, so the owning job only moves forward.
 __device__ __forceinline__ int next_job(const StreamJob *jobs, int count, int j, int unit) {
     while (j + 1 < count && jobs[j + 1].unit_begin <= unit) ++j;
@@ -473,9 +464,9 @@ struct StageA {
     uint32_t s[2][2], z[2][2];   // [row ra / ra+8][window] fp16 pair (2eh, 2eh+1)
 };
 __device__ __forceinline__ void consume_packed_m1(
-    const StreamParams &P, const StreamJob *jobs, uint8_t *smem, const uint8_t *szring,
-    uint8_t *xslots, uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
-    volatile int *abort_flag, int u0, int u1, int rg, int lane) {
+    const StreamParams &P, const StreamJob *jobs, int jf, int jc, uint8_t *smem,
+    const uint8_t *szring, uint8_t *xslots, uint64_t *full, uint64_t *empty, uint64_t *xfull,
+    uint64_t *xempty, volatile int *abort_flag, int u0, int u1, int rg, int lane) {
     const int S = P.stages;
     const int gq = lane >> 2, t = lane & 3;
     // ldmatrix: this lane gives the address of row lrow of unit (j + 4*(lane>>4))
@@ -491,7 +482,7 @@ __device__ __forceinline__ void consume_packed_m1(
     const int eh = t >> 1, ep = t & 1;
     const int ra = 16 * rg + gq;
     XCursor xc;
-    Walk k{u0, 0, find_job(jobs, P.count, u0), 0, 0u};
+    Walk k{u0, 0, jf, 0, 0u};
     float ya = 0.0f, yb = 0.0f;
     auto load = [&](StageA &r, int s, uint32_t ph) -> bool {
         if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) return false;
@@ -524,7 +515,7 @@ __device__ __forceinline__ void consume_packed_m1(
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));
         Walk n;
-        const bool more = k.next(jobs, P.count, u1, kch, S, n);
+        const bool more = k.next(jobs, jc, u1, kch, S, n);
         if (more && !load(nxt, n.sidx, n.sph)) return true;
         const int rs = dig_rs(kch);
 #pragma unroll
@@ -588,9 +579,9 @@ __device__ __forceinline__ void consume_packed_m1(
 // x rows as B columns (row 2*mp + h in columns 4h..4h+3).
 template <int MT>
 __device__ __forceinline__ void consume_packed_mx(
-    const StreamParams &P, const StreamJob *jobs, uint8_t *smem, const uint8_t *szring,
-    uint8_t *xslots, uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
-    volatile int *abort_flag, int u0, int u1, int rg, int lane) {
+    const StreamParams &P, const StreamJob *jobs, int jf, int jc, uint8_t *smem,
+    const uint8_t *szring, uint8_t *xslots, uint64_t *full, uint64_t *empty, uint64_t *xfull,
+    uint64_t *xempty, volatile int *abort_flag, int u0, int u1, int rg, int lane) {
     constexpr int MP = MT / 2;
     const int S = P.stages;
     const int gq = lane >> 2, t = lane & 3;
@@ -604,7 +595,7 @@ __device__ __forceinline__ void consume_packed_mx(
     const int eh = t >> 1, ep = t & 1;
     const int ra = 16 * rg + gq;
     XCursor xc;
-    Walk k{u0, 0, find_job(jobs, P.count, u0), 0, 0u};
+    Walk k{u0, 0, jf, 0, 0u};
     float ya[MP], yb[MP];
 #pragma unroll
     for (int p = 0; p < MP; ++p) ya[p] = yb[p] = 0.0f;
@@ -690,7 +681,7 @@ __device__ __forceinline__ void consume_packed_mx(
             }
         }
         Walk n;
-        const bool more = k.next(jobs, P.count, u1, kch, S, n);
+        const bool more = k.next(jobs, jc, u1, kch, S, n);
         if (n.kc == 0 || !more) {      // unit done: two lanes per row and x row
             const int r0 = (k.u - J.unit_begin) * kRows;
 #pragma unroll
@@ -721,8 +712,8 @@ __device__ __forceinline__ void consume_packed_mx(
 // 64 k of each window, so a row's dot product is spread over two lanes.
 template <int MT>
 __device__ __forceinline__ void consume_runtime(
-    const StreamParams &P, const StreamJob *jobs, uint8_t *smem, uint8_t *xslots,
-    uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
+    const StreamParams &P, const StreamJob *jobs, int jf, int jc, uint8_t *smem,
+    uint8_t *xslots, uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
     volatile int *abort_flag, int u0, int u1, int rg, int lane) {
     const int S = P.stages;
     const int r16 = lane >> 1, part = lane & 1;       // row in group, 32-k half
@@ -730,7 +721,7 @@ __device__ __forceinline__ void consume_runtime(
     const float L = (float)((1 << P.bits) - 1);
     const bool pass = P.bits == 16;
     XCursor xc;
-    Walk k{u0, 0, find_job(jobs, P.count, u0), 0, 0u};
+    Walk k{u0, 0, jf, 0, 0u};
     // (scale, zero) of this lane's two windows for the current and next stage
     auto load_sz = [&](const Walk &q, float4 &o) {
         const StreamJob &J = jobs[q.jidx];
@@ -762,7 +753,7 @@ __device__ __forceinline__ void consume_runtime(
         const int row = (k.u - J.unit_begin) * kRows + rr;
         const int kchunks = kchunks_of<false>(J.K);
         Walk n;
-        const bool more = k.next(jobs, P.count, u1, kchunks, S, n);
+        const bool more = k.next(jobs, jc, u1, kchunks, S, n);
         if (more) load_sz(n, fill);
         if (!mbar_wait(smem_u32(&full[k.sidx]), k.sph, abort_flag)) return true;
         const uint8_t *stage = smem + k.sidx * kStageBytes;
@@ -859,20 +850,20 @@ __device__ __forceinline__ void consume_runtime(
 // Warp 2 of a packed launch: the scale / zero slice of every stage of the
 // CTA's range, in ring order, gated by the same empty barriers as the loader
 // and counted as a second arrival on each full barrier.
-__device__ __forceinline__ void sz_stager(const StreamParams &P, const StreamJob *jobs,
-                                       uint8_t *szring, uint64_t *full, uint64_t *empty,
+__device__ __forceinline__ void sz_stager(const StreamParams &P, const StreamJob *jobs, int jf,
+                                       int jc, uint8_t *szring, uint64_t *full, uint64_t *empty,
                                        volatile int *abort_flag, int u0, int u1, int half,
                                        int lane) {
     const int S = P.stages;
-    SzWalk st{u0, 0, find_job(jobs, P.count, u0)};   // stage stored next
+    SzWalk st{u0, 0, jf};   // stage stored next
     SzWalk ld = st;                                     // stage loaded next
     bool ld_ok = true;
     SzSet A, B, C;
     sz_issue(jobs, ld, half, lane, A);
-    ld_ok = ld.next(jobs, P.count, u1);
+    ld_ok = ld.next(jobs, jc, u1);
     if (ld_ok) {
         sz_issue(jobs, ld, half, lane, B);
-        ld_ok = ld.next(jobs, P.count, u1);
+        ld_ok = ld.next(jobs, jc, u1);
     }
     int sidx = 0;
     uint32_t sph = 0;
@@ -880,7 +871,7 @@ __device__ __forceinline__ void sz_stager(const StreamParams &P, const StreamJob
     auto step = [&](const SzSet &cur, SzSet &fill) -> bool {
         if (ld_ok) {
             sz_issue(jobs, ld, half, lane, fill);
-            ld_ok = ld.next(jobs, P.count, u1);
+            ld_ok = ld.next(jobs, jc, u1);
         }
         bool got = true;
         if (lane == 0) got = mbar_wait(smem_u32(&empty[sidx]), sph ^ 1, abort_flag);
@@ -894,7 +885,7 @@ __device__ __forceinline__ void sz_stager(const StreamParams &P, const StreamJob
             sidx = 0;
             sph ^= 1;
         }
-        return !st.next(jobs, P.count, u1);
+        return !st.next(jobs, jc, u1);
     };
     while (!step(A, C) && !step(B, A) && !step(C, B)) {
     }
@@ -914,28 +905,21 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     uint64_t *xfull = bars + 2 * S, *xempty = xfull + 2;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(xempty + 2);
     uint64_t *xfirst = xempty + 3;      // the first x slot is complete
-    StreamJob *jobs = reinterpret_cast<StreamJob *>(bars + 2 * S + 8);
+    StreamJob *jobs_sm = reinterpret_cast<StreamJob *>(bars + 2 * S + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u0 = P.cta_begin[blockIdx.x], u1 = P.cta_begin[blockIdx.x + 1];
-    // The activations of this CTA's matrices go to L2 ahead of the weight
-    // stream: queued behind the first ring fill they would hold up the start.
-    if (warp >= 1 && warp < 1 + kStagers && u0 < u1) {
-        const int jf = find_job(P.jobs, P.count, u0), jl = find_job(P.jobs, P.count, u1 - 1);
-        for (int j = jf; j <= jl; ++j) {
-            const StreamJob &J = P.jobs[j];
-            if (j > jf && P.jobs[j - 1].x == J.x) continue;
-            const int lines = (int)(((int64_t)P.M * J.K * 4 + 127) / 128);
-            for (int l = 32 * (warp - 1) + lane; l < lines; l += 32 * kStagers)
-                prefetch_l2(reinterpret_cast<const char *>(J.x) + (int64_t)l * 128);
-        }
-    }
+    // This CTA's jobs (those its unit range touches) into shared memory; the
+    // table is indexed by global job number through a rebased pointer.
+    const int jf = P.cta_job[blockIdx.x];
+    const int jc = min(P.count, P.cta_job[blockIdx.x + 1] + 1);
     {
-        const uint32_t *src = reinterpret_cast<const uint32_t *>(P.jobs);
-        uint32_t *dst = reinterpret_cast<uint32_t *>(jobs);
-        const int words = P.count * (int)(sizeof(StreamJob) / 4);
-        for (int i = threadIdx.x; i < words; i += kThreads) dst[i] = src[i];
+        const uint4 *src = reinterpret_cast<const uint4 *>(&P.jobs[jf]);
+        uint4 *dst = reinterpret_cast<uint4 *>(jobs_sm);
+        const int n16 = (jc - jf) * (int)(sizeof(StreamJob) / 16);
+        for (int i = threadIdx.x; i < n16; i += kThreads) dst[i] = src[i];
     }
+    const StreamJob *jobs = jobs_sm - jf;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -951,38 +935,34 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
+    // The activations of this CTA's matrices go to L2 ahead of the weight
+    // stream: queued behind the first ring fill they would hold up the start.
+    if (warp >= 1 && warp < 1 + kStagers && u0 < u1) {
+        for (int j = jf; j < jc; ++j) {
+            const StreamJob &J = jobs[j];
+            if (j > jf && jobs[j - 1].x == J.x) continue;
+            const int lines = (int)(((int64_t)P.M * J.K * 4 + 127) / 128);
+            for (int l = 32 * (warp - 1) + lane; l < lines; l += 32 * kStagers)
+                prefetch_l2(reinterpret_cast<const char *>(J.x) + (int64_t)l * 128);
+        }
+    }
+    __syncthreads();
 
     if (warp == 0) {
         // ---------------- loader ----------------
         const uint64_t policy = evict_first_policy();
         uint32_t g = 0, armed = 0;
-        int jw = u0 < u1 ? find_job(jobs, P.count, u0) : 0;
+        int jw = jf;
         int pidx = 0;
         uint32_t pph = 0;
         bool ok = true;
         for (int u = u0; u < u1 && ok; ++u) {
-            jw = next_job(jobs, P.count, jw, u);
+            jw = next_job(jobs, jc, jw, u);
             const int j = jw;
             const StreamJob &J = jobs[j];
             const int r0 = (u - J.unit_begin) * kRows;
             const int rbytes = row_bytes_of<PACKED>(J.K);
             const int kchunks = kchunks_of<PACKED>(J.K);
-            if constexpr (PACKED) {
-                // the unit's scales and zeros (one contiguous block each) go to
-                // L2 with its weights; consumers read them a few stages later
-                const int G = J.K >> 6;
-                const int64_t b0 = (int64_t)r0 * G * 2;
-                const int64_t b1 = (int64_t)min(r0 + kRows, J.N) * G * 2;
-                const int lines = (int)((b1 - b0 + 127) >> 7) + 1;
-                const char *sb = reinterpret_cast<const char *>(J.s) + (b0 & ~(int64_t)127);
-                const char *zb = reinterpret_cast<const char *>(J.z) + (b0 & ~(int64_t)127);
-                const int64_t limit = (int64_t)J.N * G * 2 - (b0 & ~(int64_t)127);
-                for (int l = lane; l < lines; l += 32) {
-                    if ((int64_t)l * 128 >= limit) break;
-                    prefetch_l2(sb + (int64_t)l * 128);
-                    prefetch_l2(zb + (int64_t)l * 128);
-                }
-            }
             for (int kc = 0; kc < kchunks; ++kc, ++g) {
                 const int s = pidx;
                 bool got = true;
@@ -1009,6 +989,23 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
                                     policy);
                 }
                 armed |= 1u << s;
+                if (PACKED && kc == 0) {
+                    // the unit's scales and zeros (one contiguous block each)
+                    // go to L2 behind its first weights; the scale/zero
+                    // stagers read them a few stages later
+                    const int G = J.K >> 6;
+                    const int64_t b0 = (int64_t)r0 * G * 2;
+                    const int64_t b1 = (int64_t)min(r0 + kRows, J.N) * G * 2;
+                    const int lines = (int)((b1 - b0 + 127) >> 7) + 1;
+                    const int64_t a0 = b0 & ~(int64_t)127;
+                    const char *sb = reinterpret_cast<const char *>(J.s) + a0;
+                    const char *zb = reinterpret_cast<const char *>(J.z) + a0;
+                    const int64_t limit = (int64_t)J.N * G * 2 - a0;
+                    for (int l = lane; l < lines && (int64_t)l * 128 < limit; l += 32) {
+                        prefetch_l2(sb + (int64_t)l * 128);
+                        prefetch_l2(zb + (int64_t)l * 128);
+                    }
+                }
             }
         }
         // drain: copies in flight land before the CTA exits
@@ -1026,7 +1023,8 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     } else if (warp >= 2 && warp < kFirstConsumer) {
         // ---------------- scale / zero stagers (packed) ----------------
         if constexpr (PACKED) {
-            if (u0 < u1) sz_stager(P, jobs, szring, full, empty, abort_flag, u0, u1, warp - 2, lane);
+            if (u0 < u1)
+                sz_stager(P, jobs, jf, jc, szring, full, empty, abort_flag, u0, u1, warp - 2, lane);
         }
     } else {
         // the first x slot, by the x stager and the consumers together; each
@@ -1034,7 +1032,7 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
         // first xfull phase once all have
         bool first_ok = true;
         if (u0 < u1) {
-            const StreamJob &J0 = jobs[find_job(jobs, P.count, u0)];
+            const StreamJob &J0 = jobs[jf];
             stage_x<PACKED>(J0, P.M, xslots, warp == 1 ? 0 : warp - kFirstConsumer + 1,
                             kStagers, lane);
             __syncwarp();
@@ -1048,9 +1046,9 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
             // ---------------- activation stager ----------------
             const float *cur = nullptr;
             uint32_t e = 0;
-            int js = u0 < u1 ? find_job(jobs, P.count, u0) : 0;
+            int js = jf;
             for (int u = u0; u < u1 && first_ok && !*abort_flag; ++u) {
-                js = next_job(jobs, P.count, js, u);
+                js = next_job(jobs, jc, js, u);
                 const StreamJob &J = jobs[js];
                 if (u != u0 && J.x == cur) continue;
                 cur = J.x;
@@ -1070,14 +1068,15 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
             if (u0 < u1) {
                 if constexpr (PACKED) {
                     if constexpr (MT == 1)
-                        consume_packed_m1(P, jobs, smem, szring, xslots, full, empty, xfull,
-                                          xempty, abort_flag, u0, u1, rg, lane);
+                        consume_packed_m1(P, jobs, jf, jc, smem, szring, xslots, full, empty,
+                                          xfull, xempty, abort_flag, u0, u1, rg, lane);
                     else
-                        consume_packed_mx<MT>(P, jobs, smem, szring, xslots, full, empty,
-                                              xfull, xempty, abort_flag, u0, u1, rg, lane);
+                        consume_packed_mx<MT>(P, jobs, jf, jc, smem, szring, xslots, full,
+                                              empty, xfull, xempty, abort_flag, u0, u1, rg,
+                                              lane);
                 } else {
-                    consume_runtime<MT>(P, jobs, smem, xslots, full, empty, xfull, xempty,
-                                        abort_flag, u0, u1, rg, lane);
+                    consume_runtime<MT>(P, jobs, jf, jc, smem, xslots, full, empty, xfull,
+                                        xempty, abort_flag, u0, u1, rg, lane);
                 }
             }
         }
@@ -1244,16 +1243,27 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
             if (!encode_weights(enc, &P.wmap[i], G0.w, J.N, rbytes)) return BC_ERR_CUDA;
         }
         const size_t xs = xslot_bytes_for(jobs + b0, n, M, packed);
-        const int fixed = (int)(2 * xs) + kBarBytes + 1024;
-        const int per_stage = kStageBytes + (packed ? kSzBytes : 0);
-        int stages = (di.max_smem_optin - fixed) / per_stage;
-        stages = std::min(stages, 6);
-        if (stages < 2) return BC_ERR_UNSUPPORTED;
         const int grid = std::max(1, std::min({units, di.sm_count, kMaxCtas}));
         P.total_units = units;
         partition_units(P, n, packed, grid);
         P.cta_begin[grid] = units;
         P.count = n;
+        // first job of each CTA's range, and the most jobs one range touches
+        {
+            int jj = 0, most = 1;
+            for (int c = 0; c <= grid; ++c) {
+                const int u = std::min(P.cta_begin[c], units - 1);
+                while (jj + 1 < n && P.jobs[jj + 1].unit_begin <= u) ++jj;
+                P.cta_job[c] = jj;
+                if (c > 0) most = std::max(most, P.cta_job[c] - P.cta_job[c - 1] + 1);
+            }
+            P.max_cta_jobs = most;
+        }
+        const int fixed = (int)(2 * xs) + 256 + P.max_cta_jobs * (int)sizeof(StreamJob) + 1024;
+        const int per_stage = kStageBytes + (packed ? kSzBytes : 0);
+        int stages = (di.max_smem_optin - fixed) / per_stage;
+        stages = std::min(stages, 6);
+        if (stages < 2) return BC_ERR_UNSUPPORTED;
         P.M = M;
         P.bits = bits;
         P.xslot_bytes = (int)xs;
