@@ -25,16 +25,18 @@
 //
 // Packed int4 (Enargeia, "Four bits per weight": codes unpacked in registers,
 // never written back) runs on the int8 tensor cores (mma.sync m16n8k32
-// u8 x s8 -> s32).  ldmatrix brings the swizzled stage into A fragments; one
-// AND per register gives the even-k codes (q) and one the odd-k codes (16 q)
-// as unsigned bytes.  The activations are staged as integers per 64-group,
-//     x_k ~= X_k * 2^(E_g - 27),  X_k = rint(x_k 2^(27 - E_g)) (even k),
-//                                 X_k = 16 rint(x_k 2^(23 - E_g)) (odd k),
-// with max|x| < 2^E_g over the group, each split into four balanced int8
-// digits (X = d0 + 2^8 d1 + 2^16 d2 + 2^24 d3) that fill the 8 columns of B.
-// With one x row the columns hold 2 groups x 4 digits, the k slots of each
-// mma split between the two groups (block diagonal); with several x rows
-// they hold 2 rows x 4 digits.  The integer dot products are exact, so
+// u8 x s8 -> s32).  The activations are staged as integers per 64-group g
+// (max|x| < 2^E_g):  X_e = rint(x_k 2^(27-E_g)) at even k and
+// X_o = rint(x_k 2^(23-E_g)) at odd k, so x_k ~= X_e 2^(E_g-27), resp.
+// 16 X_o 2^(E_g-27).  ldmatrix brings the swizzled stage into A fragments;
+// each code byte b = q_e + 16 q_o (two neighbouring k) fills an even-k slot
+// as is and an odd-k slot as b & 0xF0 = 16 q_o, against B digits of X_e and
+// of X_o - X_e respectively:
+//     b X_e + 16 q_o (X_o - X_e) = q_e X_e + 16 q_o X_o.
+// B values are split into four balanced int8 digits (d0 + 2^8 d1 + 2^16 d2 +
+// 2^24 d3) that fill the 8 columns of B: with one x row, 2 groups x 4 digits
+// (the k slots of each mma split between the two groups, block diagonal);
+// with several x rows, 2 rows x 4 digits.  The integer sums are exact, so
 //     y = sum_g s_g ( 2^(E_g-27) sum_d 2^(8d) C_gd - z_g sum_k x_k~ )
 // carries only the rounding of x to 23-27 bits and of the fp32 epilogue.
 //
@@ -278,7 +280,7 @@ __device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
                 const int xo = __float2int_rn(v[2 * i + 1] * sc_o);  // |xo| <= 2^23
                 sum += xe + 16 * xo;
                 de[i] = digits4(xe);
-                dq[i] = digits4(xo);
+                dq[i] = digits4(xo - xe);     // odd slots carry X_odd - X_even (raw-byte A)
             }
             uint32_t te[4], to[4];
             transpose4(de, te);
@@ -534,8 +536,7 @@ __device__ __forceinline__ void consume_packed_m1(
                 const uint4 &Q = j < 2 ? Q0 : Q1;
                 const uint32_t bl = (j & 1) ? Q.z : Q.x, bu = (j & 1) ? Q.w : Q.y;
                 const uint32_t(&R)[4] = cur.R[w][j];
-                mma_i8(C, R[0] & 0x0F0F0F0Fu, R[1] & 0x0F0F0F0Fu, R[2] & 0x0F0F0F0Fu,
-                       R[3] & 0x0F0F0F0Fu, bl & m0, bl & m1);
+                mma_i8(C, R[0], R[1], R[2], R[3], bl & m0, bl & m1);
                 mma_i8(C, R[0] & 0xF0F0F0F0u, R[1] & 0xF0F0F0F0u, R[2] & 0xF0F0F0F0u,
                        R[3] & 0xF0F0F0F0u, bu & m0, bu & m1);
             }
@@ -625,14 +626,11 @@ __device__ __forceinline__ void consume_packed_mx(
             uint32_t R[4][4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) ldsm_x4(box0 + w * kBoxBytes + a_off[j], R[j]);
-            uint32_t lo[4][4], hi[4][4];
+            uint32_t hi[4][4];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    lo[j][i] = R[j][i] & 0x0F0F0F0Fu;
-                    hi[j][i] = R[j][i] & 0xF0F0F0F0u;
-                }
+                for (int i = 0; i < 4; ++i) hi[j][i] = R[j][i] & 0xF0F0F0F0u;
             if (w == 1) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));   // stage consumed
@@ -662,8 +660,8 @@ __device__ __forceinline__ void consume_packed_mx(
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     C[j][0] = C[j][1] = C[j][2] = C[j][3] = 0;
-                    mma_i8(C[j], lo[j][0], lo[j][1], hi[j][0], hi[j][1], Q[j].x, Q[j].y);
-                    mma_i8(C[j], lo[j][2], lo[j][3], hi[j][2], hi[j][3], Q[j].z, Q[j].w);
+                    mma_i8(C[j], R[j][0], R[j][1], hi[j][0], hi[j][1], Q[j].x, Q[j].y);
+                    mma_i8(C[j], R[j][2], R[j][3], hi[j][2], hi[j][3], Q[j].z, Q[j].w);
                 }
                 const float *tb = reinterpret_cast<const float *>(
                     xc.xs + (2 * mp + eh) * mb + 64 * rs + 8 * (ep * 8 * kch + 8 * k.kc + 4 * w));
