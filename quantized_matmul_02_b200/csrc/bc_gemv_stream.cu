@@ -52,6 +52,8 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstring>
+#include <memory>
 #include <mutex>
 #include <vector>
 
@@ -1218,15 +1220,55 @@ bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed,
     return tensor_map_encoder() != nullptr;
 }
 
+namespace {
+// Prepared launches of recent calls (per host thread).  A decode step calls
+// with the same matrices every time; a hit skips the tensor-map encoding and
+// the partition, leaving only the launch itself.
+struct StreamPlan {
+    std::vector<GemvJob> key;
+    int M = 0, bits = 0, dev = -1;
+    bool packed = false;
+    StreamParams P;
+    int grid = 0, smem = 0;
+};
+constexpr int kPlanCache = 4;
+
+bool same_call(const StreamPlan &p, const GemvJob *jobs, int count, int M, int bits,
+               bool packed, int dev) {
+    return p.dev == dev && p.M == M && p.bits == bits && p.packed == packed &&
+           (int)p.key.size() == count &&
+           std::memcmp(p.key.data(), jobs, sizeof(GemvJob) * count) == 0;
+}
+
+bc_status launch_plan(const StreamPlan &p, cudaStream_t s) {
+    if (p.packed)
+        return p.M <= 1 ? launch_one<true, 1>(p.P, p.grid, p.smem, s)
+             : p.M <= 2 ? launch_one<true, 2>(p.P, p.grid, p.smem, s)
+                        : launch_one<true, 4>(p.P, p.grid, p.smem, s);
+    return p.M <= 1 ? launch_one<false, 1>(p.P, p.grid, p.smem, s)
+         : p.M <= 2 ? launch_one<false, 2>(p.P, p.grid, p.smem, s)
+                    : launch_one<false, 4>(p.P, p.grid, p.smem, s);
+}
+}  // namespace
+
 bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
                              bool packed, cudaStream_t s) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BC_ERR_CUDA;
+    thread_local std::vector<std::unique_ptr<StreamPlan>> plans;
+    if (count <= kMaxJobs) {
+        for (size_t i = 0; i < plans.size(); ++i) {
+            if (!same_call(*plans[i], jobs, count, M, bits, packed, dev)) continue;
+            if (i) std::rotate(plans.begin(), plans.begin() + i, plans.begin() + i + 1);
+            return launch_plan(*plans[0], s);
+        }
+    }
     DeviceInfo di;
     if (!device_info(&di)) return BC_ERR_CUDA;
     auto enc = tensor_map_encoder();
     if (!enc) return BC_ERR_CUDA;
-    thread_local StreamParams *Pp = nullptr;
-    if (!Pp) Pp = new StreamParams();
-    StreamParams &P = *Pp;
+    std::unique_ptr<StreamPlan> plan(new StreamPlan());
+    StreamParams &P = plan->P;
     for (int b0 = 0; b0 < count; b0 += kMaxJobs) {
         const int n = std::min(kMaxJobs, count - b0);
         int units = 0;
@@ -1266,19 +1308,19 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
         P.bits = bits;
         P.xslot_bytes = (int)xs;
         P.stages = stages;
-        const int smem = stages * per_stage + fixed;
-        bc_status st;
-        if (packed) {
-            st = M <= 1 ? launch_one<true, 1>(P, grid, smem, s)
-               : M <= 2 ? launch_one<true, 2>(P, grid, smem, s)
-                        : launch_one<true, 4>(P, grid, smem, s);
-        } else {
-            const int mt = M <= 1 ? 1 : M <= 2 ? 2 : 4;
-            st = mt == 1 ? launch_one<false, 1>(P, grid, smem, s)
-               : mt == 2 ? launch_one<false, 2>(P, grid, smem, s)
-                         : launch_one<false, 4>(P, grid, smem, s);
-        }
+        plan->M = M;
+        plan->bits = bits;
+        plan->packed = packed;
+        plan->dev = dev;
+        plan->grid = grid;
+        plan->smem = stages * per_stage + fixed;
+        const bc_status st = launch_plan(*plan, s);
         if (st != BC_OK) return st;
+    }
+    if (count <= kMaxJobs) {
+        plan->key.assign(jobs, jobs + count);
+        plans.insert(plans.begin(), std::move(plan));
+        if ((int)plans.size() > kPlanCache) plans.pop_back();
     }
     return BC_OK;
 }
