@@ -185,6 +185,31 @@ BC_API size_t bc_workspace_size_batched(const bc_matmul_desc *descs, int count,
                                  int64_t M, bc_mode mode, bc_dtype x_dtype);
 
 /*
+ * Flags of bc_matmul_q_batched_ex.
+ *   BC_FLAG_STATIC_WEIGHTS  the caller promises that no work still pending
+ *     (on `stream` or elsewhere) writes any descriptor's weights, scales or
+ *     zeros -- the usual case for a model's weights during decoding.  The
+ *     decode kernel is then launched as a programmatic dependent launch: its
+ *     CTAs may start, and stream weights, scales and zeros, while the kernel
+ *     before it on the stream is still finishing; every read of x and write
+ *     of y still waits until that kernel has completed.  Back-to-back decode
+ *     steps then overlap one step's start with the previous step's end.
+ *     Ignored by the prefill (bf16 x) path and the small-launch GEMV.
+ */
+#define BC_FLAG_STATIC_WEIGHTS 1u
+
+/*
+ * bc_matmul_q_batched_ex -- bc_matmul_q_batched with `flags` (a bitwise OR
+ * of BC_FLAG_* values; unknown bits are rejected with BC_ERR_INVALID_ARG).
+ * flags = 0 is exactly bc_matmul_q_batched.
+ */
+BC_API bc_status bc_matmul_q_batched_ex(const bc_matmul_desc *descs, int count,
+                                 int64_t M, int bits, int64_t group,
+                                 bc_mode mode, bc_dtype x_dtype, void *workspace,
+                                 size_t workspace_bytes, unsigned flags,
+                                 bc_stream_t stream);
+
+/*
  * bc_matmul_q_noalloc -- the decode matmul (fp32 x, the GEMV path of
  * bc_matmul_q) for callers that cannot allocate device memory: code that
  * must not call cudaMalloc (a host callback, a fixed-pool allocator, a

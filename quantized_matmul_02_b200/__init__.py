@@ -25,10 +25,12 @@ BC_OK, BC_ERR_INVALID_ARG, BC_ERR_UNSUPPORTED, BC_ERR_ALIGNMENT, \
 BC_F32, BC_F16, BC_BF16 = 0, 1, 2
 BC_MODE_RUNTIME, BC_MODE_PACKED_INT4 = 0, 1
 GROUP_PER_CHANNEL = 0
+BC_FLAG_STATIC_WEIGHTS = 1
 
 # Every symbol include/bc.h declares.
 EXPORTS = ("bc_group_params", "bc_quantize_codes", "bc_pack_int4",
            "bc_matmul_q", "bc_workspace_size", "bc_matmul_q_batched",
+           "bc_matmul_q_batched_ex",
            "bc_workspace_size_batched", "bc_matmul_q_noalloc",
            "bc_device_timeouts",
            "bc_status_string", "bc_version")
@@ -63,6 +65,8 @@ def _load() -> ctypes.CDLL:
     lib.bc_workspace_size.restype = sz
     lib.bc_matmul_q_batched.argtypes = [ctypes.POINTER(MatmulDesc), i32, i64,
                                         i32, i64, i32, i32, P, sz, P]
+    lib.bc_matmul_q_batched_ex.argtypes = [ctypes.POINTER(MatmulDesc), i32, i64,
+                                           i32, i64, i32, i32, P, sz, ctypes.c_uint, P]
     lib.bc_workspace_size_batched.argtypes = [ctypes.POINTER(MatmulDesc), i32,
                                               i64, i32, i32]
     lib.bc_workspace_size_batched.restype = sz
@@ -75,7 +79,7 @@ def _load() -> ctypes.CDLL:
     lib.bc_status_string.restype = ctypes.c_char_p
     lib.bc_version.restype = i32
     for name in ("bc_group_params", "bc_quantize_codes", "bc_pack_int4",
-                 "bc_matmul_q", "bc_matmul_q_batched"):
+                 "bc_matmul_q", "bc_matmul_q_batched", "bc_matmul_q_batched_ex"):
         getattr(lib, name).restype = i32
     return lib
 
@@ -188,18 +192,22 @@ def workspace_size_batched(descs, M: int, mode: int, x_dtype: int) -> int:
 
 def matmul_q_batched(descs, M: int, bits: int, group: int, mode: int,
                      x_dtype: int = BC_F32, workspace: Optional[torch.Tensor] = None,
-                     stream=None) -> None:
+                     stream=None, static_weights: bool = False) -> None:
     """One grouped launch over the matrices in `descs` (from make_descs).
-    Without `workspace`, split-K scratch (if any) is taken from torch."""
+    Without `workspace`, split-K scratch (if any) is taken from torch.
+    static_weights: BC_FLAG_STATIC_WEIGHTS (no pending work writes the
+    weights, scales or zeros; the decode kernel may then start before the
+    previous kernel on the stream has finished)."""
     if workspace is None:
         need = workspace_size_batched(descs, M, mode, x_dtype)
         if need:
             workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
     wsp = _ptr(workspace) if workspace is not None else None
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check(lib.bc_matmul_q_batched(descs, len(descs), M, bits, group, mode,
-                                   x_dtype, wsp, wsb, _stream(stream)),
-           "bc_matmul_q_batched")
+    flags = BC_FLAG_STATIC_WEIGHTS if static_weights else 0
+    _check(lib.bc_matmul_q_batched_ex(descs, len(descs), M, bits, group, mode,
+                                      x_dtype, wsp, wsb, flags, _stream(stream)),
+           "bc_matmul_q_batched_ex")
 
 
 def device_timeouts() -> int:

@@ -202,7 +202,17 @@ bc_status bc_matmul_q_batched(const bc_matmul_desc *descs, int count,
                               int64_t M, int bits, int64_t group,
                               bc_mode mode, bc_dtype x_dtype, void *workspace,
                               size_t workspace_bytes, bc_stream_t stream) {
+    return bc_matmul_q_batched_ex(descs, count, M, bits, group, mode, x_dtype, workspace,
+                                  workspace_bytes, 0u, stream);
+}
+
+bc_status bc_matmul_q_batched_ex(const bc_matmul_desc *descs, int count,
+                                 int64_t M, int bits, int64_t group,
+                                 bc_mode mode, bc_dtype x_dtype, void *workspace,
+                                 size_t workspace_bytes, unsigned flags,
+                                 bc_stream_t stream) {
     if (!descs || count <= 0) return BC_ERR_INVALID_ARG;
+    if (flags & ~BC_FLAG_STATIC_WEIGHTS) return BC_ERR_INVALID_ARG;
     // group rule: 64, or per channel (0)
     if (group != 64 && group != BC_GROUP_PER_CHANNEL) return BC_ERR_UNSUPPORTED;
     bc_status st = check_matmul_common(M, bits, group, mode, x_dtype);
@@ -238,7 +248,7 @@ bc_status bc_matmul_q_batched(const bc_matmul_desc *descs, int count,
     }
     return launch_gemv(jobs.data(), count, (int)M, bits,
                        mode == BC_MODE_PACKED_INT4, workspace, workspace_bytes,
-                       s);
+                       s, (flags & BC_FLAG_STATIC_WEIGHTS) != 0);
 }
 
 bc_status bc_matmul_q(const void *x, bc_dtype x_dtype, const void *W_or_packed,

@@ -389,11 +389,11 @@ size_t gemv_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed,
 
 bc_status launch_gemv(const GemvJob *jobs, int count, int M, int bits,
                       bool packed, void *workspace, size_t ws_bytes,
-                      cudaStream_t s) {
+                      cudaStream_t s, bool early_start) {
     DeviceInfo di;
     if (!device_info(&di)) return BC_ERR_CUDA;
     if (use_stream(jobs, count, M, packed, di))
-        return launch_gemv_stream(jobs, count, M, bits, packed, s);
+        return launch_gemv_stream(jobs, count, M, bits, packed, s, early_start);
     // ~32 KB of kernel parameters, kept off the stack; the launch copies it.
     thread_local GemvParams *Pp = nullptr;
     if (!Pp) Pp = new GemvParams();

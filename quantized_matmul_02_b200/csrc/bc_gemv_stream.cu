@@ -26,9 +26,9 @@
 // Packed int4 (Enargeia, "Four bits per weight": codes unpacked in registers,
 // never written back) runs on the int8 tensor cores (mma.sync m16n8k32
 // u8 x s8 -> s32).  The activations are staged as integers per 64-group g
-// (max|x| < 2^E_g):  X_e = rint(x_k 2^(27-E_g)) at even k and
-// X_o = rint(x_k 2^(23-E_g)) at odd k, so x_k ~= X_e 2^(E_g-27), resp.
-// 16 X_o 2^(E_g-27).  ldmatrix brings the swizzled stage into A fragments;
+// (max|x| < 2^E_g):  X_e = rint(x_k 2^(30-E_g)) at even k and
+// X_o = rint(x_k 2^(26-E_g)) at odd k, so x_k ~= X_e 2^(E_g-30), resp.
+// 16 X_o 2^(E_g-30).  ldmatrix brings the swizzled stage into A fragments;
 // each code byte b = q_e + 16 q_o (two neighbouring k) fills an even-k slot
 // as is and an odd-k slot as b & 0xF0 = 16 q_o, against B digits of X_e and
 // of X_o - X_e respectively:
@@ -37,8 +37,9 @@
 // 2^24 d3) that fill the 8 columns of B: with one x row, 2 groups x 4 digits
 // (the k slots of each mma split between the two groups, block diagonal);
 // with several x rows, 2 rows x 4 digits.  The integer sums are exact, so
-//     y = sum_g s_g ( 2^(E_g-27) sum_d 2^(8d) C_gd - z_g sum_k x_k~ )
-// carries only the rounding of x to 23-27 bits and of the fp32 epilogue.
+//     y = sum_g s_g ( 2^(E_g-30) sum_d 2^(8d) C_gd - z_g sum_k x_k~ )
+// carries only the rounding of x to 2^-27 of its group maximum (even k 2^-31)
+// and that of the fp32 epilogue.
 //
 // Runtime RTN (BITCRUSH BC-06, "Under the hood": codes computed inline as
 // weights are read) runs on the CUDA cores, four threads per row, with the
@@ -76,7 +77,7 @@ constexpr int kSzBytes = 2 * kRows * 16;   // packed: fp16 scales + zeros of a s
 constexpr int kMaxJobs = 168;
 constexpr int kMaxCtas = 160;
 constexpr int kMaxM = 4;
-constexpr int kXP = 23;                 // bits of the odd-k activation integers
+constexpr int kXP = 26;                 // bits of the odd-k activation integers (even: +4)
 constexpr long long kWaitCycles = 4000000000LL;
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
 
@@ -96,6 +97,7 @@ struct __align__(64) StreamParams {
     int cta_job[kMaxCtas + 1];    // job of each CTA's first unit (count-1 past the end)
     int count, total_units, M, bits;
     int xslot_bytes, stages, max_cta_jobs;
+    int early;                    // launched as a programmatic dependent launch
 };
 static_assert(sizeof(StreamParams) <= 32000, "kernel parameter space");
 
@@ -275,12 +277,12 @@ __device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
             const float sc_e = __uint_as_float((uint32_t)(127 + kXP + 4 - E) << 23);
             const float sc_o = __uint_as_float((uint32_t)(127 + kXP - E) << 23);
             uint32_t de[4], dq[4];
-            int sum = 0;
+            long long sum = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int xe = __float2int_rn(v[2 * i] * sc_e);      // |xe| <= 2^27
-                const int xo = __float2int_rn(v[2 * i + 1] * sc_o);  // |xo| <= 2^23
-                sum += xe + 16 * xo;
+                const int xe = __float2int_rn(v[2 * i] * sc_e);      // |xe| <= 2^30
+                const int xo = __float2int_rn(v[2 * i + 1] * sc_o);  // |xo| <= 2^26
+                sum += (long long)xe + 16ll * xo;
                 de[i] = digits4(xe);
                 dq[i] = digits4(xo - xe);     // odd slots carry X_odd - X_even (raw-byte A)
             }
@@ -292,13 +294,12 @@ __device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
             for (int d = 0; d < 4; ++d)
                 *reinterpret_cast<uint2 *>(dig + (d * 4 + tt) * rs + 2 * U) =
                     make_uint2(te[d], to[d]);
-            float fs = (float)sum;
-            fs += __shfl_xor_sync(0xffffffffu, fs, 1);
-            fs += __shfl_xor_sync(0xffffffffu, fs, 2);
-            fs += __shfl_xor_sync(0xffffffffu, fs, 4);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 4);
             if (j == 0) {
                 const float f = __uint_as_float((uint32_t)(127 + E - kXP - 4) << 23);
-                tab[g] = make_float2(f, f * fs);
+                tab[g] = make_float2(f, (float)((double)f * (double)sum));
                 tab[gpad + g] = make_float2(f * 65536.0f, 0.0f);
             }
         }
@@ -847,6 +848,18 @@ __device__ __forceinline__ void consume_runtime(
     }
 }
 
+// Prefetch of the CTA's activations into L2 by staging warp `wi` of kStagers.
+__device__ __forceinline__ void prefetch_xs(const StreamParams &P, const StreamJob *jobs, int jf,
+                                            int jc, int wi, int lane) {
+    for (int j = jf; j < jc; ++j) {
+        const StreamJob &J = jobs[j];
+        if (j > jf && jobs[j - 1].x == J.x) continue;
+        const int lines = (int)(((int64_t)P.M * J.K * 4 + 127) / 128);
+        for (int l = 32 * wi + lane; l < lines; l += 32 * kStagers)
+            prefetch_l2(reinterpret_cast<const char *>(J.x) + (int64_t)l * 128);
+    }
+}
+
 // Warp 2 of a packed launch: the scale / zero slice of every stage of the
 // CTA's range, in ring order, gated by the same empty barriers as the loader
 // and counted as a second arrival on each full barrier.
@@ -909,6 +922,9 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u0 = P.cta_begin[blockIdx.x], u1 = P.cta_begin[blockIdx.x + 1];
+    // the next launch on the stream may start as SMs free up (no-op unless it
+    // was launched as a programmatic dependent launch)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // This CTA's jobs (those its unit range touches) into shared memory; the
     // table is indexed by global job number through a rebased pointer.
     const int jf = P.cta_job[blockIdx.x];
@@ -937,16 +953,11 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     __syncthreads();
     // The activations of this CTA's matrices go to L2 ahead of the weight
     // stream: queued behind the first ring fill they would hold up the start.
-    if (warp >= 1 && warp < 1 + kStagers && u0 < u1) {
-        for (int j = jf; j < jc; ++j) {
-            const StreamJob &J = jobs[j];
-            if (j > jf && jobs[j - 1].x == J.x) continue;
-            const int lines = (int)(((int64_t)P.M * J.K * 4 + 127) / 128);
-            for (int l = 32 * (warp - 1) + lane; l < lines; l += 32 * kStagers)
-                prefetch_l2(reinterpret_cast<const char *>(J.x) + (int64_t)l * 128);
-        }
-    }
-    __syncthreads();
+    // (After an early start they may not be written yet: the staging warps
+    // prefetch them once the previous kernel has completed.)
+    if (!P.early && warp >= 1 && warp < 1 + kStagers && u0 < u1)
+        prefetch_xs(P, jobs, jf, jc, warp - 1, lane);
+    if (!P.early) __syncthreads();
 
     if (warp == 0) {
         // ---------------- loader ----------------
@@ -1031,6 +1042,11 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
         // warp reports on `xfirst`, and the stager turns that into the slot's
         // first xfull phase once all have
         bool first_ok = true;
+        // x and y belong to the previous kernel until it completes (every CTA
+        // waits here, so this grid completes only after it)
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (P.early && u0 < u1)
+            prefetch_xs(P, jobs, jf, jc, warp == 1 ? 0 : warp - kFirstConsumer + 1, lane);
         if (u0 < u1) {
             const StreamJob &J0 = jobs[jf];
             stage_x<PACKED>(J0, P.M, xslots, warp == 1 ? 0 : warp - kFirstConsumer + 1,
@@ -1091,6 +1107,7 @@ constexpr int kBarBytes = 256 + kMaxJobs * (int)sizeof(StreamJob);
 
 template <bool PACKED, int MT>
 bc_status launch_one(const StreamParams &P, int grid, int smem, cudaStream_t s) {
+    // P.early: programmatic dependent launch (see the kernel's start)
     static std::mutex mu;
     static int attr_smem[64] = {};      // per device: largest size already allowed
     int dev = 0;
@@ -1105,7 +1122,20 @@ bc_status launch_one(const StreamParams &P, int grid, int smem, cudaStream_t s) 
             attr_smem[dev] = smem;
         }
     }
-    gemv_stream_kernel<PACKED, MT><<<grid, kThreads, smem, s>>>(P);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = P.early ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, gemv_stream_kernel<PACKED, MT>, P) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BC_ERR_CUDA;
+    }
     return cuda_status();
 }
 
@@ -1234,8 +1264,9 @@ struct StreamPlan {
 constexpr int kPlanCache = 4;
 
 bool same_call(const StreamPlan &p, const GemvJob *jobs, int count, int M, int bits,
-               bool packed, int dev) {
+               bool packed, int dev, bool early) {
     return p.dev == dev && p.M == M && p.bits == bits && p.packed == packed &&
+           (p.P.early != 0) == early &&
            (int)p.key.size() == count &&
            std::memcmp(p.key.data(), jobs, sizeof(GemvJob) * count) == 0;
 }
@@ -1252,13 +1283,13 @@ bc_status launch_plan(const StreamPlan &p, cudaStream_t s) {
 }  // namespace
 
 bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
-                             bool packed, cudaStream_t s) {
+                             bool packed, cudaStream_t s, bool early_start) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BC_ERR_CUDA;
     thread_local std::vector<std::unique_ptr<StreamPlan>> plans;
     if (count <= kMaxJobs) {
         for (size_t i = 0; i < plans.size(); ++i) {
-            if (!same_call(*plans[i], jobs, count, M, bits, packed, dev)) continue;
+            if (!same_call(*plans[i], jobs, count, M, bits, packed, dev, early_start)) continue;
             if (i) std::rotate(plans.begin(), plans.begin() + i, plans.begin() + i + 1);
             return launch_plan(*plans[0], s);
         }
@@ -1308,6 +1339,7 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
         P.bits = bits;
         P.xslot_bytes = (int)xs;
         P.stages = stages;
+        P.early = early_start ? 1 : 0;
         plan->M = M;
         plan->bits = bits;
         plan->packed = packed;

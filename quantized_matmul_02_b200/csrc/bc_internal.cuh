@@ -60,15 +60,17 @@ struct GemvJob {             // one matrix of a launch
 // unpack for packed codes.  Used for launches large enough to fill the GPU.
 bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed,
                            int max_smem);
+// early_start: programmatic dependent launch (weights known not to be
+// written by pending work; x / y accesses wait for the previous kernel).
 bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
-                             bool packed, cudaStream_t s);
+                             bool packed, cudaStream_t s, bool early_start);
 unsigned gemv_timeouts();
 // Bytes of split-K scratch a launch over these jobs needs.
 size_t gemv_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed,
                             int sm_count);
 bc_status launch_gemv(const GemvJob *jobs, int count, int M, int bits,
                       bool packed, void *workspace, size_t ws_bytes,
-                      cudaStream_t s);
+                      cudaStream_t s, bool early_start = false);
 
 // ---------------------------------------------------------------------------
 // tcgen05 prefill GEMM (bc_gemm_sm100.cu), packed int4 W, bf16 x, M >= 64

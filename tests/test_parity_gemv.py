@@ -254,3 +254,107 @@ def test_batched_mixed_shapes_stream(cuda_lib, M, mode, bits, group):
     for i, (ref, it) in enumerate(zip(refs, items)):
         assert_close(host(it[4]), ref["y"], ref["A"], TOL_FP32, f"matrix {i}")
     assert cuda_lib.device_timeouts() == 0
+
+
+def _stream_set(cuda_lib, M, seed, count=40):
+    """A grouped packed-int4 launch large enough for the streaming kernel."""
+    rng = np.random.default_rng(seed)
+    shapes = [(896, 896), (128, 896), (4864, 896), (896, 4864)]
+    items, Ws = [], []
+    x_dev = {}
+    for i in range(count):
+        N, K = shapes[i % len(shapes)]
+        if K not in x_dev:
+            x_dev[K] = torch.zeros((M, K), device="cuda")
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+        Wd = dev(W)
+        s, z = cuda_lib.group_params(Wd, 4, 64, torch.float16)
+        Wk = cuda_lib.pack_int4(Wd, s, z)
+        y = torch.full((M, N), float("nan"), device="cuda")
+        items.append((x_dev[K], Wk, s, z, y))
+        Ws.append(W)
+    return items, Ws, x_dev
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_static_weights_early_start_sees_new_x(cuda_lib, M):
+    """BC_FLAG_STATIC_WEIGHTS launches the decode kernel as a programmatic
+    dependent launch.  Between back-to-back launches a torch kernel on the
+    same stream rewrites x; each launch must still read the x written just
+    before it (and write y after the previous launch is done)."""
+    items, Ws, x_dev = _stream_set(cuda_lib, M, 91)
+    torch.cuda.synchronize()           # weights are complete before the launches
+    descs = cuda_lib.make_descs(items)
+    xs_host = []
+    staged = []
+    for rep in range(3):
+        xk = {K: wl.activation(60 + rep, K, "x", M, K) for K in x_dev}
+        staged.append({K: dev(v) for K, v in xk.items()})
+        xs_host.append(xk)
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for K, t in x_dev.items():      # an elementwise kernel rewrites x
+            torch.mul(staged[rep][K], 1.0, out=t)
+        cuda_lib.matmul_q_batched(descs, M, 4, 64, cuda_lib.BC_MODE_PACKED_INT4,
+                                  static_weights=True)
+    torch.cuda.synchronize()
+    last = xs_host[-1]
+    for i, ((_, _, _, _, y), W) in enumerate(zip(items, Ws)):
+        ref = oracle.matmul_q(last[W.shape[1]], W, 4, 64, "packed")
+        assert_close(host(y), ref["y"], ref["A"], TOL_FP32, f"matrix {i}")
+    assert cuda_lib.device_timeouts() == 0
+
+
+def test_static_weights_matches_default_launch(cuda_lib):
+    items, Ws, x_dev = _stream_set(cuda_lib, 1, 92)
+    for K, t in x_dev.items():
+        t.copy_(torch.from_numpy(wl.activation(70, K, "x", 1, K)).to("cuda"))
+    torch.cuda.synchronize()
+    descs = cuda_lib.make_descs(items)
+    cuda_lib.matmul_q_batched(descs, 1, 4, 64, cuda_lib.BC_MODE_PACKED_INT4)
+    torch.cuda.synchronize()
+    first = [host(it[4]).copy() for it in items]
+    for it in items:
+        it[4].fill_(float("nan"))
+    cuda_lib.matmul_q_batched(descs, 1, 4, 64, cuda_lib.BC_MODE_PACKED_INT4,
+                              static_weights=True)
+    torch.cuda.synchronize()
+    for i, it in enumerate(items):
+        assert np.array_equal(host(it[4]), first[i]), f"matrix {i}"
+
+
+def test_batched_ex_rejects_unknown_flags(cuda_lib):
+    items, _, _ = _stream_set(cuda_lib, 1, 93, count=2)
+    descs = cuda_lib.make_descs(items)
+    st = cuda_lib.lib.bc_matmul_q_batched_ex(descs, len(descs), 1, 4, 64,
+                                             cuda_lib.BC_MODE_PACKED_INT4,
+                                             cuda_lib.BC_F32, None, 0, 0x80, None)
+    assert st == cuda_lib.BC_ERR_INVALID_ARG
+
+
+def test_stream_activation_outliers(cuda_lib):
+    """Activations are staged as integers relative to their 64-group maximum;
+    a group holding an outlier 10^4 times its neighbours must still meet the
+    fp32 bar (the neighbours keep ~2^-13 relative precision or better)."""
+    rng = np.random.default_rng(77)
+    items, refs = [], []
+    x = wl.activation(80, 896, "x", 1, 896).copy()
+    x[0, ::64] *= 1.0e4                  # one outlier in every group
+    x[0, 5::64] = 1.0e-30                # and a value far below everything
+    xd = dev(x)
+    for i in range(160):
+        N, K = (896, 896)
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+        Wd = dev(W)
+        s, z = cuda_lib.group_params(Wd, 4, 64, torch.float16)
+        Wk = cuda_lib.pack_int4(Wd, s, z)
+        y = torch.full((1, N), float("nan"), device="cuda")
+        items.append((xd, Wk, s, z, y))
+        if i < 3:
+            refs.append(oracle.matmul_q(x, W, 4, 64, "packed"))
+    cuda_lib.matmul_q_batched(cuda_lib.make_descs(items), 1, 4, 64,
+                              cuda_lib.BC_MODE_PACKED_INT4)
+    torch.cuda.synchronize()
+    for i, ref in enumerate(refs):
+        assert_close(host(items[i][4]), ref["y"], ref["A"], TOL_FP32, f"matrix {i}")
+    assert cuda_lib.device_timeouts() == 0
