@@ -230,20 +230,33 @@ def build_workload(qmm, torch, name: str, copies: int):
     shape_set, layers, mode, bits, group, M, seed = WORKLOADS[name]
     mats = wl.layer_set(shape_set, layers)
     sigma = wl.SIGMA[shape_set]
-    xs_host, xs_dev = {}, {}
-    per_copy = [[] for _ in range(copies)]
-    ys = []
+    prefill = is_prefill(name)
+    # every distinct x lives in one device buffer and every y in another, so a
+    # step's inputs and outputs each cross PCIe as one copy (e2e)
+    x_keys, x_off, x_total = [], {}, 0
     for m in mats:
         key = (m.layer, m.x_tag)
-        if key not in xs_dev:
-            xh = wl.activation(seed, m.layer, m.x_tag, M, m.K)
-            if is_prefill(name):
-                xh = wl.bf16_bits(xh).view(np.int16)
-                xs_host[key] = xh
-                xs_dev[key] = torch.from_numpy(xh).cuda().view(torch.bfloat16)
-            else:
-                xs_host[key] = xh
-                xs_dev[key] = torch.from_numpy(xh).cuda()
+        if key not in x_off:
+            x_off[key] = (x_total, m.K)
+            x_keys.append(key)
+            x_total += M * m.K
+    x_all_host = np.empty(x_total, dtype=np.int16 if prefill else np.float32)
+    for key in x_keys:
+        off, K = x_off[key]
+        xh = wl.activation(seed, key[0], key[1], M, K)
+        x_all_host[off:off + M * K] = (wl.bf16_bits(xh).view(np.int16) if prefill
+                                       else xh).reshape(-1)
+    x_all_dev = torch.from_numpy(x_all_host).cuda()
+    if prefill:
+        x_all_dev = x_all_dev.view(torch.bfloat16)
+    xs_dev = {key: x_all_dev[off:off + M * K].view(M, K)
+              for key, (off, K) in x_off.items()}
+    y_all_dev = torch.empty(sum(M * m.N for m in mats), dtype=torch.float32, device="cuda")
+    per_copy = [[] for _ in range(copies)]
+    ys = []
+    y_at = 0
+    for m in mats:
+        key = (m.layer, m.x_tag)
         W = torch.from_numpy(wl.weight(seed, m.layer, m.name, m.K, m.N, sigma)).cuda()
         if mode == "packed":
             s, z = qmm.group_params(W, 4, 64, torch.float16)
@@ -255,7 +268,8 @@ def build_workload(qmm, torch, name: str, copies: int):
         else:
             s, z = qmm.group_params(W, bits, group, torch.float32)
             Wk = W
-        y = torch.empty((M, m.N), dtype=torch.float32, device="cuda")
+        y = y_all_dev[y_at:y_at + M * m.N].view(M, m.N)
+        y_at += M * m.N
         ys.append(y)
         for c in range(copies):
             if c == 0:
@@ -266,9 +280,9 @@ def build_workload(qmm, torch, name: str, copies: int):
                                     None if z is None else z.clone(), y))
     torch.cuda.synchronize()
     descs = [qmm.make_descs(items) for items in per_copy]
-    return {"mats": mats, "descs": descs, "xs_host": xs_host, "xs_dev": xs_dev,
-            "ys": ys, "per_copy": per_copy, "mode": mode, "bits": bits,
-            "group": group, "M": M}
+    return {"mats": mats, "descs": descs, "x_all_host": x_all_host, "x_all_dev": x_all_dev,
+            "xs_dev": xs_dev, "y_all_dev": y_all_dev, "ys": ys, "per_copy": per_copy,
+            "mode": mode, "bits": bits, "group": group, "M": M}
 
 
 def _oracle_x(name: str, seed: int, m) -> np.ndarray:
@@ -471,19 +485,17 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = agg["ms"] / args.steps
 
     # ---- end to end through the public API: pinned host x in, y out ----
-    xs_pinned = {k: torch.from_numpy(v).pin_memory() for k, v in W["xs_host"].items()}
+    x_pinned = torch.from_numpy(W["x_all_host"]).pin_memory()
     if prefill:
-        xs_pinned = {k: v.view(torch.bfloat16) for k, v in xs_pinned.items()}
-    ys_pinned = [torch.empty(y.shape, dtype=torch.float32).pin_memory() for y in W["ys"]]
-    h2d = sum(v.numel() * v.element_size() for v in xs_pinned.values())
-    d2h = sum(y.numel() * 4 for y in ys_pinned)
+        x_pinned = x_pinned.view(torch.bfloat16)
+    y_pinned = torch.empty(W["y_all_dev"].shape, dtype=torch.float32).pin_memory()
+    h2d = x_pinned.numel() * x_pinned.element_size()
+    d2h = y_pinned.numel() * 4
 
-    def e2e_step(i):
-        for k, v in xs_pinned.items():
-            W["xs_dev"][k].copy_(v, non_blocking=True)
+    def e2e_step(i):      # every x of the step in, the step, every y out
+        W["x_all_dev"].copy_(x_pinned, non_blocking=True)
         step(i)
-        for yd, yh in zip(W["ys"], ys_pinned):
-            yh.copy_(yd, non_blocking=True)
+        y_pinned.copy_(W["y_all_dev"], non_blocking=True)
 
     for i in range(3):
         e2e_step(i)

@@ -5,7 +5,7 @@
 // ~130-200 KB per SM in flight, with the arithmetic per weight cut down until
 // the stream, not the issue slots, sets the pace.
 //
-// One CTA per SM, persistent over a byte-balanced contiguous range of
+// One CTA per SM, persistent over a cost-balanced contiguous range of
 // "units" (128 weight rows of one matrix) that spans every matrix of a
 // grouped launch (Enargeia, "One decode step": hundreds of passes per token
 // are one launch here).  Warp roles:
@@ -14,14 +14,16 @@
 //               128 bytes, 128-byte swizzle) into a ring of up to 6 stages with
 //               full/empty mbarriers.
 //   warp 1      activation stager: the x of each new matrix goes into one of
-//               two smem slots (see below); the first slot is filled by every
-//               warp but the loader together before streaming starts.
-//   warp 2      scale/zero stager (packed): the fp16 scales and zeros of each
-//               stage (128 rows x 8 groups) into a ring slot beside it, with
-//               coalesced loads a stage ahead of the stores; its arrival is
-//               the second one each full barrier counts.
-//   warps 3-10  consumers: warp g handles rows 16g..16g+15 of each unit over
-//               both 128-byte windows of every stage.
+//               two smem slots (see below); the first slot is filled by the
+//               stager and the consumers together before streaming starts.
+//   warps 2-3   (packed) scale/zero stagers: the fp16 scales and zeros of each
+//               stage (64 rows x 8 groups each) into a ring slot beside it,
+//               with coalesced loads two stages ahead of the stores; each
+//               arrival is one more that the stage's full barrier counts.
+//   consumers   packed: 8 warps, warp g owns rows 16g..16g+15 of each unit over
+//               both 128-byte windows of every stage (tensor cores).  Runtime:
+//               16 warps of 8 rows each (CUDA-core quantizer, which needs more
+//               warps in flight to hide its latency).
 //
 // Packed int4 (Enargeia, "Four bits per weight": codes unpacked in registers,
 // never written back) runs on the int8 tensor cores (mma.sync m16n8k32
@@ -68,11 +70,16 @@ constexpr int kRows = 128;              // weight rows per unit
 constexpr int kChunk = 256;             // bytes of a row per stage
 constexpr int kBoxBytes = kRows * 128;  // one TMA box: 128 rows x 128 bytes, SW128
 constexpr int kStageBytes = 2 * kBoxBytes;
-constexpr int kConsumers = 8;
-constexpr int kStagers = 1 + kConsumers;   // warps that fill the first x slot
-constexpr int kSzWarps = 2;                // scale/zero stagers, 64 rows each
-constexpr int kFirstConsumer = 2 + kSzWarps;  // warps: loader, x stager, scale/zero stagers
-constexpr int kThreads = 32 * (kFirstConsumer + kConsumers);
+// Warp roles per mode.  Packed: loader, x stager, two scale/zero stagers
+// (64 rows each), 8 consumers of 16 rows.  Runtime: loader, x stager, 16
+// consumers of 8 rows (the CUDA-core quantizer wants more warps in flight).
+template <bool PACKED> struct Roles {
+    static constexpr int consumers = PACKED ? 8 : 16;
+    static constexpr int sz_warps = PACKED ? 2 : 0;
+    static constexpr int first_consumer = 2 + sz_warps;
+    static constexpr int threads = 32 * (first_consumer + consumers);
+    static constexpr int stagers = 1 + consumers;    // warps that fill the first x slot
+};
 constexpr int kSzBytes = 2 * kRows * 16;   // packed: fp16 scales + zeros of a stage
 constexpr int kMaxJobs = 168;
 constexpr int kMaxCtas = 160;
@@ -709,47 +716,42 @@ __device__ __forceinline__ void consume_packed_mx(
 }
 
 // ---- runtime (RTN) consumer --------------------------------------------------
-// Warp rg owns rows 16rg..16rg+15; lane (row r16, half part) takes 32 of the
-// 64 k of each window, so a row's dot product is spread over two lanes.
+// Warp cw owns rows 8cw..8cw+7 of each unit.  Lane (row r8 = lane & 7, part
+// p = lane >> 3) takes 32 of the 128 k of a stage: window p >> 1, half p & 1.
+// A quarter-warp thus reads eight different rows at one 16-byte offset,
+// which the 128-byte swizzle spreads over all banks.
 template <int MT>
 __device__ __forceinline__ void consume_runtime(
     const StreamParams &P, const StreamJob *jobs, int jf, int jc, uint8_t *smem,
     uint8_t *xslots, uint64_t *full, uint64_t *empty, uint64_t *xfull, uint64_t *xempty,
-    volatile int *abort_flag, int u0, int u1, int rg, int lane) {
+    volatile int *abort_flag, int u0, int u1, int cw, int lane) {
     const int S = P.stages;
-    const int r16 = lane >> 1, part = lane & 1;       // row in group, 32-k half
-    const int rr = 16 * rg + r16;
+    const int r8 = lane & 7, part = lane >> 3;
+    const int w = part >> 1, half = part & 1;
+    const int rr = 8 * cw + r8;
     const float L = (float)((1 << P.bits) - 1);
     const bool pass = P.bits == 16;
     XCursor xc;
     Walk k{u0, 0, jf, 0, 0u};
-    // (scale, zero) of this lane's two windows for the current and next stage
-    auto load_sz = [&](const Walk &q, float4 &o) {
+    // (scale, zero) of this lane's 32 k for a stage
+    auto load_sz = [&](const Walk &q, float2 &o) {
         const StreamJob &J = jobs[q.jidx];
         const int row = (q.u - J.unit_begin) * kRows + rr;
-        o = make_float4(1.0f, 0.0f, 1.0f, 0.0f);
-        if (pass || row >= J.N) return;
-        const float *Sf = reinterpret_cast<const float *>(J.s);
-        const float *Zf = reinterpret_cast<const float *>(J.z);
-        const int64_t gr = (int64_t)row * (J.K / J.group);
-        const int k0 = q.kc * 128;
-        if (k0 < J.K) {
-            o.x = __ldg(Sf + gr + k0 / J.group);
-            o.y = __ldg(Zf + gr + k0 / J.group);
-        }
-        if (k0 + 64 < J.K) {
-            o.z = __ldg(Sf + gr + (k0 + 64) / J.group);
-            o.w = __ldg(Zf + gr + (k0 + 64) / J.group);
-        }
+        const int k0 = q.kc * 128 + w * 64 + half * 32;
+        o = make_float2(1.0f, 0.0f);
+        if (pass || row >= J.N || k0 >= J.K) return;
+        const int64_t gi = (int64_t)row * (J.K / J.group) + k0 / J.group;
+        o.x = __ldg(reinterpret_cast<const float *>(J.s) + gi);
+        o.y = __ldg(reinterpret_cast<const float *>(J.z) + gi);
     };
-    float4 sz_a, sz_b = make_float4(1.0f, 0.0f, 1.0f, 0.0f);
+    float2 sz_a, sz_b = make_float2(1.0f, 0.0f);
     load_sz(k, sz_a);
     float yacc[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) yacc[m] = 0.0f;
     if (!x_enter(xc, jobs[k.jidx], true, xslots, P.xslot_bytes, xfull, xempty, abort_flag, lane))
         return;
-    auto step = [&](const float4 use, float4 &fill) -> bool {
+    auto step = [&](const float2 use, float2 &fill) -> bool {
         const StreamJob &J = jobs[k.jidx];
         const int row = (k.u - J.unit_begin) * kRows + rr;
         const int kchunks = kchunks_of<false>(J.K);
@@ -757,82 +759,79 @@ __device__ __forceinline__ void consume_runtime(
         const bool more = k.next(jobs, jc, u1, kchunks, S, n);
         if (more) load_sz(n, fill);
         if (!mbar_wait(smem_u32(&full[k.sidx]), k.sph, abort_flag)) return true;
-        const uint8_t *stage = smem + k.sidx * kStageBytes;
+        const uint8_t *box = smem + k.sidx * kStageBytes + w * kBoxBytes;
         const int kp = kpad_of<false>(J.K);
+        const float s_cur = use.x, z_cur = use.y;
+        const int k0 = k.kc * 128 + w * 64 + half * 32;     // this lane's 32 k
+        float part_acc[MT];
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
-            const float s_cur = w ? use.z : use.x, z_cur = w ? use.w : use.y;
-            const int k0 = k.kc * 128 + w * 64 + part * 32;     // this thread's 32 k
-            float part_acc[MT];
+        for (int m = 0; m < MT; ++m) part_acc[m] = 0.0f;
+        if (row < J.N && k0 < J.K) {
+            const float inv = rcp_approx(s_cur);
+            const float lo_c = -z_cur, hi_c = L - z_cur;
+            const float thr = 0.5f - (fmaxf(fabsf(lo_c), fabsf(hi_c)) + 2.0f) *
+                                         4.76837158203125e-07f;   // 2^-21
 #pragma unroll
-            for (int m = 0; m < MT; ++m) part_acc[m] = 0.0f;
-            if (row < J.N && k0 < J.K) {
-                const uint8_t *box = stage + w * kBoxBytes;
-                const float inv = rcp_approx(s_cur);
-                const float lo_c = -z_cur, hi_c = L - z_cur;
-                const float thr = 0.5f - (fmaxf(fabsf(lo_c), fabsf(hi_c)) + 2.0f) *
-                                             4.76837158203125e-07f;   // 2^-21
+            for (int c8 = 0; c8 < 4; ++c8) {
+                const int u16 = half * 4 + c8;
+                const uint4 raw = *reinterpret_cast<const uint4 *>(
+                    box + rr * 128 + ((u16 ^ (rr & 7)) << 4));
+                const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
+                float wv[8];
 #pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
-                    const int u16 = part * 4 + c8;
-                    const uint4 raw = *reinterpret_cast<const uint4 *>(
-                        box + rr * 128 + ((u16 ^ (rr & 7)) << 4));
-                    const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
-                    float wv[8];
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f2 = __half22float2(h2[i]);
+                    wv[2 * i] = f2.x;
+                    wv[2 * i + 1] = f2.y;
+                }
+                float cq[8];
+                if (pass) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 f2 = __half22float2(h2[i]);
-                        wv[2 * i] = f2.x;
-                        wv[2 * i + 1] = f2.y;
+                    for (int i = 0; i < 8; ++i) cq[i] = wv[i];
+                } else {
+                    float emax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float v = fmaf(wv[i], inv, kMagic);
+                        const float r = v - kMagic;
+                        const float ee = fmaf(wv[i], inv, -r);
+                        emax = fmaxf(emax, fabsf(ee));
+                        cq[i] = fminf(fmaxf(r, lo_c), hi_c);
                     }
-                    float cq[8];
-                    if (pass) {
+                    if (emax > thr) {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) cq[i] = wv[i];
-                    } else {
-                        float emax = 0.0f;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float v = fmaf(wv[i], inv, kMagic);
-                            const float r = v - kMagic;
-                            const float ee = fmaf(wv[i], inv, -r);
-                            emax = fmaxf(emax, fabsf(ee));
-                            cq[i] = fminf(fmaxf(r, lo_c), hi_c);
-                        }
-                        if (emax > thr) {
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                cq[i] = centered_code_exact(wv[i], s_cur, z_cur, L);
-                        }
-                    }
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        const float *xr = reinterpret_cast<const float *>(xc.xs) +
-                                          (int64_t)m * kp + k0 + c8 * 8;
-                        const float4 xa = *reinterpret_cast<const float4 *>(xr);
-                        const float4 xb = *reinterpret_cast<const float4 *>(xr + 4);
-                        float p = part_acc[m];
-                        p = fmaf(xa.x, cq[0], p);
-                        p = fmaf(xa.y, cq[1], p);
-                        p = fmaf(xa.z, cq[2], p);
-                        p = fmaf(xa.w, cq[3], p);
-                        p = fmaf(xb.x, cq[4], p);
-                        p = fmaf(xb.y, cq[5], p);
-                        p = fmaf(xb.z, cq[6], p);
-                        p = fmaf(xb.w, cq[7], p);
-                        part_acc[m] = p;
+                        for (int i = 0; i < 8; ++i)
+                            cq[i] = centered_code_exact(wv[i], s_cur, z_cur, L);
                     }
                 }
-            }
 #pragma unroll
-            for (int m = 0; m < MT; ++m) yacc[m] = fmaf(part_acc[m], s_cur, yacc[m]);
+                for (int m = 0; m < MT; ++m) {
+                    const float *xr = reinterpret_cast<const float *>(xc.xs) +
+                                      (int64_t)m * kp + k0 + c8 * 8;
+                    const float4 xa = *reinterpret_cast<const float4 *>(xr);
+                    const float4 xb = *reinterpret_cast<const float4 *>(xr + 4);
+                    float p = part_acc[m];
+                    p = fmaf(xa.x, cq[0], p);
+                    p = fmaf(xa.y, cq[1], p);
+                    p = fmaf(xa.z, cq[2], p);
+                    p = fmaf(xa.w, cq[3], p);
+                    p = fmaf(xb.x, cq[4], p);
+                    p = fmaf(xb.y, cq[5], p);
+                    p = fmaf(xb.z, cq[6], p);
+                    p = fmaf(xb.w, cq[7], p);
+                    part_acc[m] = p;
+                }
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));
-        if (n.kc == 0 || !more) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) yacc[m] = fmaf(part_acc[m], s_cur, yacc[m]);
+        if (n.kc == 0 || !more) {       // unit done: the four lanes of a row
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
-                yacc[m] += __shfl_xor_sync(0xffffffffu, yacc[m], 1);
+                yacc[m] += __shfl_xor_sync(0xffffffffu, yacc[m], 8);
+                yacc[m] += __shfl_xor_sync(0xffffffffu, yacc[m], 16);
                 if (part == 0 && row < J.N && m < P.M) J.y[(int64_t)m * J.N + row] = yacc[m];
                 yacc[m] = 0.0f;
             }
@@ -848,14 +847,14 @@ __device__ __forceinline__ void consume_runtime(
     }
 }
 
-// Prefetch of the CTA's activations into L2 by staging warp `wi` of kStagers.
+// Prefetch of the CTA's activations into L2 by staging warp `wi` of `nw`.
 __device__ __forceinline__ void prefetch_xs(const StreamParams &P, const StreamJob *jobs, int jf,
-                                            int jc, int wi, int lane) {
+                                            int jc, int wi, int nw, int lane) {
     for (int j = jf; j < jc; ++j) {
         const StreamJob &J = jobs[j];
         if (j > jf && jobs[j - 1].x == J.x) continue;
         const int lines = (int)(((int64_t)P.M * J.K * 4 + 127) / 128);
-        for (int l = 32 * wi + lane; l < lines; l += 32 * kStagers)
+        for (int l = 32 * wi + lane; l < lines; l += 32 * nw)
             prefetch_l2(reinterpret_cast<const char *>(J.x) + (int64_t)l * 128);
     }
 }
@@ -905,7 +904,7 @@ __device__ __forceinline__ void sz_stager(const StreamParams &P, const StreamJob
 }
 
 template <bool PACKED, int MT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<PACKED>::threads, 1)
 gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -920,6 +919,7 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     uint64_t *xfirst = xempty + 3;      // the first x slot is complete
     StreamJob *jobs_sm = reinterpret_cast<StreamJob *>(bars + 2 * S + 8);
 
+    using RL = Roles<PACKED>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u0 = P.cta_begin[blockIdx.x], u1 = P.cta_begin[blockIdx.x + 1];
     // the next launch on the stream may start as SMs free up (no-op unless it
@@ -933,20 +933,20 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
         const uint4 *src = reinterpret_cast<const uint4 *>(&P.jobs[jf]);
         uint4 *dst = reinterpret_cast<uint4 *>(jobs_sm);
         const int n16 = (jc - jf) * (int)(sizeof(StreamJob) / 16);
-        for (int i = threadIdx.x; i < n16; i += kThreads) dst[i] = src[i];
+        for (int i = threadIdx.x; i < n16; i += RL::threads) dst[i] = src[i];
     }
     const StreamJob *jobs = jobs_sm - jf;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&full[s]), PACKED ? 1 + kSzWarps : 1);
-            mbar_init(smem_u32(&empty[s]), kConsumers);
+            mbar_init(smem_u32(&full[s]), 1 + RL::sz_warps);
+            mbar_init(smem_u32(&empty[s]), RL::consumers);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&xfull[b]), 32);
-            mbar_init(smem_u32(&xempty[b]), kConsumers);
+            mbar_init(smem_u32(&xempty[b]), RL::consumers);
         }
-        mbar_init(smem_u32(xfirst), kStagers);
+        mbar_init(smem_u32(xfirst), RL::stagers);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -955,8 +955,8 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     // stream: queued behind the first ring fill they would hold up the start.
     // (After an early start they may not be written yet: the staging warps
     // prefetch them once the previous kernel has completed.)
-    if (!P.early && warp >= 1 && warp < 1 + kStagers && u0 < u1)
-        prefetch_xs(P, jobs, jf, jc, warp - 1, lane);
+    if (!P.early && warp >= 1 && warp < 1 + RL::stagers && u0 < u1)
+        prefetch_xs(P, jobs, jf, jc, warp - 1, RL::stagers, lane);
     if (!P.early) __syncthreads();
 
     if (warp == 0) {
@@ -1031,7 +1031,7 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
             }
         }
         __syncwarp();
-    } else if (warp >= 2 && warp < kFirstConsumer) {
+    } else if (warp >= 2 && warp < RL::first_consumer) {
         // ---------------- scale / zero stagers (packed) ----------------
         if constexpr (PACKED) {
             if (u0 < u1)
@@ -1046,11 +1046,12 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
         // waits here, so this grid completes only after it)
         asm volatile("griddepcontrol.wait;" ::: "memory");
         if (P.early && u0 < u1)
-            prefetch_xs(P, jobs, jf, jc, warp == 1 ? 0 : warp - kFirstConsumer + 1, lane);
+            prefetch_xs(P, jobs, jf, jc, warp == 1 ? 0 : warp - RL::first_consumer + 1,
+                        RL::stagers, lane);
         if (u0 < u1) {
             const StreamJob &J0 = jobs[jf];
-            stage_x<PACKED>(J0, P.M, xslots, warp == 1 ? 0 : warp - kFirstConsumer + 1,
-                            kStagers, lane);
+            stage_x<PACKED>(J0, P.M, xslots, warp == 1 ? 0 : warp - RL::first_consumer + 1,
+                            RL::stagers, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(xfirst));
             if (warp == 1) {
@@ -1080,7 +1081,7 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
             }
         } else {
             // ---------------- consumers ----------------
-            const int rg = warp - kFirstConsumer;
+            const int rg = warp - RL::first_consumer;
             if (u0 < u1) {
                 if constexpr (PACKED) {
                     if constexpr (MT == 1)
@@ -1124,7 +1125,7 @@ bc_status launch_one(const StreamParams &P, int grid, int smem, cudaStream_t s) 
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(Roles<PACKED>::threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
