@@ -1038,10 +1038,19 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
                 sz_stager(P, jobs, jf, jc, szring, full, empty, abort_flag, u0, u1, warp - 2, lane);
         }
     } else {
-        // the first x slot, by the x stager and the consumers together; each
-        // warp reports on `xfirst`, and the stager turns that into the slot's
-        // first xfull phase once all have
+        // The first two x slots (the CTA's first two activations, in the order
+        // its units meet them), by the x stager and the consumers together:
+        // each warp reports on `xfirst`, and the stager turns that into the
+        // slots' first xfull phases once all have.  A lone stager needs ~8k
+        // cycles for a 4864-wide x; consumers that reach a matrix switch early
+        // would wait for it.
         bool first_ok = true;
+        int j2 = -1;                     // job of the second activation, if any
+        for (int j = jf + 1; j < jc && jobs[j].unit_begin < u1; ++j)
+            if (jobs[j].x != jobs[j - 1].x) {
+                j2 = j;
+                break;
+            }
         // x and y belong to the previous kernel until it completes (every CTA
         // waits here, so this grid completes only after it)
         asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1049,28 +1058,33 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
             prefetch_xs(P, jobs, jf, jc, warp == 1 ? 0 : warp - RL::first_consumer + 1,
                         RL::stagers, lane);
         if (u0 < u1) {
-            const StreamJob &J0 = jobs[jf];
-            stage_x<PACKED>(J0, P.M, xslots, warp == 1 ? 0 : warp - RL::first_consumer + 1,
-                            RL::stagers, lane);
+            const int wi = warp == 1 ? 0 : warp - RL::first_consumer + 1;
+            stage_x<PACKED>(jobs[jf], P.M, xslots, wi, RL::stagers, lane);
+            if (j2 >= 0)
+                stage_x<PACKED>(jobs[j2], P.M, xslots + P.xslot_bytes, wi, RL::stagers, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(xfirst));
             if (warp == 1) {
                 first_ok = mbar_wait(smem_u32(xfirst), 0, abort_flag);
-                if (first_ok) mbar_arrive(smem_u32(&xfull[0]));
+                if (first_ok) {
+                    mbar_arrive(smem_u32(&xfull[0]));
+                    if (j2 >= 0) mbar_arrive(smem_u32(&xfull[1]));
+                }
             }
         }
         if (warp == 1) {
             // ---------------- activation stager ----------------
             const float *cur = nullptr;
             uint32_t e = 0;
+            const uint32_t pre = j2 >= 0 ? 2u : 1u;     // slots filled above
             int js = jf;
             for (int u = u0; u < u1 && first_ok && !*abort_flag; ++u) {
                 js = next_job(jobs, jc, js, u);
                 const StreamJob &J = jobs[js];
                 if (u != u0 && J.x == cur) continue;
                 cur = J.x;
-                if (u == u0) {     // filled above
-                    e = 1;
+                if (e < pre) {
+                    ++e;
                     continue;
                 }
                 const int slot = e & 1;
