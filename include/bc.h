@@ -181,6 +181,14 @@ BC_API bc_status bc_matmul_q_batched(const bc_matmul_desc *descs, int count,
                               bc_mode mode, bc_dtype x_dtype, void *workspace,
                               size_t workspace_bytes, bc_stream_t stream);
 
+/*
+ * bc_workspace_size_batched -- scratch bytes a bc_matmul_q_batched call over
+ * these descriptors needs.  Reads N, K and x of each descriptor: matrices
+ * that name the same non-null x (and K) share scratch, and a size computed
+ * with x = NULL holds for any x pointers of a later call with the same N, K.
+ * Returns 0 for arguments the call would reject, and for calls that need no
+ * scratch (bf16 x, and the decode kernel for fp16 weights or M <= 4).
+ */
 BC_API size_t bc_workspace_size_batched(const bc_matmul_desc *descs, int count,
                                  int64_t M, bc_mode mode, bc_dtype x_dtype);
 

@@ -183,6 +183,7 @@ size_t bc_workspace_size_batched(const bc_matmul_desc *descs, int count,
     if (!device_info(&di)) return 0;
     std::vector<GemvJob> jobs(count);
     for (int i = 0; i < count; ++i) {
+        jobs[i].x = static_cast<const float *>(descs[i].x);   // may be null
         jobs[i].N = descs[i].N;
         jobs[i].K = descs[i].K;
         jobs[i].group = 64;

@@ -362,10 +362,11 @@ bc_status launch_mt(const GemvParams &P, int mt, int grid, cudaStream_t s) {
 }
 
 // Whole launches with at least half an SM's worth of 128-row units per SM
-// go to the streaming kernel; lone small matrices keep the split-K GEMV.
+// go to the streaming kernel (M <= 4, or M <= 16 for packed codes); lone
+// small matrices keep the split-K GEMV.
 bool use_stream(const GemvJob *jobs, int count, int M, bool packed,
                 const DeviceInfo &di) {
-    if (M > 4) return false;
+    if (M > (packed ? 16 : 4)) return false;
     int64_t units = 0;
     for (int i = 0; i < count; ++i) units += (jobs[i].N + 127) / 128;
     if (units < di.sm_count / 2) return false;
@@ -377,7 +378,8 @@ bool use_stream(const GemvJob *jobs, int count, int M, bool packed,
 size_t gemv_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed,
                             int sm_count) {
     DeviceInfo di;
-    if (device_info(&di) && use_stream(jobs, count, M, packed, di)) return 0;
+    if (device_info(&di) && use_stream(jobs, count, M, packed, di))
+        return gemv_stream_workspace_bytes(jobs, count, M, packed);
     size_t worst = 0;
     for (int b = 0; b < count; b += kMaxJobs) {
         const int n = std::min(kMaxJobs, count - b);
@@ -393,7 +395,8 @@ bc_status launch_gemv(const GemvJob *jobs, int count, int M, int bits,
     DeviceInfo di;
     if (!device_info(&di)) return BC_ERR_CUDA;
     if (use_stream(jobs, count, M, packed, di))
-        return launch_gemv_stream(jobs, count, M, bits, packed, s, early_start);
+        return launch_gemv_stream(jobs, count, M, bits, packed, s, early_start, workspace,
+                                  ws_bytes);
     // ~32 KB of kernel parameters, kept off the stack; the launch copies it.
     thread_local GemvParams *Pp = nullptr;
     if (!Pp) Pp = new GemvParams();

@@ -83,7 +83,14 @@ template <bool PACKED> struct Roles {
 constexpr int kSzBytes = 2 * kRows * 16;   // packed: fp16 scales + zeros of a stage
 constexpr int kMaxJobs = 168;
 constexpr int kMaxCtas = 160;
-constexpr int kMaxM = 4;
+constexpr int kMaxM = 4;                 // rows of x held in a per-matrix smem slot
+constexpr int kMaxMChunk = 16;           // rows of x streamed per stage from the workspace
+// Chunk mode (M = 5..16, packed): the activation digits of one 512-k stage
+// chunk for one x row -- 16 rows (digit d, lane t) of kXcRS words (16 units x
+// 2 parities + 4 words of padding against bank conflicts), then (f, X~) of
+// the chunk's 8 groups for both digit pairs.
+constexpr int kXcRS = 36;
+constexpr int kXcRowBytes = 16 * kXcRS * 4 + 2 * 8 * 8;   // 2432
 constexpr int kXP = 26;                 // bits of the odd-k activation integers (even: +4)
 constexpr long long kWaitCycles = 4000000000LL;
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
@@ -105,6 +112,7 @@ struct __align__(64) StreamParams {
     int count, total_units, M, bits;
     int xslot_bytes, stages, max_cta_jobs;
     int early;                    // launched as a programmatic dependent launch
+    int xchunk_bytes;             // chunk mode: bytes of one stage's x chunk (MT rows)
 };
 static_assert(sizeof(StreamParams) <= 32000, "kernel parameter space");
 
@@ -180,6 +188,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
         : "memory");
 }
+// Contiguous global -> shared copy completing on `bar` (16-byte aligned both
+// ends, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
 __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
@@ -242,6 +259,42 @@ __device__ __forceinline__ void transpose4(const uint32_t (&w)[4], uint32_t (&o)
     o[3] = prmt(t1, t3, 0x7632);
 }
 
+// Digits of one 64-group held by 8 lanes (lane j has k = 8j .. 8j+7 of it):
+// the digit words of this lane's even-k values (te) and odd-k slots (to,
+// carrying X_odd - X_even), byte i of each at k = 8j + 2i; and, on every
+// lane of the 8, the group's f = 2^(E-30) and X~ = f * sum(X_e + 16 X_o).
+__device__ __forceinline__ void group_digits(const float (&v)[8], uint32_t (&te)[4],
+                                             uint32_t (&to)[4], float &f, float &xt) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    // max|x| < 2^E; E >= -96 keeps every scale below a normal float
+    int E = amax > 0.0f ? (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126 : 0;
+    E = max(E, -96);
+    const float sc_e = __uint_as_float((uint32_t)(127 + kXP + 4 - E) << 23);
+    const float sc_o = __uint_as_float((uint32_t)(127 + kXP - E) << 23);
+    uint32_t de[4], dq[4];
+    long long sum = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int xe = __float2int_rn(v[2 * i] * sc_e);      // |xe| <= 2^30
+        const int xo = __float2int_rn(v[2 * i + 1] * sc_o);  // |xo| <= 2^26
+        sum += (long long)xe + 16ll * xo;
+        de[i] = digits4(xe);
+        dq[i] = digits4(xo - xe);     // odd slots carry X_odd - X_even (raw-byte A)
+    }
+    transpose4(de, te);
+    transpose4(dq, to);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+    f = __uint_as_float((uint32_t)(127 + E - kXP - 4) << 23);
+    xt = (float)((double)f * (double)sum);
+}
+
 // One x row of a packed-mode slot, by warp `widx` of `nw` working together.
 // Eight lanes per 64-group, each with 8 consecutive k (one 32-k unit half).
 __device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
@@ -272,43 +325,74 @@ __device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
             const int g = 4 * (q0 + b * nw) + (lane >> 3);
             const float v[8] = {va[b][0].x, va[b][0].y, va[b][0].z, va[b][0].w,
                                 va[b][1].x, va[b][1].y, va[b][1].z, va[b][1].w};
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-            // max|x| < 2^E; E >= -96 keeps every scale below a normal float
-            int E = amax > 0.0f ? (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126 : 0;
-            E = max(E, -96);
-            const float sc_e = __uint_as_float((uint32_t)(127 + kXP + 4 - E) << 23);
-            const float sc_o = __uint_as_float((uint32_t)(127 + kXP - E) << 23);
-            uint32_t de[4], dq[4];
-            long long sum = 0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int xe = __float2int_rn(v[2 * i] * sc_e);      // |xe| <= 2^30
-                const int xo = __float2int_rn(v[2 * i + 1] * sc_o);  // |xo| <= 2^26
-                sum += (long long)xe + 16ll * xo;
-                de[i] = digits4(xe);
-                dq[i] = digits4(xo - xe);     // odd slots carry X_odd - X_even (raw-byte A)
-            }
             uint32_t te[4], to[4];
-            transpose4(de, te);
-            transpose4(dq, to);
+            float f, xt;
+            group_digits(v, te, to, f, xt);
             const int U = 2 * g + (j >> 2), tt = j & 3;
 #pragma unroll
             for (int d = 0; d < 4; ++d)
                 *reinterpret_cast<uint2 *>(dig + (d * 4 + tt) * rs + 2 * U) =
                     make_uint2(te[d], to[d]);
-            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-            sum += __shfl_xor_sync(0xffffffffu, sum, 4);
             if (j == 0) {
-                const float f = __uint_as_float((uint32_t)(127 + E - kXP - 4) << 23);
-                tab[g] = make_float2(f, (float)((double)f * (double)sum));
+                tab[g] = make_float2(f, xt);
                 tab[gpad + g] = make_float2(f * 65536.0f, 0.0f);
             }
+        }
+    }
+}
+
+// ---- chunk mode: activation digits into the workspace ---------------------------
+// One launch before the streaming kernel turns every distinct x of the call
+// into per-stage chunks: x i, chunk kc, row m at out_i + (kc*MT + m) *
+// kXcRowBytes (rows m >= M are zero).  A warp does one (x, kc, m, half)
+// task: 4 of the chunk's 8 groups.
+struct XdigTask {
+    const float *x;
+    uint8_t *out;
+    int K, task_begin;
+};
+struct XdigParams {
+    XdigTask t[kMaxJobs];
+    int count, M, MT, total;
+};
+__global__ void __launch_bounds__(256) xdig_kernel(const __grid_constant__ XdigParams P) {
+    const int lane = threadIdx.x & 31, j = lane & 7;
+    const int nw = (gridDim.x * blockDim.x) >> 5;
+    for (int task = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; task < P.total; task += nw) {
+        int lo = 0, hi = P.count - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (P.t[mid].task_begin <= task) lo = mid; else hi = mid - 1;
+        }
+        const XdigTask &T = P.t[lo];
+        int r = task - T.task_begin;
+        const int half = r & 1;
+        r >>= 1;
+        const int m = r % P.MT, kc = r / P.MT;
+        const int gl = 4 * half + (lane >> 3);           // group within the chunk
+        const int g = 8 * kc + gl;
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+        if (m < P.M && g < (T.K >> 6)) {
+            const float4 *p = reinterpret_cast<const float4 *>(T.x + (int64_t)m * T.K + 64 * g + 8 * j);
+            const float4 a = __ldg(p), b = __ldg(p + 1);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        }
+        uint32_t te[4], to[4];
+        float f, xt;
+        group_digits(v, te, to, f, xt);
+        uint8_t *row = T.out + ((int64_t)kc * P.MT + m) * kXcRowBytes;
+        uint32_t *dig = reinterpret_cast<uint32_t *>(row);
+        float2 *tab = reinterpret_cast<float2 *>(row + 16 * kXcRS * 4);
+        const int U = 2 * gl + (j >> 2), tt = j & 3;
+#pragma unroll
+        for (int d = 0; d < 4; ++d)
+            *reinterpret_cast<uint2 *>(dig + (d * 4 + tt) * kXcRS + 2 * U) = make_uint2(te[d], to[d]);
+        if (j == 0) {
+            tab[gl] = make_float2(f, xt);
+            tab[8 + gl] = make_float2(f * 65536.0f, 0.0f);
         }
     }
 }
@@ -585,15 +669,19 @@ __device__ __forceinline__ void consume_packed_m1(
     }
 }
 
-// ---- packed consumer, 2 or 4 x rows ------------------------------------------------
+// ---- packed consumer, 2 to 16 x rows ------------------------------------------------
 // Each mma takes one 32-k unit (slots 0-15 even k, 16-31 odd k) and a pair of
-// x rows as B columns (row 2*mp + h in columns 4h..4h+3).
+// x rows as B columns (row 2*mp + h in columns 4h..4h+3).  With 2 or 4 rows
+// the digits come from the matrix's x slot; with 8 or 16 (chunk mode, XC)
+// from the stage's own x chunk, which the loader streams with the weights.
 template <int MT>
 __device__ __forceinline__ void consume_packed_mx(
     const StreamParams &P, const StreamJob *jobs, int jf, int jc, uint8_t *smem,
     const uint8_t *szring, uint8_t *xslots, uint64_t *full, uint64_t *empty, uint64_t *xfull,
-    uint64_t *xempty, volatile int *abort_flag, int u0, int u1, int rg, int lane) {
+    uint64_t *xempty, volatile int *abort_flag, int u0, int u1, int rg, int lane,
+    const uint8_t *xring) {
     constexpr int MP = MT / 2;
+    constexpr bool XC = MT > kMaxM;
     const int S = P.stages;
     const int gq = lane >> 2, t = lane & 3;
     // ldmatrix: this lane gives the address of row lrow of unit (2j + (lane>>4))
@@ -610,13 +698,21 @@ __device__ __forceinline__ void consume_packed_mx(
     float ya[MP], yb[MP];
 #pragma unroll
     for (int p = 0; p < MP; ++p) ya[p] = yb[p] = 0.0f;
-    if (!x_enter(xc, jobs[k.jidx], true, xslots, P.xslot_bytes, xfull, xempty, abort_flag, lane))
+    if (!XC && !x_enter(xc, jobs[k.jidx], true, xslots, P.xslot_bytes, xfull, xempty,
+                        abort_flag, lane))
         return;
     auto step = [&]() -> bool {
         const StreamJob &J = jobs[k.jidx];
         const int kch = kchunks_of<true>(J.K);
-        const int rs = dig_rs(kch);
-        const int mb = xrow_bytes<true>(J.K);
+        // x rows: slot rows of `mb` bytes (digit stride rs, k offset of this
+        // chunk), or chunk rows of kXcRowBytes
+        const int rs = XC ? kXcRS : dig_rs(kch);
+        const int mb = XC ? kXcRowBytes : xrow_bytes<true>(J.K);
+        const uint8_t *xb = XC ? xring + k.sidx * P.xchunk_bytes : xc.xs;
+        const int u_off = XC ? 0 : 16 * k.kc;            // unit offset of this chunk
+        const int tab_off = XC ? 16 * kXcRS * 4 : 64 * rs;
+        const int g_off = XC ? 0 : 8 * k.kc;              // group offset of this chunk
+        const int gpad = XC ? 8 : 8 * kch;
         if (!mbar_wait(smem_u32(&full[k.sidx]), k.sph, abort_flag)) return true;
         const uint32_t box0 = smem_u32(smem + k.sidx * kStageBytes);
         // scales / zeros of rows ra, ra+8, groups 4w..4w+3 of both windows
@@ -641,7 +737,7 @@ __device__ __forceinline__ void consume_packed_mx(
             for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) hi[j][i] = R[j][i] & 0xF0F0F0F0u;
-            if (w == 1) {
+            if (!XC && w == 1) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));   // stage consumed
             }
@@ -661,8 +757,8 @@ __device__ __forceinline__ void consume_packed_mx(
             for (int mp = 0; mp < MP; ++mp) {
                 // B: this lane's words for units 0..7 of the window, both parities
                 const uint32_t *xd =
-                    reinterpret_cast<const uint32_t *>(xc.xs + (2 * mp + bh) * mb) +
-                    (bd * 4 + t) * rs + 2 * (16 * k.kc + 8 * w);
+                    reinterpret_cast<const uint32_t *>(xb + (2 * mp + bh) * mb) +
+                    (bd * 4 + t) * rs + 2 * (u_off + 8 * w);
                 uint4 Q[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) Q[j] = reinterpret_cast<const uint4 *>(xd)[j];
@@ -674,7 +770,7 @@ __device__ __forceinline__ void consume_packed_mx(
                     mma_i8(C[j], R[j][2], R[j][3], hi[j][2], hi[j][3], Q[j].z, Q[j].w);
                 }
                 const float *tb = reinterpret_cast<const float *>(
-                    xc.xs + (2 * mp + eh) * mb + 64 * rs + 8 * (ep * 8 * kch + 8 * k.kc + 4 * w));
+                    xb + (2 * mp + eh) * mb + tab_off + 8 * (ep * gpad + g_off + 4 * w));
                 const float4 t01 = reinterpret_cast<const float4 *>(tb)[0];
                 const float4 t23 = reinterpret_cast<const float4 *>(tb)[1];
                 const float f[4] = {t01.x, t01.z, t23.x, t23.z};
@@ -687,6 +783,10 @@ __device__ __forceinline__ void consume_packed_mx(
                     yb[mp] = fmaf(sb[g], fmaf(f[g], vb, -zb[g] * X[g]), yb[mp]);
                 }
             }
+        }
+        if (XC) {        // the stage's x chunk was read up to the last row pair
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));
         }
         Walk n;
         const bool more = k.next(jobs, jc, u1, kch, S, n);
@@ -705,8 +805,9 @@ __device__ __forceinline__ void consume_packed_mx(
             }
         }
         if (!more) return true;
-        if (n.kc == 0 && !x_enter(xc, jobs[n.jidx], false, xslots, P.xslot_bytes, xfull,
-                                  xempty, abort_flag, lane))
+        if (!XC && n.kc == 0 &&
+            !x_enter(xc, jobs[n.jidx], false, xslots, P.xslot_bytes, xfull, xempty, abort_flag,
+                     lane))
             return true;
         k = n;
         return false;
@@ -910,8 +1011,10 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int S = P.stages;
+    constexpr bool XC = PACKED && MT > kMaxM;         // x streamed per stage
     uint8_t *szring = smem + S * kStageBytes;
-    uint8_t *xslots = szring + (PACKED ? S * kSzBytes : 0);
+    uint8_t *xring = szring + (PACKED ? S * kSzBytes : 0);     // chunk mode only
+    uint8_t *xslots = xring + (XC ? S * P.xchunk_bytes : 0);
     uint64_t *bars = reinterpret_cast<uint64_t *>(xslots + 2 * P.xslot_bytes);
     uint64_t *full = bars, *empty = bars + S;
     uint64_t *xfull = bars + 2 * S, *xempty = xfull + 2;
@@ -955,12 +1058,14 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     // stream: queued behind the first ring fill they would hold up the start.
     // (After an early start they may not be written yet: the staging warps
     // prefetch them once the previous kernel has completed.)
-    if (!P.early && warp >= 1 && warp < 1 + RL::stagers && u0 < u1)
+    if (!XC && !P.early && warp >= 1 && warp < 1 + RL::stagers && u0 < u1)
         prefetch_xs(P, jobs, jf, jc, warp - 1, RL::stagers, lane);
     if (!P.early) __syncthreads();
 
     if (warp == 0) {
         // ---------------- loader ----------------
+        // chunk mode: the x chunks are written by the kernel just before
+        if (XC) asm volatile("griddepcontrol.wait;" ::: "memory");
         const uint64_t policy = evict_first_policy();
         uint32_t g = 0, armed = 0;
         int jw = jf;
@@ -993,11 +1098,17 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
                     // a window wholly past the row end is not loaded: its codes
                     // meet zero activation digits (packed) or are skipped (runtime)
                     const int nbox = (rbytes - kc * kChunk) > 128 ? 2 : 1;
-                    mbar_expect_tx(fb, (uint32_t)(nbox * kBoxBytes));
+                    mbar_expect_tx(fb, (uint32_t)(nbox * kBoxBytes) +
+                                           (XC ? (uint32_t)P.xchunk_bytes : 0u));
                     const uint32_t st = smem_u32(smem + s * kStageBytes);
                     for (int b = 0; b < nbox; ++b)
                         tma_load_2d(st + b * kBoxBytes, &P.wmap[j], kc * kChunk + b * 128, r0, fb,
                                     policy);
+                    if (XC)      // job.x holds this matrix's x chunks in chunk mode
+                        bulk_load(smem_u32(xring + s * P.xchunk_bytes),
+                                  reinterpret_cast<const uint8_t *>(J.x) +
+                                      (int64_t)kc * P.xchunk_bytes,
+                                  (uint32_t)P.xchunk_bytes, fb);
                 }
                 armed |= 1u << s;
                 if (PACKED && kc == 0) {
@@ -1046,7 +1157,7 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
         // would wait for it.
         bool first_ok = true;
         int j2 = -1;                     // job of the second activation, if any
-        for (int j = jf + 1; j < jc && jobs[j].unit_begin < u1; ++j)
+        for (int j = jf + 1; !XC && j < jc && jobs[j].unit_begin < u1; ++j)
             if (jobs[j].x != jobs[j - 1].x) {
                 j2 = j;
                 break;
@@ -1054,10 +1165,10 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
         // x and y belong to the previous kernel until it completes (every CTA
         // waits here, so this grid completes only after it)
         asm volatile("griddepcontrol.wait;" ::: "memory");
-        if (P.early && u0 < u1)
+        if (!XC && P.early && u0 < u1)
             prefetch_xs(P, jobs, jf, jc, warp == 1 ? 0 : warp - RL::first_consumer + 1,
                         RL::stagers, lane);
-        if (u0 < u1) {
+        if (!XC && u0 < u1) {
             const int wi = warp == 1 ? 0 : warp - RL::first_consumer + 1;
             stage_x<PACKED>(jobs[jf], P.M, xslots, wi, RL::stagers, lane);
             if (j2 >= 0)
@@ -1073,7 +1184,8 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
             }
         }
         if (warp == 1) {
-            // ---------------- activation stager ----------------
+            // ---------------- activation stager (slot mode) ----------------
+            if (XC) first_ok = false;
             const float *cur = nullptr;
             uint32_t e = 0;
             const uint32_t pre = j2 >= 0 ? 2u : 1u;     // slots filled above
@@ -1104,7 +1216,7 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
                     else
                         consume_packed_mx<MT>(P, jobs, jf, jc, smem, szring, xslots, full,
                                               empty, xfull, xempty, abort_flag, u0, u1, rg,
-                                              lane);
+                                              lane, xring);
                 } else {
                     consume_runtime<MT>(P, jobs, jf, jc, smem, xslots, full, empty, xfull,
                                         xempty, abort_flag, u0, u1, rg, lane);
@@ -1194,6 +1306,34 @@ size_t xslot_bytes_for(const GemvJob *jobs, int count, int M, bool packed) {
     return (xmax + 127) / 128 * 128;
 }
 
+// Chunk mode: packed launches with 5..16 x rows stream x per stage.
+bool chunk_mode(int M, bool packed) { return packed && M > kMaxM && M <= kMaxMChunk; }
+int chunk_mt(int M) { return M <= 8 ? 8 : 16; }
+
+// Workspace layout of the chunk-mode activation digits: each distinct
+// (x, K) of the launch once, in job order; off[i] is job i's offset.  A null
+// x (a size query without pointers) is never shared, which bounds any call.
+size_t xdig_layout(const GemvJob *jobs, int count, int M, std::vector<size_t> *off,
+                   std::vector<int> *first) {
+    const size_t mtb = (size_t)chunk_mt(M) * kXcRowBytes;
+    size_t total = 0;
+    if (off) off->assign(count, 0);
+    if (first) first->clear();
+    for (int i = 0; i < count; ++i) {
+        int prev = -1;
+        for (int q = 0; q < i && prev < 0 && jobs[i].x; ++q)
+            if (jobs[q].x == jobs[i].x && jobs[q].K == jobs[i].K) prev = q;
+        if (prev >= 0) {
+            if (off) (*off)[i] = (*off)[prev];
+            continue;
+        }
+        if (off) (*off)[i] = total;
+        if (first) first->push_back(i);
+        total += (size_t)kchunks_of<true>((int)jobs[i].K) * mtb;
+    }
+    return total;
+}
+
 // Contiguous unit ranges, one per CTA, that minimise the largest range's cost
 // (the classic linear partition: binary search on the bound, greedy fill).
 // A unit costs its weight bytes plus a fixed share for its end-of-unit work,
@@ -1255,14 +1395,26 @@ void partition_units(StreamParams &P, int n, bool packed, int grid) {
 
 bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed,
                            int max_smem) {
-    if (M < 1 || M > kMaxM || count < 1) return false;
+    const bool xc = chunk_mode(M, packed);
+    if (M < 1 || (M > kMaxM && !xc) || count < 1) return false;
     for (int i = 0; i < count; ++i)
         if (jobs[i].N >= (1 << 30) || jobs[i].K >= (1 << 24)) return false;
-    const size_t xs = xslot_bytes_for(jobs, count, M, packed);
+    const size_t xs = xc ? 0 : xslot_bytes_for(jobs, count, M, packed);
     const size_t fixed = 2 * xs + kBarBytes + 1024;
-    const size_t per_stage = kStageBytes + (packed ? kSzBytes : 0);
+    const size_t per_stage = kStageBytes + (packed ? kSzBytes : 0) +
+                             (xc ? (size_t)chunk_mt(M) * kXcRowBytes : 0);
     if (fixed + 2 * per_stage > (size_t)max_smem) return false;
     return tensor_map_encoder() != nullptr;
+}
+
+size_t gemv_stream_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed) {
+    if (!chunk_mode(M, packed)) return 0;
+    // launches above kMaxJobs matrices reuse the space batch by batch
+    size_t worst = 0;
+    for (int b = 0; b < count; b += kMaxJobs)
+        worst = std::max(worst, xdig_layout(jobs + b, std::min(kMaxJobs, count - b), M,
+                                            nullptr, nullptr));
+    return worst ? worst + 256 : 0;
 }
 
 namespace {
@@ -1273,20 +1425,30 @@ struct StreamPlan {
     std::vector<GemvJob> key;
     int M = 0, bits = 0, dev = -1;
     bool packed = false;
+    const void *ws = nullptr;    // chunk mode: the workspace the chunk pointers point into
     StreamParams P;
     int grid = 0, smem = 0;
+    XdigParams X;                // chunk mode: the pre-pass over the distinct x
+    int xgrid = 0;
 };
 constexpr int kPlanCache = 4;
 
 bool same_call(const StreamPlan &p, const GemvJob *jobs, int count, int M, int bits,
-               bool packed, int dev, bool early) {
+               bool packed, int dev, bool early, const void *ws) {
     return p.dev == dev && p.M == M && p.bits == bits && p.packed == packed &&
-           (p.P.early != 0) == early &&
+           (p.P.early != 0) == early && (!chunk_mode(M, packed) || p.ws == ws) &&
            (int)p.key.size() == count &&
            std::memcmp(p.key.data(), jobs, sizeof(GemvJob) * count) == 0;
 }
 
 bc_status launch_plan(const StreamPlan &p, cudaStream_t s) {
+    if (chunk_mode(p.M, p.packed)) {
+        xdig_kernel<<<p.xgrid, 256, 0, s>>>(p.X);
+        const bc_status st = cuda_status();
+        if (st != BC_OK) return st;
+        return chunk_mt(p.M) == 8 ? launch_one<true, 8>(p.P, p.grid, p.smem, s)
+                                  : launch_one<true, 16>(p.P, p.grid, p.smem, s);
+    }
     if (p.packed)
         return p.M <= 1 ? launch_one<true, 1>(p.P, p.grid, p.smem, s)
              : p.M <= 2 ? launch_one<true, 2>(p.P, p.grid, p.smem, s)
@@ -1298,13 +1460,20 @@ bc_status launch_plan(const StreamPlan &p, cudaStream_t s) {
 }  // namespace
 
 bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
-                             bool packed, cudaStream_t s, bool early_start) {
+                             bool packed, cudaStream_t s, bool early_start, void *workspace,
+                             size_t ws_bytes) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BC_ERR_CUDA;
+    const bool xc = chunk_mode(M, packed);
+    if (xc) {
+        const size_t need = gemv_stream_workspace_bytes(jobs, count, M, packed);
+        if (!workspace || ws_bytes < need) return BC_ERR_WORKSPACE;
+    }
     thread_local std::vector<std::unique_ptr<StreamPlan>> plans;
     if (count <= kMaxJobs) {
         for (size_t i = 0; i < plans.size(); ++i) {
-            if (!same_call(*plans[i], jobs, count, M, bits, packed, dev, early_start)) continue;
+            if (!same_call(*plans[i], jobs, count, M, bits, packed, dev, early_start, workspace))
+                continue;
             if (i) std::rotate(plans.begin(), plans.begin() + i, plans.begin() + i + 1);
             return launch_plan(*plans[0], s);
         }
@@ -1328,7 +1497,34 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
             units += (J.N + kRows - 1) / kRows;
             if (!encode_weights(enc, &P.wmap[i], G0.w, J.N, rbytes)) return BC_ERR_CUDA;
         }
-        const size_t xs = xslot_bytes_for(jobs + b0, n, M, packed);
+        P.xchunk_bytes = 0;
+        if (xc) {       // the jobs' x point at their chunks in the workspace
+            const int MT = chunk_mt(M);
+            std::vector<size_t> off;
+            std::vector<int> first;
+            xdig_layout(jobs + b0, n, M, &off, &first);
+            uint8_t *ws = reinterpret_cast<uint8_t *>(
+                (reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255));
+            for (int i = 0; i < n; ++i) P.jobs[i].x = reinterpret_cast<const float *>(ws + off[i]);
+            XdigParams &X = plan->X;
+            int tasks = 0;
+            X.count = (int)first.size();
+            for (int q = 0; q < X.count; ++q) {
+                const GemvJob &G0 = jobs[b0 + first[q]];
+                X.t[q].x = G0.x;
+                X.t[q].out = ws + off[first[q]];
+                X.t[q].K = (int)G0.K;
+                X.t[q].task_begin = tasks;
+                tasks += kchunks_of<true>((int)G0.K) * MT * 2;
+            }
+            X.M = M;
+            X.MT = MT;
+            X.total = tasks;
+            plan->xgrid = std::max(1, std::min((tasks + 7) / 8, 4 * di.sm_count));
+            plan->ws = workspace;
+            P.xchunk_bytes = MT * kXcRowBytes;
+        }
+        const size_t xs = xc ? 0 : xslot_bytes_for(jobs + b0, n, M, packed);
         const int grid = std::max(1, std::min({units, di.sm_count, kMaxCtas}));
         P.total_units = units;
         partition_units(P, n, packed, grid);
@@ -1346,7 +1542,7 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
             P.max_cta_jobs = most;
         }
         const int fixed = (int)(2 * xs) + 256 + P.max_cta_jobs * (int)sizeof(StreamJob) + 1024;
-        const int per_stage = kStageBytes + (packed ? kSzBytes : 0);
+        const int per_stage = kStageBytes + (packed ? kSzBytes : 0) + P.xchunk_bytes;
         int stages = (di.max_smem_optin - fixed) / per_stage;
         stages = std::min(stages, 6);
         if (stages < 2) return BC_ERR_UNSUPPORTED;

@@ -56,14 +56,19 @@ struct GemvJob {             // one matrix of a launch
     int64_t N, K;
     int64_t group;           // 64 or K
 };
-// Streaming GEMV (bc_gemv_stream.cu): M <= 4, bulk-copy ring, mma.sync
-// unpack for packed codes.  Used for launches large enough to fill the GPU.
+// Streaming GEMV (bc_gemv_stream.cu): M <= 4 (M <= 16 for packed codes),
+// bulk-copy ring, int8 tensor-core products.  Used for launches large
+// enough to fill the GPU.
 bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed,
                            int max_smem);
+// Workspace the streaming kernel needs: the activation digits of packed
+// launches with M > 4 (one copy per distinct non-null x; 0 otherwise).
+size_t gemv_stream_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed);
 // early_start: programmatic dependent launch (weights known not to be
 // written by pending work; x / y accesses wait for the previous kernel).
 bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
-                             bool packed, cudaStream_t s, bool early_start);
+                             bool packed, cudaStream_t s, bool early_start, void *workspace,
+                             size_t ws_bytes);
 unsigned gemv_timeouts();
 // Bytes of split-K scratch a launch over these jobs needs.
 size_t gemv_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed,

@@ -211,13 +211,14 @@ def test_determinism_batched(cuda_lib):
         assert torch.equal(o, outs[0])
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 13, 16])
 @pytest.mark.parametrize("mode,bits,group", [("packed", 4, 64), ("runtime", 5, 64),
                                              ("runtime", 3, 0), ("runtime", 16, 64)])
 def test_batched_mixed_shapes_stream(cuda_lib, M, mode, bits, group):
     """A grouped launch large enough for the streaming kernel, with ragged
     row blocks (N not a multiple of 128) and K tails (K not a multiple of
-    the 256-byte stage chunk), several matrices sharing one x."""
+    the 256-byte stage chunk), several matrices sharing one x.  Packed codes
+    at M = 5..16 take the chunked-activation form (rows padded to 8 or 16)."""
     rng = np.random.default_rng(M * 10 + bits)
     shapes = [(37, 192), (200, 896), (896, 1024), (130, 64), (256, 4864),
               (1000, 320)]
@@ -276,7 +277,7 @@ def _stream_set(cuda_lib, M, seed, count=40):
     return items, Ws, x_dev
 
 
-@pytest.mark.parametrize("M", [1, 2])
+@pytest.mark.parametrize("M", [1, 2, 11])
 def test_static_weights_early_start_sees_new_x(cuda_lib, M):
     """BC_FLAG_STATIC_WEIGHTS launches the decode kernel as a programmatic
     dependent launch.  Between back-to-back launches a torch kernel on the
@@ -356,5 +357,38 @@ def test_stream_activation_outliers(cuda_lib):
                               cuda_lib.BC_MODE_PACKED_INT4)
     torch.cuda.synchronize()
     for i, ref in enumerate(refs):
+        assert_close(host(items[i][4]), ref["y"], ref["A"], TOL_FP32, f"matrix {i}")
+    assert cuda_lib.device_timeouts() == 0
+
+
+def test_chunked_activation_workspace(cuda_lib):
+    """Packed launches with M > 4 keep the activation digits in the caller's
+    workspace: a size queried without x pointers covers the call, matrices
+    sharing an x share space, and a short workspace is refused before any
+    work is enqueued."""
+    M = 16
+    items, Ws, x_dev = _stream_set(cuda_lib, M, 94)
+    descs = cuda_lib.make_descs(items)
+    mode = cuda_lib.BC_MODE_PACKED_INT4
+    need = cuda_lib.workspace_size_batched(descs, M, mode, cuda_lib.BC_F32)
+    anon = cuda_lib.make_descs(items)
+    for d in anon:
+        d.x = None
+    bound = cuda_lib.workspace_size_batched(anon, M, mode, cuda_lib.BC_F32)
+    assert 0 < need < bound
+    short = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    st = cuda_lib.lib.bc_matmul_q_batched_ex(descs, len(descs), M, 4, 64, mode,
+                                             cuda_lib.BC_F32, cuda_lib._ptr(short),
+                                             need - 256, 0, None)
+    assert st == cuda_lib.BC_ERR_WORKSPACE
+    xk = {K: wl.activation(70, K, "x", M, K) for K in x_dev}
+    for K, t in x_dev.items():
+        t.copy_(dev(xk[K]))
+    ws = torch.empty(bound, dtype=torch.uint8, device="cuda")
+    cuda_lib.matmul_q_batched(descs, M, 4, 64, mode, workspace=ws)
+    torch.cuda.synchronize()
+    for i in (0, 1, 2, 3, 38, 39):
+        W = Ws[i]
+        ref = oracle.matmul_q(xk[W.shape[1]], W, 4, 64, "packed")
         assert_close(host(items[i][4]), ref["y"], ref["A"], TOL_FP32, f"matrix {i}")
     assert cuda_lib.device_timeouts() == 0
