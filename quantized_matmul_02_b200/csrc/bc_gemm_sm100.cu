@@ -26,6 +26,7 @@
 // wait that runs out records a timeout, the CTA stops, waits (bounded) for
 // its own TMA copies in flight and frees its TMEM.
 #include "bc_internal.cuh"
+#include "bc_tc.cuh"
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -76,9 +77,7 @@ template <int BNX> struct Cfg {
     static constexpr int kBarBytes = 4096;     // barriers + job table copy
     static constexpr int kSmem = kStages * kStageBytes + kBarBytes + 1024;
     // instruction descriptor: D f32, A/B bf16, K-major both, N, M = 128
-    static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                                       ((uint32_t)(BNX >> 3) << 17) |
-                                       ((uint32_t)(kBM >> 4) << 24);
+    static constexpr uint32_t kIdesc = tc::idesc_bf16(kBM, BNX);
 };
 
 // ---- small PTX wrappers ----------------------------------------------------
@@ -130,45 +129,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-// K-major, 128-byte swizzle, 8-row atoms 1024 bytes apart.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
-           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) |
-           ((uint64_t)2 << 61);
-}
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b,
-                                         uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate) : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-        ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-          "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
-          "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
-          "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-          "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]),
-          "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 __device__ __forceinline__ uint32_t lop3_nib(uint32_t w) {
     // ((w & 0x000F000F) | 0x43004300): two bf16 values 128 + nibble
@@ -318,13 +278,11 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kMmaWarp) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(tmem_slot)), "r"(C::kTmemCols) : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        tc::alloc(smem_u32(tmem_slot), C::kTmemCols);
     }
-    tc_fence_before();
+    tc::fence_before();
     __syncthreads();
-    tc_fence_after();
+    tc::fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int K_tiles_dummy = 0;
     (void)K_tiles_dummy;
@@ -370,47 +328,60 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
             }
         }
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
-            uint32_t g = 0;
-            int lt = 0;
-            for (int tile = blockIdx.x; tile < P.total_tiles && !*abort_flag;
-                 tile += gridDim.x, ++lt) {
-                const int j = find_job(sjobs, P.count, tile);
-                const int kblocks = sjobs[j].K / kBK;
-                const int buf = lt & 1;
-                const uint32_t aph = (lt >> 1) & 1;
-                if (!mbar_wait(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + buf * BNX;
-                bool ok = true;
-                for (int kb = 0; kb < kblocks; ++kb, ++g) {
-                    const int s = g % C::kStages;
-                    const uint32_t ph = (g / C::kStages) & 1;
-                    if (!mbar_wait(smem_u32(&full_tma[s]), ph, abort_flag) ||
-                        !mbar_wait(smem_u32(&full_dq[s]), ph, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    uint8_t *st = smem + s * C::kStageBytes;
-                    const uint32_t a0 = smem_u32(st), b0 = smem_u32(st + C::kABytes);
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-                        mma_bf16(d_tmem, sw128_desc(a0 + kk * 32),
-                                 sw128_desc(b0 + kk * 32), C::kIdesc,
-                                 (kb > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(smem_u32(&empty[s]));        // stage reusable
+        // The whole warp walks the tiles and waits; one elected lane issues a
+        // stage's four MMAs and commits.  Descriptors are formed once and
+        // advanced by constant offsets (16-byte units of the start address):
+        // an MMA issued from a lone diverged lane with descriptors rebuilt per
+        // instruction costs several times the tensor core's own time.
+        const uint64_t adesc0 = tc::sw128_desc(smem_u32(smem));
+        const uint64_t bdesc0 = tc::sw128_desc(smem_u32(smem + C::kABytes));
+        uint32_t g = 0;
+        int lt = 0;
+        for (int tile = blockIdx.x;
+             tile < P.total_tiles && !__shfl_sync(0xffffffffu, (int)*abort_flag, 0);
+             tile += gridDim.x, ++lt) {
+            const int j = find_job(sjobs, P.count, tile);
+            const int kblocks = sjobs[j].K / kBK;
+            const int buf = lt & 1;
+            const uint32_t aph = (lt >> 1) & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag)))
+                break;
+            tc::fence_after();
+            const uint32_t d_tmem = tmem_base + buf * BNX;
+            bool ok = true;
+            for (int kb = 0; kb < kblocks; ++kb, ++g) {
+                const int s = g % C::kStages;
+                const uint32_t ph = (g / C::kStages) & 1;
+                bool w = mbar_wait(smem_u32(&full_tma[s]), ph, abort_flag);
+                if (w) w = mbar_wait(smem_u32(&full_dq[s]), ph, abort_flag);
+                if (!__all_sync(0xffffffffu, w)) {
+                    ok = false;
+                    break;
                 }
-                if (!ok) break;
-                mma_commit(smem_u32(&acc_full[buf]));       // tile accumulated
+                tc::fence_after();
+                const uint64_t so = (uint64_t)((s * C::kStageBytes) >> 4);
+                if (tc::elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc::mma_bf16_ss(d_tmem, adesc0 + so + 2 * kk, bdesc0 + so + 2 * kk,
+                                        C::kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    tc::commit(smem_u32(&empty[s]));        // stage reusable
+                }
+                __syncwarp();
             }
-            // every MMA this thread issued has finished before TMEM is freed
-            mma_commit(smem_u32(mma_done));
+            if (!ok) break;
+            if (tc::elect_one()) tc::commit(smem_u32(&acc_full[buf]));   // tile accumulated
+            __syncwarp();
+        }
+        // every MMA issued has finished before TMEM is freed
+        if (tc::elect_one()) tc::commit(smem_u32(mma_done));
+        __syncwarp();
+        if (lane == 0) {
             const long long t0 = clock64();
             while (!mbar_try(smem_u32(mma_done), 0) && clock64() - t0 < kWaitCycles) {
             }
         }
+        __syncwarp();
     } else if (warp < kDqWarp0 + kDqWarps) {
         // dequant: thread -> (row r, half h) of the 128 x 64 weight tile.
         // Scale/zero come from global memory.  They are fetched kLook blocks
@@ -507,13 +478,13 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
             const int buf = lt & 1;
             const uint32_t aph = (lt >> 1) & 1;
             if (!mbar_wait(smem_u32(&acc_full[buf]), aph, abort_flag)) break;
-            tc_fence_after();
+            tc::fence_after();
             const int n = nb * kBM + 32 * q + lane;
             const int m0 = xb * BNX;
 #pragma unroll 1
             for (int c = 0; c < BNX / 32; ++c) {
                 uint32_t v[32];
-                tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + buf * BNX + c * 32, v);
+                tc::ld32(tmem_base + ((uint32_t)(32 * q) << 16) + buf * BNX + c * 32, v);
                 if (n < J.N) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -522,18 +493,17 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
                     }
                 }
             }
-            tc_fence_before();
+            tc::fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&acc_empty[buf]));
         }
     }
 
-    tc_fence_before();
+    tc::fence_before();
     __syncthreads();
     if (warp == kMmaWarp) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
-                     ::"r"(tmem_base), "r"(C::kTmemCols) : "memory");
+        tc::fence_after();
+        tc::dealloc(tmem_base, C::kTmemCols);
     }
 }
 

@@ -50,6 +50,7 @@
 // Every mbarrier wait is bounded; a wait that runs out stops the CTA (its
 // outputs are then incomplete) and is counted for bc_device_timeouts.
 #include "bc_internal.cuh"
+#include "bc_tc.cuh"
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -1004,6 +1005,95 @@ __device__ __forceinline__ void sz_stager(const StreamParams &P, const StreamJob
     }
 }
 
+// Loader warp: the TMA of every stage of the CTA's unit range (the weights
+// of 128 rows x 256 bytes as two 128-byte boxes, and in the chunk modes the
+// stage's activation chunk, `xchunk` bytes from job.x + kc * xchunk into ring
+// slot s at xring + s * xstride), gated by the empty barriers.  It then waits
+// (bounded) for its copies in flight, so none lands after the CTA has exited.
+template <bool PACKED>
+__device__ void load_stages(const StreamParams &P, const StreamJob *jobs, int jf, int jc,
+                            int u0, int u1, uint8_t *smem, uint8_t *xring, int xchunk,
+                            int xstride, uint64_t *full, uint64_t *empty,
+                            volatile int *abort_flag, int lane) {
+    const int S = P.stages;
+    // chunk modes: the x chunks are written by the kernel just before
+    if (xchunk) asm volatile("griddepcontrol.wait;" ::: "memory");
+    const uint64_t policy = evict_first_policy();
+    uint32_t g = 0, armed = 0;
+    int jw = jf;
+    int pidx = 0;
+    uint32_t pph = 0;
+    bool ok = true;
+    for (int u = u0; u < u1 && ok; ++u) {
+        jw = next_job(jobs, jc, jw, u);
+        const int j = jw;
+        const StreamJob &J = jobs[j];
+        const int r0 = (u - J.unit_begin) * kRows;
+        const int rbytes = row_bytes_of<PACKED>(J.K);
+        const int kchunks = kchunks_of<PACKED>(J.K);
+        for (int kc = 0; kc < kchunks; ++kc, ++g) {
+            const int s = pidx;
+            bool got = true;
+            if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), pph ^ 1, abort_flag);
+            got = __shfl_sync(0xffffffffu, got, 0);
+            __syncwarp();
+            if (!got) {
+                ok = false;
+                break;
+            }
+            if (++pidx == S) {
+                pidx = 0;
+                pph ^= 1;
+            }
+            const uint32_t fb = smem_u32(&full[s]);
+            if (lane == 0) {
+                // a window wholly past the row end is not loaded: its codes
+                // meet zero activations (packed) or are skipped (runtime)
+                const int nbox = (rbytes - kc * kChunk) > 128 ? 2 : 1;
+                mbar_expect_tx(fb, (uint32_t)(nbox * kBoxBytes + xchunk));
+                const uint32_t st = smem_u32(smem + s * kStageBytes);
+                for (int b = 0; b < nbox; ++b)
+                    tma_load_2d(st + b * kBoxBytes, &P.wmap[j], kc * kChunk + b * 128, r0, fb,
+                                policy);
+                if (xchunk)      // job.x holds this matrix's x chunks in chunk modes
+                    bulk_load(smem_u32(xring + s * xstride),
+                              reinterpret_cast<const uint8_t *>(J.x) + (int64_t)kc * xchunk,
+                              (uint32_t)xchunk, fb);
+            }
+            armed |= 1u << s;
+            if (PACKED && kc == 0) {
+                // the unit's scales and zeros (one contiguous block each)
+                // go to L2 behind its first weights; the scale/zero
+                // stagers read them a few stages later
+                const int G = J.K >> 6;
+                const int64_t b0 = (int64_t)r0 * G * 2;
+                const int64_t b1 = (int64_t)min(r0 + kRows, J.N) * G * 2;
+                const int lines = (int)((b1 - b0 + 127) >> 7) + 1;
+                const int64_t a0 = b0 & ~(int64_t)127;
+                const char *sb = reinterpret_cast<const char *>(J.s) + a0;
+                const char *zb = reinterpret_cast<const char *>(J.z) + a0;
+                const int64_t limit = (int64_t)J.N * G * 2 - a0;
+                for (int l = lane; l < lines && (int64_t)l * 128 < limit; l += 32) {
+                    prefetch_l2(sb + (int64_t)l * 128);
+                    prefetch_l2(zb + (int64_t)l * 128);
+                }
+            }
+        }
+    }
+    // drain: copies in flight land before the CTA exits
+    if (lane == 0 && g > 0) {
+        for (int q = 0; q < S; ++q) {
+            if (!(armed & (1u << q))) continue;
+            const uint32_t gl = (g - 1) - (((g - 1) % S + S - q) % S);
+            const long long t0 = clock64();
+            while (!mbar_try(smem_u32(&full[q]), (gl / S) & 1) &&
+                   clock64() - t0 < kWaitCycles) {
+            }
+        }
+    }
+    __syncwarp();
+}
+
 template <bool PACKED, int MT>
 __global__ void __launch_bounds__(Roles<PACKED>::threads, 1)
 gemv_stream_kernel(const __grid_constant__ StreamParams P) {
@@ -1064,84 +1154,8 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
 
     if (warp == 0) {
         // ---------------- loader ----------------
-        // chunk mode: the x chunks are written by the kernel just before
-        if (XC) asm volatile("griddepcontrol.wait;" ::: "memory");
-        const uint64_t policy = evict_first_policy();
-        uint32_t g = 0, armed = 0;
-        int jw = jf;
-        int pidx = 0;
-        uint32_t pph = 0;
-        bool ok = true;
-        for (int u = u0; u < u1 && ok; ++u) {
-            jw = next_job(jobs, jc, jw, u);
-            const int j = jw;
-            const StreamJob &J = jobs[j];
-            const int r0 = (u - J.unit_begin) * kRows;
-            const int rbytes = row_bytes_of<PACKED>(J.K);
-            const int kchunks = kchunks_of<PACKED>(J.K);
-            for (int kc = 0; kc < kchunks; ++kc, ++g) {
-                const int s = pidx;
-                bool got = true;
-                if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), pph ^ 1, abort_flag);
-                got = __shfl_sync(0xffffffffu, got, 0);
-                __syncwarp();
-                if (!got) {
-                    ok = false;
-                    break;
-                }
-                if (++pidx == S) {
-                    pidx = 0;
-                    pph ^= 1;
-                }
-                const uint32_t fb = smem_u32(&full[s]);
-                if (lane == 0) {
-                    // a window wholly past the row end is not loaded: its codes
-                    // meet zero activation digits (packed) or are skipped (runtime)
-                    const int nbox = (rbytes - kc * kChunk) > 128 ? 2 : 1;
-                    mbar_expect_tx(fb, (uint32_t)(nbox * kBoxBytes) +
-                                           (XC ? (uint32_t)P.xchunk_bytes : 0u));
-                    const uint32_t st = smem_u32(smem + s * kStageBytes);
-                    for (int b = 0; b < nbox; ++b)
-                        tma_load_2d(st + b * kBoxBytes, &P.wmap[j], kc * kChunk + b * 128, r0, fb,
-                                    policy);
-                    if (XC)      // job.x holds this matrix's x chunks in chunk mode
-                        bulk_load(smem_u32(xring + s * P.xchunk_bytes),
-                                  reinterpret_cast<const uint8_t *>(J.x) +
-                                      (int64_t)kc * P.xchunk_bytes,
-                                  (uint32_t)P.xchunk_bytes, fb);
-                }
-                armed |= 1u << s;
-                if (PACKED && kc == 0) {
-                    // the unit's scales and zeros (one contiguous block each)
-                    // go to L2 behind its first weights; the scale/zero
-                    // stagers read them a few stages later
-                    const int G = J.K >> 6;
-                    const int64_t b0 = (int64_t)r0 * G * 2;
-                    const int64_t b1 = (int64_t)min(r0 + kRows, J.N) * G * 2;
-                    const int lines = (int)((b1 - b0 + 127) >> 7) + 1;
-                    const int64_t a0 = b0 & ~(int64_t)127;
-                    const char *sb = reinterpret_cast<const char *>(J.s) + a0;
-                    const char *zb = reinterpret_cast<const char *>(J.z) + a0;
-                    const int64_t limit = (int64_t)J.N * G * 2 - a0;
-                    for (int l = lane; l < lines && (int64_t)l * 128 < limit; l += 32) {
-                        prefetch_l2(sb + (int64_t)l * 128);
-                        prefetch_l2(zb + (int64_t)l * 128);
-                    }
-                }
-            }
-        }
-        // drain: copies in flight land before the CTA exits
-        if (lane == 0 && g > 0) {
-            for (int q = 0; q < S; ++q) {
-                if (!(armed & (1u << q))) continue;
-                const uint32_t gl = (g - 1) - (((g - 1) % S + S - q) % S);
-                const long long t0 = clock64();
-                while (!mbar_try(smem_u32(&full[q]), (gl / S) & 1) &&
-                       clock64() - t0 < kWaitCycles) {
-                }
-            }
-        }
-        __syncwarp();
+        load_stages<PACKED>(P, jobs, jf, jc, u0, u1, smem, xring, XC ? P.xchunk_bytes : 0,
+                            P.xchunk_bytes, full, empty, abort_flag, lane);
     } else if (warp >= 2 && warp < RL::first_consumer) {
         // ---------------- scale / zero stagers (packed) ----------------
         if constexpr (PACKED) {
@@ -1227,6 +1241,386 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     __syncthreads();
 }
 
+// ---- tensor-core decode (tcgen05), packed codes, 1..16 x rows ---------------------
+// Swap-AB: the unit's 128 weight rows are the MMA's M (TMEM lanes) and the x
+// rows its N = 16.  Per 64-group of K:
+//   * A = 1 + q/16 in bf16 (exact), unpacked by transform warps straight from
+//     the swizzled weight stage into tensor memory (32 columns per group);
+//   * B = x split into two bf16 pieces, hi = bf16(x), lo = bf16(x - hi), so
+//     x~ = hi + lo carries 16 significant bits; a pre-pass writes them per
+//     stage chunk in the MMA's K-major 128-byte-swizzled layout, with
+//     X~ = sum over the group of x~ (fp64 sum, rounded once);
+//   * tcgen05.mma.kind::f16 (A from TMEM, B from smem, fp32 in TMEM) gives
+//     D = sum_k (1 + q_k/16) x~_k, so that
+//         s sum_k (q_k - z) x~_k = 16 s D - s (16 + z) X~,
+//     two FMAs per output and group in the epilogue warps.
+// With 8 x rows or fewer both pieces share one MMA (B rows 0-7 hi, 8-15 lo,
+// added in the epilogue); with 16 the pieces are two MMAs into one D.
+// Products are exact; D carries fp32 accumulation only.  The codes enter A
+// in the order (k_i, k_i+4) per TMEM column of each 8-k block; the pre-pass
+// writes x~ in that same order.
+namespace tcd {
+constexpr int kGroups = 8;                  // 64-groups per stage
+constexpr int kTmemCols = 512;
+constexpr int kAcol = 0;                    // A slots: 8 x 32 columns
+constexpr int kDcol = 256;                  // D slots: 8 x 16 columns
+constexpr int kLoaderWarp = 0, kMmaWarp = 1, kSzWarp0 = 2, kTrWarp0 = 4, kTrWarps = 8;
+constexpr int kEpWarp0 = 12, kEpWarps = 8;
+constexpr int kThreads = 32 * (kEpWarp0 + kEpWarps);
+constexpr uint32_t kIdesc = tc::idesc_bf16(128, 16);
+template <int MT> struct Chunk {
+    static constexpr int kTile = 2048;                     // 16 rows x 128 bytes
+    static constexpr int kTiles = MT == 16 ? 2 * kGroups : kGroups;
+    static constexpr int kTab = kTiles * kTile;            // X~ [group][MT] f32
+    static constexpr int kBytes = kTab + kGroups * MT * 4;
+    static constexpr int kStride = (kBytes + 1023) / 1024 * 1024;   // smem slot
+};
+// B row of x row m, piece p (0 hi, 1 lo) of group gl within a chunk: byte
+// offset of its 128-byte row.
+template <int MT> __host__ __device__ __forceinline__ int brow_off(int gl, int m, int p) {
+    const int tile = MT == 16 ? p * kGroups + gl : gl;
+    const int row = MT == 16 ? m : 8 * p + m;
+    return tile * Chunk<MT>::kTile + (row >> 3) * 1024 + (row & 7) * 128;
+}
+}  // namespace tcd
+
+// Pre-pass: the bf16 pieces of every distinct x of the launch, per stage
+// chunk, into the workspace.  A warp does one (x, chunk, row m, half) task,
+// 4 groups of 64 k, 8 lanes per group, 8 k per lane (one 16-byte piece of
+// a B row).  Rows m >= M and groups past K/64 are zero.
+template <int MT>
+__global__ void __launch_bounds__(256) xpieces_kernel(const __grid_constant__ XdigParams P) {
+    using C = tcd::Chunk<MT>;
+    const int lane = threadIdx.x & 31, j = lane & 7;
+    const int nw = (gridDim.x * blockDim.x) >> 5;
+    for (int task = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; task < P.total; task += nw) {
+        int lo = 0, hi = P.count - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (P.t[mid].task_begin <= task) lo = mid; else hi = mid - 1;
+        }
+        const XdigTask &T = P.t[lo];
+        int r = task - T.task_begin;
+        const int half = r & 1;
+        r >>= 1;
+        const int m = r % MT, kc = r / MT;
+        const int gl = 4 * half + (lane >> 3);
+        const int g = tcd::kGroups * kc + gl;
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+        if (m < P.M && g < (T.K >> 6)) {
+            const float4 *p = reinterpret_cast<const float4 *>(T.x + (int64_t)m * T.K + 64 * g + 8 * j);
+            const float4 a = __ldg(p), b = __ldg(p + 1);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        }
+        uint32_t wh[4], wl[4];
+        double sum = 0.0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(v[i]), h1 = __float2bfloat16_rn(v[i + 4]);
+            const float r0 = v[i] - __bfloat162float(h0), r1 = v[i + 4] - __bfloat162float(h1);
+            const __nv_bfloat16 l0 = __float2bfloat16_rn(r0), l1 = __float2bfloat16_rn(r1);
+            wh[i] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+            wl[i] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+            sum += (double)__bfloat162float(h0) + (double)__bfloat162float(l0);
+            sum += (double)__bfloat162float(h1) + (double)__bfloat162float(l1);
+        }
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+        uint8_t *chunk = T.out + (int64_t)kc * C::kBytes;
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const int row = MT == 16 ? m : 8 * p + m;
+            uint8_t *dst = chunk + tcd::brow_off<MT>(gl, m, p) + ((j ^ (row & 7)) << 4);
+            *reinterpret_cast<uint4 *>(dst) = p ? make_uint4(wl[0], wl[1], wl[2], wl[3])
+                                                : make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        }
+        if (j == 0) reinterpret_cast<float *>(chunk + C::kTab)[gl * MT + m] = (float)sum;
+    }
+}
+
+// (bf16 1 + q/16) pairs for the codes of one 32-bit word (k0..k7, low nibble
+// first): word i holds (k_i, k_i+4).
+__device__ __forceinline__ void unpack_a(uint32_t w, uint32_t *o) {
+    uint32_t t;
+    asm("lop3.b32 %0, %1, 0x00780078, 0x3F803F80, 0xEA;" : "=r"(t) : "r"(w << 3));
+    o[0] = t;
+    asm("lop3.b32 %0, %1, 0x00780078, 0x3F803F80, 0xEA;" : "=r"(t) : "r"(w >> 1));
+    o[1] = t;
+    asm("lop3.b32 %0, %1, 0x00780078, 0x3F803F80, 0xEA;" : "=r"(t) : "r"(w >> 5));
+    o[2] = t;
+    asm("lop3.b32 %0, %1, 0x00780078, 0x3F803F80, 0xEA;" : "=r"(t) : "r"(w >> 9));
+    o[3] = t;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(tcd::kThreads, 1)
+gemv_tc_kernel(const __grid_constant__ StreamParams P) {
+    using C = tcd::Chunk<MT>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int S = P.stages;
+    uint8_t *szring = smem + S * kStageBytes;
+    uint8_t *xring = szring + S * kSzBytes;            // 1024-aligned slots
+    uint64_t *bars = reinterpret_cast<uint64_t *>(xring + S * C::kStride);
+    uint64_t *full = bars, *empty = bars + S;
+    uint64_t *afull = bars + 2 * S;                     // A slot written (4 warps)
+    uint64_t *done = afull + tcd::kGroups;              // MMAs of a group complete
+    uint64_t *dempty = done + tcd::kGroups;             // D slot read (4 warps)
+    uint64_t *mma_final = dempty + tcd::kGroups;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(mma_final + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_final + 1) + 1;
+    StreamJob *jobs_sm = reinterpret_cast<StreamJob *>(mma_final + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u0 = P.cta_begin[blockIdx.x], u1 = P.cta_begin[blockIdx.x + 1];
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int jf = P.cta_job[blockIdx.x];
+    const int jc = min(P.count, P.cta_job[blockIdx.x + 1] + 1);
+    {
+        const uint4 *src = reinterpret_cast<const uint4 *>(&P.jobs[jf]);
+        uint4 *dst = reinterpret_cast<uint4 *>(jobs_sm);
+        const int n16 = (jc - jf) * (int)(sizeof(StreamJob) / 16);
+        for (int i = threadIdx.x; i < n16; i += tcd::kThreads) dst[i] = src[i];
+    }
+    const StreamJob *jobs = jobs_sm - jf;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(smem_u32(&full[s]), 1 + 2);       // loader + two scale/zero stagers
+            mbar_init(smem_u32(&empty[s]), tcd::kTrWarps + tcd::kEpWarps + 1);
+        }
+        for (int b = 0; b < tcd::kGroups; ++b) {
+            mbar_init(smem_u32(&afull[b]), 4);
+            mbar_init(smem_u32(&done[b]), 1);
+            mbar_init(smem_u32(&dempty[b]), tcd::kEpWarps);
+        }
+        mbar_init(smem_u32(mma_final), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == tcd::kMmaWarp) tc::alloc(smem_u32(tmem_slot), tcd::kTmemCols);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (u0 < u1) {
+        if (warp == tcd::kLoaderWarp) {
+            load_stages<true>(P, jobs, jf, jc, u0, u1, smem, xring, C::kBytes, C::kStride, full,
+                              empty, abort_flag, lane);
+        } else if (warp == tcd::kMmaWarp) {
+            // The whole warp walks the stages and waits; one elected lane issues
+            // each group's MMAs.  Descriptors are formed once and advanced by
+            // constant offsets (16-byte units in the start-address field).
+            const uint64_t bdesc0 = tc::sw128_desc(smem_u32(xring));
+            uint32_t g = 0;
+            int j = jf;
+            bool ok = true;
+            for (int u = u0; u < u1 && ok; ++u) {
+                j = next_job(jobs, jc, j, u);
+                const int kch = kchunks_of<true>(jobs[j].K);
+                for (int kc = 0; kc < kch; ++kc, ++g) {
+                    const int s = (int)(g % (uint32_t)S);
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait(smem_u32(&full[s]), (g / S) & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    const uint64_t bs = bdesc0 + (uint64_t)((s * C::kStride) >> 4);
+#pragma unroll 1
+                    for (int gl = 0; gl < tcd::kGroups; ++gl) {
+                        bool w = mbar_wait(smem_u32(&afull[gl]), g & 1, abort_flag);
+                        if (w && g > 0) w = mbar_wait(smem_u32(&dempty[gl]), (g - 1) & 1, abort_flag);
+                        if (!__all_sync(0xffffffffu, w)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after();
+                        if (tc::elect_one()) {
+                            const uint32_t d = tmem + tcd::kDcol + 16 * gl;
+                            const uint32_t a = tmem + tcd::kAcol + 32 * gl;
+#pragma unroll
+                            for (int p = 0; p < (MT == 16 ? 2 : 1); ++p) {
+                                const uint64_t bd = bs + (uint64_t)(tcd::brow_off<MT>(gl, 0, p) >> 4);
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    tc::mma_bf16_ts(d, a + 8 * kk, bd + 2 * kk, tcd::kIdesc,
+                                                    (p | kk) ? 1u : 0u);
+                            }
+                            tc::commit(smem_u32(&done[gl]));
+                        }
+                        __syncwarp();
+                    }
+                    if (!ok) break;
+                    if (tc::elect_one()) tc::commit(smem_u32(&empty[s]));     // x chunk read
+                    __syncwarp();
+                }
+            }
+            // every MMA issued has completed before TMEM is freed
+            if (tc::elect_one()) tc::commit(smem_u32(mma_final));
+            __syncwarp();
+            if (lane == 0) {
+                const long long t0 = clock64();
+                while (!mbar_try(smem_u32(mma_final), 0) && clock64() - t0 < kWaitCycles) {
+                }
+            }
+            __syncwarp();
+        } else if (warp < tcd::kTrWarp0) {
+            sz_stager(P, jobs, jf, jc, szring, full, empty, abort_flag, u0, u1,
+                      warp - tcd::kSzWarp0, lane);
+        } else if (warp < tcd::kEpWarp0) {
+            // ---- transform: codes -> A = 1 + q/16 (bf16) in TMEM ----
+            // Warp (quarter q = warp & 3, parity par) writes lanes 32q..32q+31
+            // (its rows) of the A slots of groups par, par + 2, ... of a stage.
+            const int q = warp & 3, par = (warp - tcd::kTrWarp0) >> 2;
+            const int r = 32 * q + lane;
+            const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + tcd::kAcol;
+            uint32_t g = 0;
+            int j = jf;
+            bool ok = true;
+            for (int u = u0; u < u1 && ok; ++u) {
+                j = next_job(jobs, jc, j, u);
+                const int kch = kchunks_of<true>(jobs[j].K);
+                for (int kc = 0; kc < kch; ++kc, ++g) {
+                    const int s = (int)(g % (uint32_t)S);
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait(smem_u32(&full[s]), (g / S) & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t *st = smem + s * kStageBytes;
+#pragma unroll 1
+                    for (int t = 0; t < tcd::kGroups / 2; ++t) {
+                        const int gl = 2 * t + par;
+                        // the A slot is free once the previous stage's MMAs on it are done
+                        if (g > 0 &&
+                            !__all_sync(0xffffffffu, mbar_wait(smem_u32(&done[gl]), (g - 1) & 1,
+                                                               abort_flag))) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after();
+                        const uint8_t *box = st + (gl >> 2) * kBoxBytes + r * 128;
+                        const int c0 = 2 * (gl & 3);
+                        const uint4 v0 = *reinterpret_cast<const uint4 *>(box + ((c0 ^ (r & 7)) << 4));
+                        const uint4 v1 =
+                            *reinterpret_cast<const uint4 *>(box + (((c0 + 1) ^ (r & 7)) << 4));
+                        uint32_t o[32];
+                        unpack_a(v0.x, o + 0);
+                        unpack_a(v0.y, o + 4);
+                        unpack_a(v0.z, o + 8);
+                        unpack_a(v0.w, o + 12);
+                        unpack_a(v1.x, o + 16);
+                        unpack_a(v1.y, o + 20);
+                        unpack_a(v1.z, o + 24);
+                        unpack_a(v1.w, o + 28);
+                        tc::st32(lane_base + 32 * gl, o);
+                        tc::fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&afull[gl]));
+                    }
+                    if (!ok) break;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&empty[s]));   // codes read
+                }
+            }
+        } else {
+            // ---- epilogue: y[m][row] += 16 s D - s (16 + z) X~ ----
+            // Warp (quarter q, half h) takes x rows h*MT/2 .. of its 32 weight
+            // rows, over every group.
+            constexpr int MH = MT / 2;
+            const int q = warp & 3, h = (warp - tcd::kEpWarp0) >> 2, m0 = h * MH;
+            const int r = 32 * q + lane;
+            const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + tcd::kDcol;
+            float y[MH];
+#pragma unroll
+            for (int m = 0; m < MH; ++m) y[m] = 0.0f;
+            uint32_t g = 0;
+            int j = jf;
+            bool ok = true;
+            for (int u = u0; u < u1 && ok; ++u) {
+                j = next_job(jobs, jc, j, u);
+                const StreamJob &J = jobs[j];
+                const int kch = kchunks_of<true>(J.K);
+                for (int kc = 0; kc < kch; ++kc, ++g) {
+                    const int s = (int)(g % (uint32_t)S);
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait(smem_u32(&full[s]), (g / S) & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    const uint4 sv = *reinterpret_cast<const uint4 *>(szring + s * kSzBytes + r * 16);
+                    const uint4 zv = *reinterpret_cast<const uint4 *>(
+                        szring + s * kSzBytes + kSzBytes / 2 + r * 16);
+                    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+                    const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
+                    const float *tab =
+                        reinterpret_cast<const float *>(xring + s * C::kStride + C::kTab) + m0;
+#pragma unroll
+                    for (int gl = 0; gl < tcd::kGroups; ++gl) {
+                        if (!__all_sync(0xffffffffu,
+                                        mbar_wait(smem_u32(&done[gl]), g & 1, abort_flag))) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after();
+                        float D[MH];
+                        if constexpr (MT == 16) {
+                            uint32_t d[8];
+                            tc::ld8(lane_base + 16 * gl + m0, d);
+#pragma unroll
+                            for (int i = 0; i < MH; ++i) D[i] = __uint_as_float(d[i]);
+                        } else {
+                            uint32_t d[16];
+                            tc::ld16(lane_base + 16 * gl, d);
+#pragma unroll
+                            for (int i = 0; i < MH; ++i)
+                                D[i] = __uint_as_float(d[m0 + i]) + __uint_as_float(d[8 + m0 + i]);
+                        }
+                        tc::fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&dempty[gl]));
+                        const float2 s2 = half2_bits_to_float2(sw[gl >> 1]);
+                        const float2 z2 = half2_bits_to_float2(zw[gl >> 1]);
+                        const float sc = (gl & 1) ? s2.y : s2.x, zc = (gl & 1) ? z2.y : z2.x;
+                        const float s16 = 16.0f * sc, szc = -sc * (16.0f + zc);
+                        const float4 *t4 = reinterpret_cast<const float4 *>(tab + gl * MT);
+#pragma unroll
+                        for (int m4 = 0; m4 < MH / 4; ++m4) {
+                            const float4 X = t4[m4];
+                            const float Xm[4] = {X.x, X.y, X.z, X.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                y[4 * m4 + i] = fmaf(s16, D[4 * m4 + i], fmaf(szc, Xm[i], y[4 * m4 + i]));
+                        }
+                    }
+                    if (!ok) break;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&empty[s]));   // scales, X~ read
+                    if (kc + 1 == kch) {
+                        const int n = (u - J.unit_begin) * kRows + r;
+#pragma unroll
+                        for (int i = 0; i < MH; ++i) {
+                            if (m0 + i < P.M && n < J.N) J.y[(int64_t)(m0 + i) * J.N + n] = y[i];
+                            y[i] = 0.0f;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    tc::fence_before();
+    __syncthreads();
+    if (warp == tcd::kMmaWarp) {
+        tc::fence_after();
+        tc::dealloc(tmem, tcd::kTmemCols);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -1260,6 +1654,39 @@ bc_status launch_one(const StreamParams &P, int grid, int smem, cudaStream_t s) 
     cfg.attrs = attr;
     cfg.numAttrs = P.early ? 1 : 0;
     if (cudaLaunchKernelEx(&cfg, gemv_stream_kernel<PACKED, MT>, P) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BC_ERR_CUDA;
+    }
+    return cuda_status();
+}
+
+template <int MT>
+bc_status launch_tc(const StreamParams &P, int grid, int smem, cudaStream_t s) {
+    static std::mutex mu;
+    static int attr_smem[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return BC_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (smem > attr_smem[dev]) {
+            if (cudaFuncSetAttribute(gemv_tc_kernel<MT>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem) != cudaSuccess)
+                return BC_ERR_CUDA;
+            attr_smem[dev] = smem;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(tcd::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = P.early ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, gemv_tc_kernel<MT>, P) != cudaSuccess) {
         (void)cudaGetLastError();
         return BC_ERR_CUDA;
     }
@@ -1306,16 +1733,23 @@ size_t xslot_bytes_for(const GemvJob *jobs, int count, int M, bool packed) {
     return (xmax + 127) / 128 * 128;
 }
 
-// Chunk mode: packed launches with 5..16 x rows stream x per stage.
+// Chunk mode: packed launches with 5..16 x rows run the tensor-core decode
+// kernel, which streams x per stage from the workspace.
 bool chunk_mode(int M, bool packed) { return packed && M > kMaxM && M <= kMaxMChunk; }
 int chunk_mt(int M) { return M <= 8 ? 8 : 16; }
+size_t chunk_bytes(int M) {
+    return chunk_mt(M) == 8 ? tcd::Chunk<8>::kBytes : tcd::Chunk<16>::kBytes;
+}
+size_t chunk_stride(int M) {
+    return chunk_mt(M) == 8 ? tcd::Chunk<8>::kStride : tcd::Chunk<16>::kStride;
+}
 
 // Workspace layout of the chunk-mode activation digits: each distinct
 // (x, K) of the launch once, in job order; off[i] is job i's offset.  A null
 // x (a size query without pointers) is never shared, which bounds any call.
 size_t xdig_layout(const GemvJob *jobs, int count, int M, std::vector<size_t> *off,
                    std::vector<int> *first) {
-    const size_t mtb = (size_t)chunk_mt(M) * kXcRowBytes;
+    const size_t mtb = chunk_bytes(M);
     size_t total = 0;
     if (off) off->assign(count, 0);
     if (first) first->clear();
@@ -1402,7 +1836,7 @@ bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed,
     const size_t xs = xc ? 0 : xslot_bytes_for(jobs, count, M, packed);
     const size_t fixed = 2 * xs + kBarBytes + 1024;
     const size_t per_stage = kStageBytes + (packed ? kSzBytes : 0) +
-                             (xc ? (size_t)chunk_mt(M) * kXcRowBytes : 0);
+                             (xc ? chunk_stride(M) : 0);
     if (fixed + 2 * per_stage > (size_t)max_smem) return false;
     return tensor_map_encoder() != nullptr;
 }
@@ -1443,11 +1877,14 @@ bool same_call(const StreamPlan &p, const GemvJob *jobs, int count, int M, int b
 
 bc_status launch_plan(const StreamPlan &p, cudaStream_t s) {
     if (chunk_mode(p.M, p.packed)) {
-        xdig_kernel<<<p.xgrid, 256, 0, s>>>(p.X);
+        if (chunk_mt(p.M) == 8)
+            xpieces_kernel<8><<<p.xgrid, 256, 0, s>>>(p.X);
+        else
+            xpieces_kernel<16><<<p.xgrid, 256, 0, s>>>(p.X);
         const bc_status st = cuda_status();
         if (st != BC_OK) return st;
-        return chunk_mt(p.M) == 8 ? launch_one<true, 8>(p.P, p.grid, p.smem, s)
-                                  : launch_one<true, 16>(p.P, p.grid, p.smem, s);
+        return chunk_mt(p.M) == 8 ? launch_tc<8>(p.P, p.grid, p.smem, s)
+                                  : launch_tc<16>(p.P, p.grid, p.smem, s);
     }
     if (p.packed)
         return p.M <= 1 ? launch_one<true, 1>(p.P, p.grid, p.smem, s)
@@ -1522,7 +1959,7 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
             X.total = tasks;
             plan->xgrid = std::max(1, std::min((tasks + 7) / 8, 4 * di.sm_count));
             plan->ws = workspace;
-            P.xchunk_bytes = MT * kXcRowBytes;
+            P.xchunk_bytes = (int)chunk_bytes(M);
         }
         const size_t xs = xc ? 0 : xslot_bytes_for(jobs + b0, n, M, packed);
         const int grid = std::max(1, std::min({units, di.sm_count, kMaxCtas}));
@@ -1541,8 +1978,10 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
             }
             P.max_cta_jobs = most;
         }
-        const int fixed = (int)(2 * xs) + 256 + P.max_cta_jobs * (int)sizeof(StreamJob) + 1024;
-        const int per_stage = kStageBytes + (packed ? kSzBytes : 0) + P.xchunk_bytes;
+        const int fixed = (int)(2 * xs) + (xc ? 512 : 256) +
+                          P.max_cta_jobs * (int)sizeof(StreamJob) + 1024;
+        const int per_stage = kStageBytes + (packed ? kSzBytes : 0) +
+                              (xc ? (int)chunk_stride(M) : 0);
         int stages = (di.max_smem_optin - fixed) / per_stage;
         stages = std::min(stages, 6);
         if (stages < 2) return BC_ERR_UNSUPPORTED;
