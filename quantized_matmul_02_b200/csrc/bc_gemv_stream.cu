@@ -1254,33 +1254,36 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
 //     D = sum_k (1 + q_k/16) x~_k, so that
 //         s sum_k (q_k - z) x~_k = 16 s D - s (16 + z) X~,
 //     two FMAs per output and group in the epilogue warps.
-// With 8 x rows or fewer both pieces share one MMA (B rows 0-7 hi, 8-15 lo,
-// added in the epilogue); with 16 the pieces are two MMAs into one D.
-// Products are exact; D carries fp32 accumulation only.  The codes enter A
-// in the order (k_i, k_i+4) per TMEM column of each 8-k block; the pre-pass
-// writes x~ in that same order.
+// Both pieces share one MMA: B rows 0..MT-1 hold hi, MT..2MT-1 lo (N = 2 MT),
+// added in the epilogue.  Products are exact; D carries fp32 accumulation
+// only.  The codes enter A in the order (k_i, k_i+4) per TMEM column of each
+// 8-k block; the pre-pass writes x~ in that same order.
+//
+// Tensor memory holds two half-stage sets (4 groups each) of A (4 x 32
+// columns) and of D (4 x 2 MT columns), so the transform, the MMAs and the
+// epilogue work on different half-stages; within a half-stage the MMAs of
+// the four groups are interleaved, so one group's dependent accumulation
+// hides behind the others.
 namespace tcd {
 constexpr int kGroups = 8;                  // 64-groups per stage
+constexpr int kHalf = 4;                    // groups per half-stage
 constexpr int kTmemCols = 512;
-constexpr int kAcol = 0;                    // A slots: 8 x 32 columns
-constexpr int kDcol = 256;                  // D slots: 8 x 16 columns
+constexpr int kAcol = 0;                    // A: 2 sets x 4 groups x 32 columns
+constexpr int kDcol = 256;                  // D: 2 sets x 4 groups x 2 MT columns
 constexpr int kLoaderWarp = 0, kMmaWarp = 1, kSzWarp0 = 2, kTrWarp0 = 4, kTrWarps = 8;
 constexpr int kEpWarp0 = 12, kEpWarps = 8;
 constexpr int kThreads = 32 * (kEpWarp0 + kEpWarps);
-constexpr uint32_t kIdesc = tc::idesc_bf16(128, 16);
 template <int MT> struct Chunk {
-    static constexpr int kTile = 2048;                     // 16 rows x 128 bytes
-    static constexpr int kTiles = MT == 16 ? 2 * kGroups : kGroups;
-    static constexpr int kTab = kTiles * kTile;            // X~ [group][MT] f32
+    static constexpr int kTile = 2 * MT * 128;             // 2 MT rows x 128 bytes
+    static constexpr int kTab = kGroups * kTile;           // X~ [group][MT] f32
     static constexpr int kBytes = kTab + kGroups * MT * 4;
     static constexpr int kStride = (kBytes + 1023) / 1024 * 1024;   // smem slot
 };
 // B row of x row m, piece p (0 hi, 1 lo) of group gl within a chunk: byte
 // offset of its 128-byte row.
 template <int MT> __host__ __device__ __forceinline__ int brow_off(int gl, int m, int p) {
-    const int tile = MT == 16 ? p * kGroups + gl : gl;
-    const int row = MT == 16 ? m : 8 * p + m;
-    return tile * Chunk<MT>::kTile + (row >> 3) * 1024 + (row & 7) * 128;
+    const int row = p * MT + m;
+    return gl * Chunk<MT>::kTile + (row >> 3) * 1024 + (row & 7) * 128;
 }
 }  // namespace tcd
 
@@ -1333,7 +1336,7 @@ __global__ void __launch_bounds__(256) xpieces_kernel(const __grid_constant__ Xd
         uint8_t *chunk = T.out + (int64_t)kc * C::kBytes;
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
-            const int row = MT == 16 ? m : 8 * p + m;
+            const int row = p * MT + m;
             uint8_t *dst = chunk + tcd::brow_off<MT>(gl, m, p) + ((j ^ (row & 7)) << 4);
             *reinterpret_cast<uint4 *>(dst) = p ? make_uint4(wl[0], wl[1], wl[2], wl[3])
                                                 : make_uint4(wh[0], wh[1], wh[2], wh[3]);
@@ -1360,6 +1363,9 @@ template <int MT>
 __global__ void __launch_bounds__(tcd::kThreads, 1)
 gemv_tc_kernel(const __grid_constant__ StreamParams P) {
     using C = tcd::Chunk<MT>;
+    constexpr int NB = 2 * MT;                       // MMA N: hi and lo rows of B
+    constexpr int MH = MT / 2;                       // x rows per epilogue warp
+    constexpr uint32_t kIdesc = tc::idesc_bf16(128, NB);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -1368,13 +1374,13 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
     uint8_t *xring = szring + S * kSzBytes;            // 1024-aligned slots
     uint64_t *bars = reinterpret_cast<uint64_t *>(xring + S * C::kStride);
     uint64_t *full = bars, *empty = bars + S;
-    uint64_t *afull = bars + 2 * S;                     // A slot written (4 warps)
-    uint64_t *done = afull + tcd::kGroups;              // MMAs of a group complete
-    uint64_t *dempty = done + tcd::kGroups;             // D slot read (4 warps)
-    uint64_t *mma_final = dempty + tcd::kGroups;
+    uint64_t *afull = bars + 2 * S;                     // A set written (8 warps)
+    uint64_t *done = afull + 2;                         // MMAs of a half-stage complete
+    uint64_t *dempty = done + 2;                        // D set read (8 warps)
+    uint64_t *mma_final = dempty + 2;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(mma_final + 1);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_final + 1) + 1;
-    StreamJob *jobs_sm = reinterpret_cast<StreamJob *>(mma_final + 2);
+    StreamJob *jobs_sm = reinterpret_cast<StreamJob *>(bars + 2 * S + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u0 = P.cta_begin[blockIdx.x], u1 = P.cta_begin[blockIdx.x + 1];
@@ -1393,8 +1399,8 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
             mbar_init(smem_u32(&full[s]), 1 + 2);       // loader + two scale/zero stagers
             mbar_init(smem_u32(&empty[s]), tcd::kTrWarps + tcd::kEpWarps + 1);
         }
-        for (int b = 0; b < tcd::kGroups; ++b) {
-            mbar_init(smem_u32(&afull[b]), 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&afull[b]), tcd::kTrWarps);
             mbar_init(smem_u32(&done[b]), 1);
             mbar_init(smem_u32(&dempty[b]), tcd::kEpWarps);
         }
@@ -1407,6 +1413,10 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = *tmem_slot;
+    // warp-uniform bounded wait
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, abort_flag));
+    };
 
     if (u0 < u1) {
         if (warp == tcd::kLoaderWarp) {
@@ -1414,8 +1424,9 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
                               empty, abort_flag, lane);
         } else if (warp == tcd::kMmaWarp) {
             // The whole warp walks the stages and waits; one elected lane issues
-            // each group's MMAs.  Descriptors are formed once and advanced by
-            // constant offsets (16-byte units in the start-address field).
+            // a half-stage's MMAs, interleaved over its four groups.
+            // Descriptors are formed once and advanced by constant offsets
+            // (16-byte units of the start address).
             const uint64_t bdesc0 = tc::sw128_desc(smem_u32(xring));
             uint32_t g = 0;
             int j = jf;
@@ -1423,41 +1434,38 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
             for (int u = u0; u < u1 && ok; ++u) {
                 j = next_job(jobs, jc, j, u);
                 const int kch = kchunks_of<true>(jobs[j].K);
-                for (int kc = 0; kc < kch; ++kc, ++g) {
+                for (int kc = 0; kc < kch && ok; ++kc, ++g) {
                     const int s = (int)(g % (uint32_t)S);
-                    if (!__all_sync(0xffffffffu,
-                                    mbar_wait(smem_u32(&full[s]), (g / S) & 1, abort_flag))) {
+                    if (!wait_all(&full[s], (g / S) & 1)) {
                         ok = false;
                         break;
                     }
                     const uint64_t bs = bdesc0 + (uint64_t)((s * C::kStride) >> 4);
-#pragma unroll 1
-                    for (int gl = 0; gl < tcd::kGroups; ++gl) {
-                        bool w = mbar_wait(smem_u32(&afull[gl]), g & 1, abort_flag);
-                        if (w && g > 0) w = mbar_wait(smem_u32(&dempty[gl]), (g - 1) & 1, abort_flag);
+#pragma unroll
+                    for (int hs = 0; hs < 2; ++hs) {
+                        bool w = mbar_wait(smem_u32(&afull[hs]), g & 1, abort_flag);
+                        if (w && g > 0) w = mbar_wait(smem_u32(&dempty[hs]), (g - 1) & 1, abort_flag);
                         if (!__all_sync(0xffffffffu, w)) {
                             ok = false;
                             break;
                         }
                         tc::fence_after();
                         if (tc::elect_one()) {
-                            const uint32_t d = tmem + tcd::kDcol + 16 * gl;
-                            const uint32_t a = tmem + tcd::kAcol + 32 * gl;
+                            const uint32_t d0 = tmem + tcd::kDcol + hs * tcd::kHalf * NB;
+                            const uint32_t a0 = tmem + tcd::kAcol + hs * tcd::kHalf * 32;
+                            const uint64_t b0 = bs + (uint64_t)((hs * tcd::kHalf * C::kTile) >> 4);
 #pragma unroll
-                            for (int p = 0; p < (MT == 16 ? 2 : 1); ++p) {
-                                const uint64_t bd = bs + (uint64_t)(tcd::brow_off<MT>(gl, 0, p) >> 4);
+                            for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    tc::mma_bf16_ts(d, a + 8 * kk, bd + 2 * kk, tcd::kIdesc,
-                                                    (p | kk) ? 1u : 0u);
-                            }
-                            tc::commit(smem_u32(&done[gl]));
+                                for (int gi = 0; gi < tcd::kHalf; ++gi)
+                                    tc::mma_bf16_ts(d0 + gi * NB, a0 + gi * 32 + 8 * kk,
+                                                    b0 + (uint64_t)((gi * C::kTile) >> 4) + 2 * kk,
+                                                    kIdesc, kk ? 1u : 0u);
+                            tc::commit(smem_u32(&done[hs]));
+                            if (hs == 1) tc::commit(smem_u32(&empty[s]));    // x chunk read
                         }
                         __syncwarp();
                     }
-                    if (!ok) break;
-                    if (tc::elect_one()) tc::commit(smem_u32(&empty[s]));     // x chunk read
-                    __syncwarp();
                 }
             }
             // every MMA issued has completed before TMEM is freed
@@ -1475,7 +1483,7 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
         } else if (warp < tcd::kEpWarp0) {
             // ---- transform: codes -> A = 1 + q/16 (bf16) in TMEM ----
             // Warp (quarter q = warp & 3, parity par) writes lanes 32q..32q+31
-            // (its rows) of the A slots of groups par, par + 2, ... of a stage.
+            // (its rows) for groups par and par + 2 of each half-stage.
             const int q = warp & 3, par = (warp - tcd::kTrWarp0) >> 2;
             const int r = 32 * q + lane;
             const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + tcd::kAcol;
@@ -1485,43 +1493,44 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
             for (int u = u0; u < u1 && ok; ++u) {
                 j = next_job(jobs, jc, j, u);
                 const int kch = kchunks_of<true>(jobs[j].K);
-                for (int kc = 0; kc < kch; ++kc, ++g) {
+                for (int kc = 0; kc < kch && ok; ++kc, ++g) {
                     const int s = (int)(g % (uint32_t)S);
-                    if (!__all_sync(0xffffffffu,
-                                    mbar_wait(smem_u32(&full[s]), (g / S) & 1, abort_flag))) {
+                    if (!wait_all(&full[s], (g / S) & 1)) {
                         ok = false;
                         break;
                     }
                     const uint8_t *st = smem + s * kStageBytes;
-#pragma unroll 1
-                    for (int t = 0; t < tcd::kGroups / 2; ++t) {
-                        const int gl = 2 * t + par;
-                        // the A slot is free once the previous stage's MMAs on it are done
-                        if (g > 0 &&
-                            !__all_sync(0xffffffffu, mbar_wait(smem_u32(&done[gl]), (g - 1) & 1,
-                                                               abort_flag))) {
+#pragma unroll
+                    for (int hs = 0; hs < 2; ++hs) {
+                        // the A set is free once the previous stage's MMAs on it are done
+                        if (g > 0 && !wait_all(&done[hs], (g - 1) & 1)) {
                             ok = false;
                             break;
                         }
                         tc::fence_after();
-                        const uint8_t *box = st + (gl >> 2) * kBoxBytes + r * 128;
-                        const int c0 = 2 * (gl & 3);
-                        const uint4 v0 = *reinterpret_cast<const uint4 *>(box + ((c0 ^ (r & 7)) << 4));
-                        const uint4 v1 =
-                            *reinterpret_cast<const uint4 *>(box + (((c0 + 1) ^ (r & 7)) << 4));
-                        uint32_t o[32];
-                        unpack_a(v0.x, o + 0);
-                        unpack_a(v0.y, o + 4);
-                        unpack_a(v0.z, o + 8);
-                        unpack_a(v0.w, o + 12);
-                        unpack_a(v1.x, o + 16);
-                        unpack_a(v1.y, o + 20);
-                        unpack_a(v1.z, o + 24);
-                        unpack_a(v1.w, o + 28);
-                        tc::st32(lane_base + 32 * gl, o);
+                        const uint8_t *box = st + hs * kBoxBytes + r * 128;
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const int gi = 2 * i + par;          // group within the half
+                            const uint4 v0 =
+                                *reinterpret_cast<const uint4 *>(box + (((2 * gi) ^ (r & 7)) << 4));
+                            const uint4 v1 =
+                                *reinterpret_cast<const uint4 *>(box + (((2 * gi + 1) ^ (r & 7)) << 4));
+                            uint32_t o[32];
+                            unpack_a(v0.x, o + 0);
+                            unpack_a(v0.y, o + 4);
+                            unpack_a(v0.z, o + 8);
+                            unpack_a(v0.w, o + 12);
+                            unpack_a(v1.x, o + 16);
+                            unpack_a(v1.y, o + 20);
+                            unpack_a(v1.z, o + 24);
+                            unpack_a(v1.w, o + 28);
+                            tc::st32_nw(lane_base + hs * tcd::kHalf * 32 + gi * 32, o);
+                        }
+                        tc::wait_st();
                         tc::fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(smem_u32(&afull[gl]));
+                        if (lane == 0) mbar_arrive(smem_u32(&afull[hs]));
                     }
                     if (!ok) break;
                     __syncwarp();
@@ -1529,16 +1538,15 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
                 }
             }
         } else {
-            // ---- epilogue: y[m][row] += 16 s D - s (16 + z) X~ ----
+            // ---- epilogue: y[m][row] += 16 s (D_hi + D_lo) - s (16 + z) X~ ----
             // Warp (quarter q, half h) takes x rows h*MT/2 .. of its 32 weight
             // rows, over every group.
-            constexpr int MH = MT / 2;
             const int q = warp & 3, h = (warp - tcd::kEpWarp0) >> 2, m0 = h * MH;
             const int r = 32 * q + lane;
             const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + tcd::kDcol;
             float y[MH];
 #pragma unroll
-            for (int m = 0; m < MH; ++m) y[m] = 0.0f;
+            for (int i = 0; i < MH; ++i) y[i] = 0.0f;
             uint32_t g = 0;
             int j = jf;
             bool ok = true;
@@ -1546,10 +1554,9 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
                 j = next_job(jobs, jc, j, u);
                 const StreamJob &J = jobs[j];
                 const int kch = kchunks_of<true>(J.K);
-                for (int kc = 0; kc < kch; ++kc, ++g) {
+                for (int kc = 0; kc < kch && ok; ++kc, ++g) {
                     const int s = (int)(g % (uint32_t)S);
-                    if (!__all_sync(0xffffffffu,
-                                    mbar_wait(smem_u32(&full[s]), (g / S) & 1, abort_flag))) {
+                    if (!wait_all(&full[s], (g / S) & 1)) {
                         ok = false;
                         break;
                     }
@@ -1561,41 +1568,60 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
                     const float *tab =
                         reinterpret_cast<const float *>(xring + s * C::kStride + C::kTab) + m0;
 #pragma unroll
-                    for (int gl = 0; gl < tcd::kGroups; ++gl) {
-                        if (!__all_sync(0xffffffffu,
-                                        mbar_wait(smem_u32(&done[gl]), g & 1, abort_flag))) {
+                    for (int hs = 0; hs < 2; ++hs) {
+                        if (!wait_all(&done[hs], g & 1)) {
                             ok = false;
                             break;
                         }
                         tc::fence_after();
-                        float D[MH];
-                        if constexpr (MT == 16) {
-                            uint32_t d[8];
-                            tc::ld8(lane_base + 16 * gl + m0, d);
 #pragma unroll
-                            for (int i = 0; i < MH; ++i) D[i] = __uint_as_float(d[i]);
-                        } else {
-                            uint32_t d[16];
-                            tc::ld16(lane_base + 16 * gl, d);
+                        for (int pr = 0; pr < 2; ++pr) {
+                            float D[2][MH];
 #pragma unroll
-                            for (int i = 0; i < MH; ++i)
-                                D[i] = __uint_as_float(d[m0 + i]) + __uint_as_float(d[8 + m0 + i]);
-                        }
-                        tc::fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(smem_u32(&dempty[gl]));
-                        const float2 s2 = half2_bits_to_float2(sw[gl >> 1]);
-                        const float2 z2 = half2_bits_to_float2(zw[gl >> 1]);
-                        const float sc = (gl & 1) ? s2.y : s2.x, zc = (gl & 1) ? z2.y : z2.x;
-                        const float s16 = 16.0f * sc, szc = -sc * (16.0f + zc);
-                        const float4 *t4 = reinterpret_cast<const float4 *>(tab + gl * MT);
+                            for (int e = 0; e < 2; ++e) {
+                                const uint32_t col =
+                                    lane_base + (hs * tcd::kHalf + 2 * pr + e) * NB + m0;
+                                if constexpr (MH == 8) {
+                                    uint32_t a[8], b[8];
+                                    tc::ld8_nw(col, a);
+                                    tc::ld8_nw(col + MT, b);
+                                    tc::wait_ld();
 #pragma unroll
-                        for (int m4 = 0; m4 < MH / 4; ++m4) {
-                            const float4 X = t4[m4];
-                            const float Xm[4] = {X.x, X.y, X.z, X.w};
+                                    for (int i = 0; i < MH; ++i)
+                                        D[e][i] = __uint_as_float(a[i]) + __uint_as_float(b[i]);
+                                } else {
+                                    uint32_t a[4], b[4];
+                                    tc::ld4_nw(col, a);
+                                    tc::ld4_nw(col + MT, b);
+                                    tc::wait_ld();
 #pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                y[4 * m4 + i] = fmaf(s16, D[4 * m4 + i], fmaf(szc, Xm[i], y[4 * m4 + i]));
+                                    for (int i = 0; i < MH; ++i)
+                                        D[e][i] = __uint_as_float(a[i]) + __uint_as_float(b[i]);
+                                }
+                            }
+                            if (pr == 1) {        // this warp's reads of the D set are done
+                                tc::fence_before();
+                                __syncwarp();
+                                if (lane == 0) mbar_arrive(smem_u32(&dempty[hs]));
+                            }
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int gl = hs * tcd::kHalf + 2 * pr + e;
+                                const float2 s2 = half2_bits_to_float2(sw[gl >> 1]);
+                                const float2 z2 = half2_bits_to_float2(zw[gl >> 1]);
+                                const float sc = e ? s2.y : s2.x, zc = e ? z2.y : z2.x;
+                                const float s16 = 16.0f * sc, szc = -sc * (16.0f + zc);
+                                const float4 *t4 = reinterpret_cast<const float4 *>(tab + gl * MT);
+#pragma unroll
+                                for (int m4 = 0; m4 < MH / 4; ++m4) {
+                                    const float4 X = t4[m4];
+                                    const float Xm[4] = {X.x, X.y, X.z, X.w};
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i)
+                                        y[4 * m4 + i] = fmaf(s16, D[e][4 * m4 + i],
+                                                             fmaf(szc, Xm[i], y[4 * m4 + i]));
+                                }
+                            }
                         }
                     }
                     if (!ok) break;
