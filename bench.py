@@ -90,16 +90,31 @@ def workload_flops(name: str) -> int:
     return sum(2 * M * m.N * m.K for m in wl.layer_set(shape_set, layers))
 
 
+def decode_kernel(name: str) -> str:
+    """The decode kernel the library picks for a workload's grouped call
+    (all decode workloads here are large enough for the streaming kernels)."""
+    _, _, mode, bits, _, M, _ = WORKLOADS[name]
+    if M <= 4:
+        return "stream"
+    if M <= 16 and (mode == "packed" or bits <= 8):
+        return "tc"
+    return "general"
+
+
 def launches_per_step(name: str, count: int) -> int:
     """Kernel launches the library makes for one grouped call (its own
     chunking of the descriptor list: 80 matrices per tensor-core GEMM
-    launch, 400 per streaming GEMV launch, 368 x 16-row chunks of M for the
-    general GEMV)."""
+    launch; 168 per streaming decode launch, plus the activation pre-pass
+    before each launch of the tensor-core decode kernel; 368 x 16-row
+    chunks of M for the general GEMV)."""
     M = WORKLOADS[name][5]
     if is_prefill(name):
         return -(-count // 80)
-    if M <= 4:
-        return -(-count // 400)
+    kind = decode_kernel(name)
+    if kind == "stream":
+        return -(-count // 168)
+    if kind == "tc":
+        return 2 * -(-count // 168)
     return -(-M // 16) * -(-count // 368)
 
 
@@ -548,8 +563,9 @@ def run_ours(args, rank, world, local_rank):
                 "traffic": traffic,
                 "peak_source": f"{peaks['source']} copy bandwidth "
                                "(MEASURED_PEAKS.json hbm_gbs)",
-                "kernel": "gemv_stream_kernel (bc_gemv_stream.cu)" if M <= 4
-                          else "gemv_kernel (bc_gemv.cu)",
+                "kernel": {"stream": "gemv_stream_kernel (bc_gemv_stream.cu)",
+                           "tc": "gemv_tc_kernel (bc_gemv_stream.cu)",
+                           "general": "gemv_kernel (bc_gemv.cu)"}[decode_kernel(name)],
                 "avg_step_us": avg_launch_ms * 1e3}
     line = {
         "metric": METRIC, "value": agg["value"], "unit": unit,

@@ -362,25 +362,29 @@ bc_status launch_mt(const GemvParams &P, int mt, int grid, cudaStream_t s) {
 }
 
 // Whole launches with at least half an SM's worth of 128-row units per SM
-// go to the streaming kernel (M <= 4, or M <= 16 for packed codes); lone
-// small matrices keep the split-K GEMV.
-bool use_stream(const GemvJob *jobs, int count, int M, bool packed,
+// go to the streaming kernels (M <= 4; M <= 16 for packed codes and for
+// runtime RTN below 16 bits); lone small matrices keep the split-K GEMV.
+bool use_stream(const GemvJob *jobs, int count, int M, bool packed, int bits,
                 const DeviceInfo &di) {
-    if (M > (packed ? 16 : 4)) return false;
+    if (M > (packed || bits <= 8 ? 16 : 4)) return false;
     int64_t units = 0;
     for (int i = 0; i < count; ++i) units += (jobs[i].N + 127) / 128;
     if (units < di.sm_count / 2) return false;
-    return gemv_stream_supported(jobs, count, M, packed, di.max_smem_optin);
+    return gemv_stream_supported(jobs, count, M, packed, bits, di.max_smem_optin);
 }
 
 }  // namespace
 
 size_t gemv_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed,
                             int sm_count) {
+    // The bit width is not known here: a runtime launch that the tensor-core
+    // decode kernel would take at 2..8 bits uses the general GEMV at 16.
     DeviceInfo di;
-    if (device_info(&di) && use_stream(jobs, count, M, packed, di))
-        return gemv_stream_workspace_bytes(jobs, count, M, packed);
     size_t worst = 0;
+    if (device_info(&di) && use_stream(jobs, count, M, packed, 8, di)) {
+        worst = gemv_stream_workspace_bytes(jobs, count, M, packed, 8);
+        if (packed || M <= 4) return worst;
+    }
     for (int b = 0; b < count; b += kMaxJobs) {
         const int n = std::min(kMaxJobs, count - b);
         Plan p = make_plan(jobs + b, n, std::min(M, 16), packed, sm_count);
@@ -394,7 +398,7 @@ bc_status launch_gemv(const GemvJob *jobs, int count, int M, int bits,
                       cudaStream_t s, bool early_start) {
     DeviceInfo di;
     if (!device_info(&di)) return BC_ERR_CUDA;
-    if (use_stream(jobs, count, M, packed, di))
+    if (use_stream(jobs, count, M, packed, bits, di))
         return launch_gemv_stream(jobs, count, M, bits, packed, s, early_start, workspace,
                                   ws_bytes);
     // ~32 KB of kernel parameters, kept off the stack; the launch copies it.

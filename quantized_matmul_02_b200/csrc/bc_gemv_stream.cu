@@ -18,8 +18,8 @@
 //               stager and the consumers together before streaming starts.
 //   warps 2-3   (packed) scale/zero stagers: the fp16 scales and zeros of each
 //               stage (64 rows x 8 groups each) into a ring slot beside it,
-//               with coalesced loads two stages ahead of the stores; each
-//               arrival is one more that the stage's full barrier counts.
+//               with coalesced loads two stages ahead of the stores; every
+//               lane of them arrives on the stage's full barrier.
 //   consumers   packed: 8 warps, warp g owns rows 16g..16g+15 of each unit over
 //               both 128-byte windows of every stage (tensor cores).  Runtime:
 //               16 warps of 8 rows each (CUDA-core quantizer, which needs more
@@ -48,7 +48,11 @@
 // exact-rounding fast path of the general GEMV (bc_gemv.cu).
 //
 // Every mbarrier wait is bounded; a wait that runs out stops the CTA (its
-// outputs are then incomplete) and is counted for bc_device_timeouts.
+// outputs are then incomplete) and is counted for bc_device_timeouts.  A
+// thread that read or wrote a shared-memory slot arrives on the slot's
+// barrier itself: an arrive orders only the arriving thread's own accesses,
+// so a single lane arriving for its warp could let the producer overwrite a
+// slot while other lanes' loads are still in flight.
 #include "bc_internal.cuh"
 #include "bc_tc.cuh"
 
@@ -85,13 +89,7 @@ constexpr int kSzBytes = 2 * kRows * 16;   // packed: fp16 scales + zeros of a s
 constexpr int kMaxJobs = 168;
 constexpr int kMaxCtas = 160;
 constexpr int kMaxM = 4;                 // rows of x held in a per-matrix smem slot
-constexpr int kMaxMChunk = 16;           // rows of x streamed per stage from the workspace
-// Chunk mode (M = 5..16, packed): the activation digits of one 512-k stage
-// chunk for one x row -- 16 rows (digit d, lane t) of kXcRS words (16 units x
-// 2 parities + 4 words of padding against bank conflicts), then (f, X~) of
-// the chunk's 8 groups for both digit pairs.
-constexpr int kXcRS = 36;
-constexpr int kXcRowBytes = 16 * kXcRS * 4 + 2 * 8 * 8;   // 2432
+constexpr int kMaxMChunk = 16;           // packed: rows of x of the tensor-core kernel
 constexpr int kXP = 26;                 // bits of the odd-k activation integers (even: +4)
 constexpr long long kWaitCycles = 4000000000LL;
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
@@ -113,7 +111,7 @@ struct __align__(64) StreamParams {
     int count, total_units, M, bits;
     int xslot_bytes, stages, max_cta_jobs;
     int early;                    // launched as a programmatic dependent launch
-    int xchunk_bytes;             // chunk mode: bytes of one stage's x chunk (MT rows)
+    int xchunk_bytes;             // tensor-core kernel: bytes of one stage's x chunk
 };
 static_assert(sizeof(StreamParams) <= 32000, "kernel parameter space");
 
@@ -342,11 +340,10 @@ __device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
     }
 }
 
-// ---- chunk mode: activation digits into the workspace ---------------------------
-// One launch before the streaming kernel turns every distinct x of the call
-// into per-stage chunks: x i, chunk kc, row m at out_i + (kc*MT + m) *
-// kXcRowBytes (rows m >= M are zero).  A warp does one (x, kc, m, half)
-// task: 4 of the chunk's 8 groups.
+// ---- activation pre-pass tasks (tensor-core kernel) -----------------------------
+// One launch before the tensor-core kernel prepares every distinct x of the
+// call per stage chunk (see xpieces_kernel); tasks are numbered per x from
+// task_begin.
 struct XdigTask {
     const float *x;
     uint8_t *out;
@@ -356,48 +353,6 @@ struct XdigParams {
     XdigTask t[kMaxJobs];
     int count, M, MT, total;
 };
-__global__ void __launch_bounds__(256) xdig_kernel(const __grid_constant__ XdigParams P) {
-    const int lane = threadIdx.x & 31, j = lane & 7;
-    const int nw = (gridDim.x * blockDim.x) >> 5;
-    for (int task = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; task < P.total; task += nw) {
-        int lo = 0, hi = P.count - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (P.t[mid].task_begin <= task) lo = mid; else hi = mid - 1;
-        }
-        const XdigTask &T = P.t[lo];
-        int r = task - T.task_begin;
-        const int half = r & 1;
-        r >>= 1;
-        const int m = r % P.MT, kc = r / P.MT;
-        const int gl = 4 * half + (lane >> 3);           // group within the chunk
-        const int g = 8 * kc + gl;
-        float v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-        if (m < P.M && g < (T.K >> 6)) {
-            const float4 *p = reinterpret_cast<const float4 *>(T.x + (int64_t)m * T.K + 64 * g + 8 * j);
-            const float4 a = __ldg(p), b = __ldg(p + 1);
-            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-        }
-        uint32_t te[4], to[4];
-        float f, xt;
-        group_digits(v, te, to, f, xt);
-        uint8_t *row = T.out + ((int64_t)kc * P.MT + m) * kXcRowBytes;
-        uint32_t *dig = reinterpret_cast<uint32_t *>(row);
-        float2 *tab = reinterpret_cast<float2 *>(row + 16 * kXcRS * 4);
-        const int U = 2 * gl + (j >> 2), tt = j & 3;
-#pragma unroll
-        for (int d = 0; d < 4; ++d)
-            *reinterpret_cast<uint2 *>(dig + (d * 4 + tt) * kXcRS + 2 * U) = make_uint2(te[d], to[d]);
-        if (j == 0) {
-            tab[gl] = make_float2(f, xt);
-            tab[8 + gl] = make_float2(f * 65536.0f, 0.0f);
-        }
-    }
-}
-
 // One x row of a runtime-mode slot: fp32, zero past K.
 __device__ void stage_x_runtime(const float *__restrict__ xr, int K, uint8_t *xm,
                                 int widx, int nw, int lane) {
@@ -447,7 +402,7 @@ __device__ __forceinline__ bool x_enter(XCursor &c, const StreamJob &J, bool fir
     if (!first && J.x == c.cur) return true;
     if (!first) {
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&xempty[(c.e - 1) & 1]));
+        mbar_arrive(smem_u32(&xempty[(c.e - 1) & 1]));     // every lane, after its reads
     }
     c.cur = J.x;
     if (!mbar_wait(smem_u32(&xfull[c.e & 1]), (c.e >> 1) & 1, abort_flag)) return false;
@@ -610,7 +565,7 @@ __device__ __forceinline__ void consume_packed_m1(
         // stage released: the arrive's release semantics order this warp's
         // ldmatrix reads (made visible to lane 0 by the warp sync) before it
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));
+        mbar_arrive(smem_u32(&empty[k.sidx]));       // every lane, after its reads
         Walk n;
         const bool more = k.next(jobs, jc, u1, kch, S, n);
         if (more && !load(nxt, n.sidx, n.sph)) return true;
@@ -670,19 +625,16 @@ __device__ __forceinline__ void consume_packed_m1(
     }
 }
 
-// ---- packed consumer, 2 to 16 x rows ------------------------------------------------
+// ---- packed consumer, 2 or 4 x rows ------------------------------------------------
 // Each mma takes one 32-k unit (slots 0-15 even k, 16-31 odd k) and a pair of
-// x rows as B columns (row 2*mp + h in columns 4h..4h+3).  With 2 or 4 rows
-// the digits come from the matrix's x slot; with 8 or 16 (chunk mode, XC)
-// from the stage's own x chunk, which the loader streams with the weights.
+// x rows as B columns (row 2*mp + h in columns 4h..4h+3), digits from the
+// matrix's x slot.
 template <int MT>
 __device__ __forceinline__ void consume_packed_mx(
     const StreamParams &P, const StreamJob *jobs, int jf, int jc, uint8_t *smem,
     const uint8_t *szring, uint8_t *xslots, uint64_t *full, uint64_t *empty, uint64_t *xfull,
-    uint64_t *xempty, volatile int *abort_flag, int u0, int u1, int rg, int lane,
-    const uint8_t *xring) {
+    uint64_t *xempty, volatile int *abort_flag, int u0, int u1, int rg, int lane) {
     constexpr int MP = MT / 2;
-    constexpr bool XC = MT > kMaxM;
     const int S = P.stages;
     const int gq = lane >> 2, t = lane & 3;
     // ldmatrix: this lane gives the address of row lrow of unit (2j + (lane>>4))
@@ -699,21 +651,19 @@ __device__ __forceinline__ void consume_packed_mx(
     float ya[MP], yb[MP];
 #pragma unroll
     for (int p = 0; p < MP; ++p) ya[p] = yb[p] = 0.0f;
-    if (!XC && !x_enter(xc, jobs[k.jidx], true, xslots, P.xslot_bytes, xfull, xempty,
-                        abort_flag, lane))
+    if (!x_enter(xc, jobs[k.jidx], true, xslots, P.xslot_bytes, xfull, xempty, abort_flag, lane))
         return;
     auto step = [&]() -> bool {
         const StreamJob &J = jobs[k.jidx];
         const int kch = kchunks_of<true>(J.K);
-        // x rows: slot rows of `mb` bytes (digit stride rs, k offset of this
-        // chunk), or chunk rows of kXcRowBytes
-        const int rs = XC ? kXcRS : dig_rs(kch);
-        const int mb = XC ? kXcRowBytes : xrow_bytes<true>(J.K);
-        const uint8_t *xb = XC ? xring + k.sidx * P.xchunk_bytes : xc.xs;
-        const int u_off = XC ? 0 : 16 * k.kc;            // unit offset of this chunk
-        const int tab_off = XC ? 16 * kXcRS * 4 : 64 * rs;
-        const int g_off = XC ? 0 : 8 * k.kc;              // group offset of this chunk
-        const int gpad = XC ? 8 : 8 * kch;
+        // x rows: slot rows of `mb` bytes (digit stride rs, k offset of this chunk)
+        const int rs = dig_rs(kch);
+        const int mb = xrow_bytes<true>(J.K);
+        const uint8_t *xb = xc.xs;
+        const int u_off = 16 * k.kc;            // unit offset of this chunk
+        const int tab_off = 64 * rs;
+        const int g_off = 8 * k.kc;              // group offset of this chunk
+        const int gpad = 8 * kch;
         if (!mbar_wait(smem_u32(&full[k.sidx]), k.sph, abort_flag)) return true;
         const uint32_t box0 = smem_u32(smem + k.sidx * kStageBytes);
         // scales / zeros of rows ra, ra+8, groups 4w..4w+3 of both windows
@@ -738,9 +688,9 @@ __device__ __forceinline__ void consume_packed_mx(
             for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) hi[j][i] = R[j][i] & 0xF0F0F0F0u;
-            if (!XC && w == 1) {
+            if (w == 1) {
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));   // stage consumed
+                mbar_arrive(smem_u32(&empty[k.sidx]));   // stage consumed (every lane)
             }
             float sa[4], sb[4], za[4], zb[4];
 #pragma unroll
@@ -785,10 +735,6 @@ __device__ __forceinline__ void consume_packed_mx(
                 }
             }
         }
-        if (XC) {        // the stage's x chunk was read up to the last row pair
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));
-        }
         Walk n;
         const bool more = k.next(jobs, jc, u1, kch, S, n);
         if (n.kc == 0 || !more) {      // unit done: two lanes per row and x row
@@ -806,7 +752,7 @@ __device__ __forceinline__ void consume_packed_mx(
             }
         }
         if (!more) return true;
-        if (!XC && n.kc == 0 &&
+        if (n.kc == 0 &&
             !x_enter(xc, jobs[n.jidx], false, xslots, P.xslot_bytes, xfull, xempty, abort_flag,
                      lane))
             return true;
@@ -925,8 +871,7 @@ __device__ __forceinline__ void consume_runtime(
                 }
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty[k.sidx]));
+        mbar_arrive(smem_u32(&empty[k.sidx]));       // every lane, after its reads
 #pragma unroll
         for (int m = 0; m < MT; ++m) yacc[m] = fmaf(part_acc[m], s_cur, yacc[m]);
         if (n.kc == 0 || !more) {       // unit done: the four lanes of a row
@@ -961,9 +906,9 @@ __device__ __forceinline__ void prefetch_xs(const StreamParams &P, const StreamJ
     }
 }
 
-// Warp 2 of a packed launch: the scale / zero slice of every stage of the
-// CTA's range, in ring order, gated by the same empty barriers as the loader
-// and counted as a second arrival on each full barrier.
+// Warps 2-3 of a packed launch: the scale / zero slice of every stage of the
+// CTA's range, in ring order, gated by the same empty barriers as the loader;
+// every lane arrives on the stage's full barrier after its stores.
 __device__ __forceinline__ void sz_stager(const StreamParams &P, const StreamJob *jobs, int jf,
                                        int jc, uint8_t *szring, uint64_t *full, uint64_t *empty,
                                        volatile int *abort_flag, int u0, int u1, int half,
@@ -993,8 +938,9 @@ __device__ __forceinline__ void sz_stager(const StreamParams &P, const StreamJob
         __syncwarp();
         if (!got) return true;
         sz_store(jobs, st, half, lane, cur, szring + sidx * kSzBytes);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&full[sidx]));
+        // every lane arrives after its own stores (an arrive orders the
+        // arriving thread's accesses only)
+        mbar_arrive(smem_u32(&full[sidx]));
         if (++sidx == S) {
             sidx = 0;
             sph ^= 1;
@@ -1006,18 +952,19 @@ __device__ __forceinline__ void sz_stager(const StreamParams &P, const StreamJob
 }
 
 // Loader warp: the TMA of every stage of the CTA's unit range (the weights
-// of 128 rows x 256 bytes as two 128-byte boxes, and in the chunk modes the
-// stage's activation chunk, `xchunk` bytes from job.x + kc * xchunk into ring
-// slot s at xring + s * xstride), gated by the empty barriers.  It then waits
-// (bounded) for its copies in flight, so none lands after the CTA has exited.
+// of 128 rows x 256 bytes as two 128-byte boxes), gated by the empty
+// barriers.  For the tensor-core kernel (xslots > 0) it also loads each
+// stage's activation chunk, `xchunk` bytes from job.x + kc * xchunk, into a
+// ring of `xslots` slots at xring + slot * xstride with barriers xfull /
+// xempty.  It then waits (bounded) for its copies in flight, so none lands
+// after the CTA has exited.
 template <bool PACKED>
 __device__ void load_stages(const StreamParams &P, const StreamJob *jobs, int jf, int jc,
                             int u0, int u1, uint8_t *smem, uint8_t *xring, int xchunk,
                             int xstride, uint64_t *full, uint64_t *empty,
-                            volatile int *abort_flag, int lane) {
+                            volatile int *abort_flag, int lane, int xslots = 0,
+                            uint64_t *xfull = nullptr, uint64_t *xempty = nullptr) {
     const int S = P.stages;
-    // chunk modes: the x chunks are written by the kernel just before
-    if (xchunk) asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint64_t policy = evict_first_policy();
     uint32_t g = 0, armed = 0;
     int jw = jf;
@@ -1050,15 +997,32 @@ __device__ void load_stages(const StreamParams &P, const StreamJob *jobs, int jf
                 // a window wholly past the row end is not loaded: its codes
                 // meet zero activations (packed) or are skipped (runtime)
                 const int nbox = (rbytes - kc * kChunk) > 128 ? 2 : 1;
-                mbar_expect_tx(fb, (uint32_t)(nbox * kBoxBytes + xchunk));
+                mbar_expect_tx(fb, (uint32_t)(nbox * kBoxBytes));
                 const uint32_t st = smem_u32(smem + s * kStageBytes);
                 for (int b = 0; b < nbox; ++b)
                     tma_load_2d(st + b * kBoxBytes, &P.wmap[j], kc * kChunk + b * 128, r0, fb,
                                 policy);
-                if (xchunk)      // job.x holds this matrix's x chunks in chunk modes
-                    bulk_load(smem_u32(xring + s * xstride),
-                              reinterpret_cast<const uint8_t *>(J.x) + (int64_t)kc * xchunk,
-                              (uint32_t)xchunk, fb);
+                if (xslots) {      // job.x holds this matrix's x chunks
+                    const uint8_t *xsrc =
+                        reinterpret_cast<const uint8_t *>(J.x) + (int64_t)kc * xchunk;
+                    const int xs = (int)(g % (uint32_t)xslots);
+                    const uint32_t use = g / (uint32_t)xslots;
+                    got = use == 0 || mbar_wait(smem_u32(&xempty[xs]), (use - 1) & 1, abort_flag);
+                    if (got) {
+                        const uint32_t xb = smem_u32(&xfull[xs]);
+                        mbar_expect_tx(xb, (uint32_t)xchunk);
+                        bulk_load(smem_u32(xring + xs * xstride), xsrc, (uint32_t)xchunk, xb);
+                    }
+                }
+            }
+            if (xslots) {
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (!got) {
+                    ok = false;
+                    armed |= 1u << s;
+                    ++g;
+                    break;
+                }
             }
             armed |= 1u << s;
             if (PACKED && kc == 0) {
@@ -1090,6 +1054,15 @@ __device__ void load_stages(const StreamParams &P, const StreamJob *jobs, int jf
                    clock64() - t0 < kWaitCycles) {
             }
         }
+        // the activation ring: the last x load of each slot (an x load was
+        // issued for every stage below g, except perhaps the last)
+        for (uint32_t k = 0; xslots && k < (uint32_t)xslots && k < g; ++k) {
+            const uint32_t gl = g - 1 - k;
+            const long long t0 = clock64();
+            while (!mbar_try(smem_u32(&xfull[gl % xslots]), (gl / xslots) & 1) &&
+                   clock64() - t0 < kWaitCycles) {
+            }
+        }
     }
     __syncwarp();
 }
@@ -1101,10 +1074,8 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int S = P.stages;
-    constexpr bool XC = PACKED && MT > kMaxM;         // x streamed per stage
     uint8_t *szring = smem + S * kStageBytes;
-    uint8_t *xring = szring + (PACKED ? S * kSzBytes : 0);     // chunk mode only
-    uint8_t *xslots = xring + (XC ? S * P.xchunk_bytes : 0);
+    uint8_t *xslots = szring + (PACKED ? S * kSzBytes : 0);
     uint64_t *bars = reinterpret_cast<uint64_t *>(xslots + 2 * P.xslot_bytes);
     uint64_t *full = bars, *empty = bars + S;
     uint64_t *xfull = bars + 2 * S, *xempty = xfull + 2;
@@ -1132,14 +1103,14 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&full[s]), 1 + RL::sz_warps);
-            mbar_init(smem_u32(&empty[s]), RL::consumers);
+            mbar_init(smem_u32(&full[s]), 1 + RL::sz_warps * 32);
+            mbar_init(smem_u32(&empty[s]), RL::consumers * 32);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&xfull[b]), 32);
-            mbar_init(smem_u32(&xempty[b]), RL::consumers);
+            mbar_init(smem_u32(&xempty[b]), RL::consumers * 32);
         }
-        mbar_init(smem_u32(xfirst), RL::stagers);
+        mbar_init(smem_u32(xfirst), RL::stagers * 32);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -1148,14 +1119,14 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     // stream: queued behind the first ring fill they would hold up the start.
     // (After an early start they may not be written yet: the staging warps
     // prefetch them once the previous kernel has completed.)
-    if (!XC && !P.early && warp >= 1 && warp < 1 + RL::stagers && u0 < u1)
+    if (!P.early && warp >= 1 && warp < 1 + RL::stagers && u0 < u1)
         prefetch_xs(P, jobs, jf, jc, warp - 1, RL::stagers, lane);
     if (!P.early) __syncthreads();
 
     if (warp == 0) {
         // ---------------- loader ----------------
-        load_stages<PACKED>(P, jobs, jf, jc, u0, u1, smem, xring, XC ? P.xchunk_bytes : 0,
-                            P.xchunk_bytes, full, empty, abort_flag, lane);
+        load_stages<PACKED>(P, jobs, jf, jc, u0, u1, smem, nullptr, 0, 0, full, empty,
+                            abort_flag, lane);
     } else if (warp >= 2 && warp < RL::first_consumer) {
         // ---------------- scale / zero stagers (packed) ----------------
         if constexpr (PACKED) {
@@ -1171,7 +1142,7 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
         // would wait for it.
         bool first_ok = true;
         int j2 = -1;                     // job of the second activation, if any
-        for (int j = jf + 1; !XC && j < jc && jobs[j].unit_begin < u1; ++j)
+        for (int j = jf + 1; j < jc && jobs[j].unit_begin < u1; ++j)
             if (jobs[j].x != jobs[j - 1].x) {
                 j2 = j;
                 break;
@@ -1179,16 +1150,16 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
         // x and y belong to the previous kernel until it completes (every CTA
         // waits here, so this grid completes only after it)
         asm volatile("griddepcontrol.wait;" ::: "memory");
-        if (!XC && P.early && u0 < u1)
+        if (P.early && u0 < u1)
             prefetch_xs(P, jobs, jf, jc, warp == 1 ? 0 : warp - RL::first_consumer + 1,
                         RL::stagers, lane);
-        if (!XC && u0 < u1) {
+        if (u0 < u1) {
             const int wi = warp == 1 ? 0 : warp - RL::first_consumer + 1;
             stage_x<PACKED>(jobs[jf], P.M, xslots, wi, RL::stagers, lane);
             if (j2 >= 0)
                 stage_x<PACKED>(jobs[j2], P.M, xslots + P.xslot_bytes, wi, RL::stagers, lane);
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(xfirst));
+            mbar_arrive(smem_u32(xfirst));       // every lane, after its writes
             if (warp == 1) {
                 first_ok = mbar_wait(smem_u32(xfirst), 0, abort_flag);
                 if (first_ok) {
@@ -1199,7 +1170,6 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
         }
         if (warp == 1) {
             // ---------------- activation stager (slot mode) ----------------
-            if (XC) first_ok = false;
             const float *cur = nullptr;
             uint32_t e = 0;
             const uint32_t pre = j2 >= 0 ? 2u : 1u;     // slots filled above
@@ -1230,7 +1200,7 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
                     else
                         consume_packed_mx<MT>(P, jobs, jf, jc, smem, szring, xslots, full,
                                               empty, xfull, xempty, abort_flag, u0, u1, rg,
-                                              lane, xring);
+                                              lane);
                 } else {
                     consume_runtime<MT>(P, jobs, jf, jc, smem, xslots, full, empty, xfull,
                                         xempty, abort_flag, u0, u1, rg, lane);
@@ -1241,39 +1211,51 @@ gemv_stream_kernel(const __grid_constant__ StreamParams P) {
     __syncthreads();
 }
 
-// ---- tensor-core decode (tcgen05), packed codes, 1..16 x rows ---------------------
+// ---- tensor-core decode (tcgen05), 5..16 x rows -------------------------------
 // Swap-AB: the unit's 128 weight rows are the MMA's M (TMEM lanes) and the x
-// rows its N = 16.  Per 64-group of K:
-//   * A = 1 + q/16 in bf16 (exact), unpacked by transform warps straight from
-//     the swizzled weight stage into tensor memory (32 columns per group);
+// rows its N.  Per 64-group of K:
+//   * A holds the codes in bf16 (exact), written by transform warps straight
+//     into tensor memory (32 columns per group):
+//       - packed: A = 1 + q/16, unpacked from the swizzled stage of int4 codes;
+//       - runtime: A = q, the RTN code of each fp16 weight (BITCRUSH BC-06,
+//         "Under the hood": codes formed as the weights are read), exact by
+//         the same fast path and fallback as the other decode kernels;
 //   * B = x split into two bf16 pieces, hi = bf16(x), lo = bf16(x - hi), so
 //     x~ = hi + lo carries 16 significant bits; a pre-pass writes them per
 //     stage chunk in the MMA's K-major 128-byte-swizzled layout, with
 //     X~ = sum over the group of x~ (fp64 sum, rounded once);
 //   * tcgen05.mma.kind::f16 (A from TMEM, B from smem, fp32 in TMEM) gives
-//     D = sum_k (1 + q_k/16) x~_k, so that
-//         s sum_k (q_k - z) x~_k = 16 s D - s (16 + z) X~,
-//     two FMAs per output and group in the epilogue warps.
+//     D = sum_k A_k x~_k per group, and the epilogue warps form
+//         s sum_k (q_k - z) x~_k = 16 s D - s (16 + z) X~   (packed)
+//                                 =    s D - s z X~         (runtime),
+//     two FMAs per output and group.
 // Both pieces share one MMA: B rows 0..MT-1 hold hi, MT..2MT-1 lo (N = 2 MT),
 // added in the epilogue.  Products are exact; D carries fp32 accumulation
 // only.  The codes enter A in the order (k_i, k_i+4) per TMEM column of each
 // 8-k block; the pre-pass writes x~ in that same order.
 //
-// Tensor memory holds two half-stage sets (4 groups each) of A (4 x 32
-// columns) and of D (4 x 2 MT columns), so the transform, the MMAs and the
-// epilogue work on different half-stages; within a half-stage the MMAs of
-// the four groups are interleaved, so one group's dependent accumulation
-// hides behind the others.
+// Tensor memory holds two sets of A (up to 4 groups x 32 columns) and of D
+// (groups x 2 MT columns), so the transform, the MMAs and the epilogue work
+// on different sets; within a set the MMAs of its groups are interleaved,
+// so one group's dependent accumulation hides behind the others.  A packed
+// stage (512 k) is two sets of 4 groups, a runtime stage (128 k) one set of
+// 2.  The activation chunks have a ring of their own (two slots), which
+// leaves shared memory for a deeper weight ring.
 namespace tcd {
-constexpr int kGroups = 8;                  // 64-groups per stage
-constexpr int kHalf = 4;                    // groups per half-stage
 constexpr int kTmemCols = 512;
-constexpr int kAcol = 0;                    // A: 2 sets x 4 groups x 32 columns
-constexpr int kDcol = 256;                  // D: 2 sets x 4 groups x 2 MT columns
+constexpr int kAcol = 0;                    // A: 2 sets x up to 4 groups x 32 columns
+constexpr int kDcol = 256;                  // D: 2 sets x up to 4 groups x 2 MT columns
 constexpr int kLoaderWarp = 0, kMmaWarp = 1, kSzWarp0 = 2, kTrWarp0 = 4, kTrWarps = 8;
 constexpr int kEpWarp0 = 12, kEpWarps = 8;
 constexpr int kThreads = 32 * (kEpWarp0 + kEpWarps);
-template <int MT> struct Chunk {
+constexpr int kXSlots = 2;                      // activation-chunk ring
+template <bool PACKED> struct Geo {
+    static constexpr int kGroups = PACKED ? 8 : 2;         // 64-groups per stage
+    static constexpr int kSetGroups = PACKED ? 4 : 2;      // groups per TMEM set
+    static constexpr int kSets = kGroups / kSetGroups;     // sets per stage
+};
+template <bool PACKED, int MT> struct Chunk {
+    static constexpr int kGroups = Geo<PACKED>::kGroups;
     static constexpr int kTile = 2 * MT * 128;             // 2 MT rows x 128 bytes
     static constexpr int kTab = kGroups * kTile;           // X~ [group][MT] f32
     static constexpr int kBytes = kTab + kGroups * MT * 4;
@@ -1283,17 +1265,18 @@ template <int MT> struct Chunk {
 // offset of its 128-byte row.
 template <int MT> __host__ __device__ __forceinline__ int brow_off(int gl, int m, int p) {
     const int row = p * MT + m;
-    return gl * Chunk<MT>::kTile + (row >> 3) * 1024 + (row & 7) * 128;
+    return gl * (2 * MT * 128) + (row >> 3) * 1024 + (row & 7) * 128;
 }
 }  // namespace tcd
 
 // Pre-pass: the bf16 pieces of every distinct x of the launch, per stage
-// chunk, into the workspace.  A warp does one (x, chunk, row m, half) task,
-// 4 groups of 64 k, 8 lanes per group, 8 k per lane (one 16-byte piece of
-// a B row).  Rows m >= M and groups past K/64 are zero.
-template <int MT>
+// chunk, into the workspace.  A warp does one (x, chunk, row m, quad) task:
+// up to 4 groups of 64 k, 8 lanes per group, 8 k per lane (one 16-byte piece
+// of a B row).  Rows m >= M and groups past K/64 are zero.
+template <bool PACKED, int MT>
 __global__ void __launch_bounds__(256) xpieces_kernel(const __grid_constant__ XdigParams P) {
-    using C = tcd::Chunk<MT>;
+    using C = tcd::Chunk<PACKED, MT>;
+    constexpr int Q = (C::kGroups + 3) / 4;          // quads per chunk
     const int lane = threadIdx.x & 31, j = lane & 7;
     const int nw = (gridDim.x * blockDim.x) >> 5;
     for (int task = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; task < P.total; task += nw) {
@@ -1304,15 +1287,15 @@ __global__ void __launch_bounds__(256) xpieces_kernel(const __grid_constant__ Xd
         }
         const XdigTask &T = P.t[lo];
         int r = task - T.task_begin;
-        const int half = r & 1;
-        r >>= 1;
+        const int quad = r % Q;
+        r /= Q;
         const int m = r % MT, kc = r / MT;
-        const int gl = 4 * half + (lane >> 3);
-        const int g = tcd::kGroups * kc + gl;
+        const int gl = 4 * quad + (lane >> 3);
+        const int g = C::kGroups * kc + gl;
         float v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-        if (m < P.M && g < (T.K >> 6)) {
+        if (m < P.M && gl < C::kGroups && g < (T.K >> 6)) {
             const float4 *p = reinterpret_cast<const float4 *>(T.x + (int64_t)m * T.K + 64 * g + 8 * j);
             const float4 a = __ldg(p), b = __ldg(p + 1);
             v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
@@ -1333,6 +1316,7 @@ __global__ void __launch_bounds__(256) xpieces_kernel(const __grid_constant__ Xd
         sum += __shfl_xor_sync(0xffffffffu, sum, 1);
         sum += __shfl_xor_sync(0xffffffffu, sum, 2);
         sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+        if (gl >= C::kGroups) continue;
         uint8_t *chunk = T.out + (int64_t)kc * C::kBytes;
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
@@ -1359,23 +1343,65 @@ __device__ __forceinline__ void unpack_a(uint32_t w, uint32_t *o) {
     o[3] = t;
 }
 
-template <int MT>
+// Runtime RTN: codes q of 8 fp16 weights (one 16-byte chunk, k0..k7) as
+// bf16 pairs (k_i, k_i+4).  Fast path: q - z = clamp(rint(w / s), -z, L - z)
+// through the approximate reciprocal, exact unless some |w/s - w rcp(s)|
+// could reach a rounding boundary (then the chunk takes the exact quotient);
+// q = (q - z) + z in exact integer arithmetic.
+__device__ __forceinline__ void rtn_codes8(uint4 raw, float s, float z, float L,
+                                           uint32_t *o) {
+    const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
+    float wv[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f2 = __half22float2(h2[i]);
+        wv[2 * i] = f2.x;
+        wv[2 * i + 1] = f2.y;
+    }
+    const float inv = rcp_approx(s);
+    const float lo_c = -z, hi_c = L - z;
+    const float thr = 0.5f - (fmaxf(fabsf(lo_c), fabsf(hi_c)) + 2.0f) * 4.76837158203125e-07f;
+    float cq[8];
+    float emax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float v = fmaf(wv[i], inv, kMagic);
+        const float r = v - kMagic;
+        const float ee = fmaf(wv[i], inv, -r);
+        emax = fmaxf(emax, fabsf(ee));
+        cq[i] = fminf(fmaxf(r, lo_c), hi_c);
+    }
+    if (emax > thr) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cq[i] = centered_code_exact(wv[i], s, z, L);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 p = __floats2bfloat162_rn(cq[i] + z, cq[i + 4] + z);
+        o[i] = *reinterpret_cast<const uint32_t *>(&p);
+    }
+}
+
+template <bool PACKED, int MT>
 __global__ void __launch_bounds__(tcd::kThreads, 1)
 gemv_tc_kernel(const __grid_constant__ StreamParams P) {
-    using C = tcd::Chunk<MT>;
+    using C = tcd::Chunk<PACKED, MT>;
+    using G = tcd::Geo<PACKED>;
     constexpr int NB = 2 * MT;                       // MMA N: hi and lo rows of B
     constexpr int MH = MT / 2;                       // x rows per epilogue warp
+    constexpr int SG = G::kSetGroups;
     constexpr uint32_t kIdesc = tc::idesc_bf16(128, NB);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int S = P.stages;
     uint8_t *szring = smem + S * kStageBytes;
-    uint8_t *xring = szring + S * kSzBytes;            // 1024-aligned slots
-    uint64_t *bars = reinterpret_cast<uint64_t *>(xring + S * C::kStride);
+    uint8_t *xring = szring + (PACKED ? S * kSzBytes : 0);     // 1024-aligned slots
+    uint64_t *bars = reinterpret_cast<uint64_t *>(xring + tcd::kXSlots * C::kStride);
     uint64_t *full = bars, *empty = bars + S;
-    uint64_t *afull = bars + 2 * S;                     // A set written (8 warps)
-    uint64_t *done = afull + 2;                         // MMAs of a half-stage complete
+    uint64_t *xfull = bars + 2 * S, *xempty = xfull + tcd::kXSlots;
+    uint64_t *afull = xempty + tcd::kXSlots;            // A set written (8 warps)
+    uint64_t *done = afull + 2;                         // MMAs of a set complete
     uint64_t *dempty = done + 2;                        // D set read (8 warps)
     uint64_t *mma_final = dempty + 2;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(mma_final + 1);
@@ -1396,8 +1422,14 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
     const StreamJob *jobs = jobs_sm - jf;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&full[s]), 1 + 2);       // loader + two scale/zero stagers
-            mbar_init(smem_u32(&empty[s]), tcd::kTrWarps + tcd::kEpWarps + 1);
+            // loader, plus every lane of the two scale/zero stagers (packed)
+            mbar_init(smem_u32(&full[s]), PACKED ? 1 + 2 * 32 : 1);
+            // transform warps (one arrival each), epilogue threads
+            mbar_init(smem_u32(&empty[s]), tcd::kTrWarps + tcd::kEpWarps * 32);
+        }
+        for (int b = 0; b < tcd::kXSlots; ++b) {
+            mbar_init(smem_u32(&xfull[b]), 1);
+            mbar_init(smem_u32(&xempty[b]), 1 + tcd::kEpWarps * 32);   // MMAs + epilogue threads
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&afull[b]), tcd::kTrWarps);
@@ -1417,52 +1449,62 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
     auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
         return __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, abort_flag));
     };
+    // runtime mode: (scale, zero) of weight row `row`, group gg of job J
+    auto rt_sz = [&](const StreamJob &J, int row, int gg) -> float2 {
+        if (row >= J.N || 64 * gg >= J.K) return make_float2(0.0f, 0.0f);
+        const int64_t gi = (int64_t)row * (J.K / J.group) + (64 * gg) / J.group;
+        return make_float2(__ldg(reinterpret_cast<const float *>(J.s) + gi),
+                           __ldg(reinterpret_cast<const float *>(J.z) + gi));
+    };
 
     if (u0 < u1) {
         if (warp == tcd::kLoaderWarp) {
-            load_stages<true>(P, jobs, jf, jc, u0, u1, smem, xring, C::kBytes, C::kStride, full,
-                              empty, abort_flag, lane);
+            // activation chunks: written by the pre-pass kernel just before
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            load_stages<PACKED>(P, jobs, jf, jc, u0, u1, smem, xring, C::kBytes, C::kStride, full,
+                                empty, abort_flag, lane, tcd::kXSlots, xfull, xempty);
         } else if (warp == tcd::kMmaWarp) {
             // The whole warp walks the stages and waits; one elected lane issues
-            // a half-stage's MMAs, interleaved over its four groups.
-            // Descriptors are formed once and advanced by constant offsets
-            // (16-byte units of the start address).
+            // a set's MMAs, interleaved over its groups.  Descriptors are formed
+            // once and advanced by constant offsets (16-byte units of the start
+            // address).
             const uint64_t bdesc0 = tc::sw128_desc(smem_u32(xring));
             uint32_t g = 0;
             int j = jf;
             bool ok = true;
             for (int u = u0; u < u1 && ok; ++u) {
                 j = next_job(jobs, jc, j, u);
-                const int kch = kchunks_of<true>(jobs[j].K);
+                const int kch = kchunks_of<PACKED>(jobs[j].K);
                 for (int kc = 0; kc < kch && ok; ++kc, ++g) {
-                    const int s = (int)(g % (uint32_t)S);
-                    if (!wait_all(&full[s], (g / S) & 1)) {
+                    const int xs = (int)(g % tcd::kXSlots);
+                    if (!wait_all(&xfull[xs], (g / tcd::kXSlots) & 1)) {
                         ok = false;
                         break;
                     }
-                    const uint64_t bs = bdesc0 + (uint64_t)((s * C::kStride) >> 4);
+                    const uint64_t bs = bdesc0 + (uint64_t)((xs * C::kStride) >> 4);
 #pragma unroll
-                    for (int hs = 0; hs < 2; ++hs) {
-                        bool w = mbar_wait(smem_u32(&afull[hs]), g & 1, abort_flag);
-                        if (w && g > 0) w = mbar_wait(smem_u32(&dempty[hs]), (g - 1) & 1, abort_flag);
+                    for (int hs = 0; hs < G::kSets; ++hs) {
+                        const uint32_t t = g * G::kSets + hs, b = t & 1, k = t >> 1;
+                        bool w = mbar_wait(smem_u32(&afull[b]), k & 1, abort_flag);
+                        if (w && k > 0) w = mbar_wait(smem_u32(&dempty[b]), (k - 1) & 1, abort_flag);
                         if (!__all_sync(0xffffffffu, w)) {
                             ok = false;
                             break;
                         }
                         tc::fence_after();
                         if (tc::elect_one()) {
-                            const uint32_t d0 = tmem + tcd::kDcol + hs * tcd::kHalf * NB;
-                            const uint32_t a0 = tmem + tcd::kAcol + hs * tcd::kHalf * 32;
-                            const uint64_t b0 = bs + (uint64_t)((hs * tcd::kHalf * C::kTile) >> 4);
+                            const uint32_t d0 = tmem + tcd::kDcol + b * SG * NB;
+                            const uint32_t a0 = tmem + tcd::kAcol + b * SG * 32;
+                            const uint64_t b0 = bs + (uint64_t)((hs * SG * C::kTile) >> 4);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-                                for (int gi = 0; gi < tcd::kHalf; ++gi)
+                                for (int gi = 0; gi < SG; ++gi)
                                     tc::mma_bf16_ts(d0 + gi * NB, a0 + gi * 32 + 8 * kk,
                                                     b0 + (uint64_t)((gi * C::kTile) >> 4) + 2 * kk,
                                                     kIdesc, kk ? 1u : 0u);
-                            tc::commit(smem_u32(&done[hs]));
-                            if (hs == 1) tc::commit(smem_u32(&empty[s]));    // x chunk read
+                            tc::commit(smem_u32(&done[b]));
+                            if (hs == G::kSets - 1) tc::commit(smem_u32(&xempty[xs]));  // x read
                         }
                         __syncwarp();
                     }
@@ -1478,59 +1520,83 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
             }
             __syncwarp();
         } else if (warp < tcd::kTrWarp0) {
-            sz_stager(P, jobs, jf, jc, szring, full, empty, abort_flag, u0, u1,
-                      warp - tcd::kSzWarp0, lane);
+            if constexpr (PACKED)
+                sz_stager(P, jobs, jf, jc, szring, full, empty, abort_flag, u0, u1,
+                          warp - tcd::kSzWarp0, lane);
         } else if (warp < tcd::kEpWarp0) {
-            // ---- transform: codes -> A = 1 + q/16 (bf16) in TMEM ----
+            // ---- transform: codes -> A (bf16) in TMEM ----
             // Warp (quarter q = warp & 3, parity par) writes lanes 32q..32q+31
-            // (its rows) for groups par and par + 2 of each half-stage.
+            // (its rows) for groups par, par + 2, ... of each set.
             const int q = warp & 3, par = (warp - tcd::kTrWarp0) >> 2;
             const int r = 32 * q + lane;
             const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + tcd::kAcol;
+            const float L = (float)((1 << P.bits) - 1);
             uint32_t g = 0;
             int j = jf;
             bool ok = true;
             for (int u = u0; u < u1 && ok; ++u) {
                 j = next_job(jobs, jc, j, u);
-                const int kch = kchunks_of<true>(jobs[j].K);
+                const StreamJob &J = jobs[j];
+                const int kch = kchunks_of<PACKED>(J.K);
+                const int row = (u - J.unit_begin) * kRows + r;
                 for (int kc = 0; kc < kch && ok; ++kc, ++g) {
                     const int s = (int)(g % (uint32_t)S);
+                    float2 szv[SG / 2];
+                    if constexpr (!PACKED) {       // this warp's groups of the stage
+#pragma unroll
+                        for (int i = 0; i < SG / 2; ++i)
+                            szv[i] = rt_sz(J, row, G::kGroups * kc + par + 2 * i);
+                    }
                     if (!wait_all(&full[s], (g / S) & 1)) {
                         ok = false;
                         break;
                     }
                     const uint8_t *st = smem + s * kStageBytes;
 #pragma unroll
-                    for (int hs = 0; hs < 2; ++hs) {
-                        // the A set is free once the previous stage's MMAs on it are done
-                        if (g > 0 && !wait_all(&done[hs], (g - 1) & 1)) {
+                    for (int hs = 0; hs < G::kSets; ++hs) {
+                        const uint32_t t = g * G::kSets + hs, b = t & 1, k = t >> 1;
+                        // the A set is free once the MMAs of its previous use are done
+                        if (k > 0 && !wait_all(&done[b], (k - 1) & 1)) {
                             ok = false;
                             break;
                         }
                         tc::fence_after();
-                        const uint8_t *box = st + hs * kBoxBytes + r * 128;
 #pragma unroll
-                        for (int i = 0; i < 2; ++i) {
-                            const int gi = 2 * i + par;          // group within the half
-                            const uint4 v0 =
-                                *reinterpret_cast<const uint4 *>(box + (((2 * gi) ^ (r & 7)) << 4));
-                            const uint4 v1 =
-                                *reinterpret_cast<const uint4 *>(box + (((2 * gi + 1) ^ (r & 7)) << 4));
+                        for (int i = 0; i < SG / 2; ++i) {
+                            const int gi = 2 * i + par;          // group within the set
                             uint32_t o[32];
-                            unpack_a(v0.x, o + 0);
-                            unpack_a(v0.y, o + 4);
-                            unpack_a(v0.z, o + 8);
-                            unpack_a(v0.w, o + 12);
-                            unpack_a(v1.x, o + 16);
-                            unpack_a(v1.y, o + 20);
-                            unpack_a(v1.z, o + 24);
-                            unpack_a(v1.w, o + 28);
-                            tc::st32_nw(lane_base + hs * tcd::kHalf * 32 + gi * 32, o);
+                            if constexpr (PACKED) {
+                                const uint8_t *box = st + hs * kBoxBytes + r * 128;
+                                const uint4 v0 = *reinterpret_cast<const uint4 *>(
+                                    box + (((2 * gi) ^ (r & 7)) << 4));
+                                const uint4 v1 = *reinterpret_cast<const uint4 *>(
+                                    box + (((2 * gi + 1) ^ (r & 7)) << 4));
+                                unpack_a(v0.x, o + 0);
+                                unpack_a(v0.y, o + 4);
+                                unpack_a(v0.z, o + 8);
+                                unpack_a(v0.w, o + 12);
+                                unpack_a(v1.x, o + 16);
+                                unpack_a(v1.y, o + 20);
+                                unpack_a(v1.z, o + 24);
+                                unpack_a(v1.w, o + 28);
+                            } else {
+                                // group gi is the stage's box gi: 64 fp16 of row r
+                                const uint8_t *box = st + gi * kBoxBytes + r * 128;
+#pragma unroll
+                                for (int c = 0; c < 8; ++c) {
+                                    const uint4 raw =
+                                        *reinterpret_cast<const uint4 *>(box + ((c ^ (r & 7)) << 4));
+                                    rtn_codes8(raw, szv[i].x, szv[i].y, L, o + 4 * c);
+                                }
+                            }
+                            // tcgen05.st is warp-collective: reconverge after
+                            // the lanes that took the exact quotient
+                            __syncwarp();
+                            tc::st32(lane_base + b * SG * 32 + gi * 32, o);
                         }
-                        tc::wait_st();
                         tc::fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(smem_u32(&afull[hs]));
+                        if (lane == 0) mbar_arrive(smem_u32(&afull[b]));
                     }
                     if (!ok) break;
                     __syncwarp();
@@ -1538,7 +1604,7 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
                 }
             }
         } else {
-            // ---- epilogue: y[m][row] += 16 s (D_hi + D_lo) - s (16 + z) X~ ----
+            // ---- epilogue: y[m][row] += sc D - sz X~ ----
             // Warp (quarter q, half h) takes x rows h*MT/2 .. of its 32 weight
             // rows, over every group.
             const int q = warp & 3, h = (warp - tcd::kEpWarp0) >> 2, m0 = h * MH;
@@ -1553,85 +1619,118 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
             for (int u = u0; u < u1 && ok; ++u) {
                 j = next_job(jobs, jc, j, u);
                 const StreamJob &J = jobs[j];
-                const int kch = kchunks_of<true>(J.K);
+                const int kch = kchunks_of<PACKED>(J.K);
+                const int row = (u - J.unit_begin) * kRows + r;
                 for (int kc = 0; kc < kch && ok; ++kc, ++g) {
                     const int s = (int)(g % (uint32_t)S);
+                    // scale and zero of each group of the stage: packed fp16 words
+                    // from the stage's scale/zero slot, runtime fp32 (sc, -sc z)
+                    uint32_t sw[4], zw[4];
+                    float2 rcoef[PACKED ? 1 : G::kGroups];
+                    if constexpr (!PACKED) {
+#pragma unroll
+                        for (int gl = 0; gl < G::kGroups; ++gl) {
+                            const float2 v = rt_sz(J, row, G::kGroups * kc + gl);
+                            rcoef[gl] = make_float2(v.x, -v.x * v.y);
+                        }
+                    }
                     if (!wait_all(&full[s], (g / S) & 1)) {
                         ok = false;
                         break;
                     }
-                    const uint4 sv = *reinterpret_cast<const uint4 *>(szring + s * kSzBytes + r * 16);
-                    const uint4 zv = *reinterpret_cast<const uint4 *>(
-                        szring + s * kSzBytes + kSzBytes / 2 + r * 16);
-                    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
-                    const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
+                    if constexpr (PACKED) {
+                        const uint4 sv =
+                            *reinterpret_cast<const uint4 *>(szring + s * kSzBytes + r * 16);
+                        const uint4 zv = *reinterpret_cast<const uint4 *>(
+                            szring + s * kSzBytes + kSzBytes / 2 + r * 16);
+                        sw[0] = sv.x; sw[1] = sv.y; sw[2] = sv.z; sw[3] = sv.w;
+                        zw[0] = zv.x; zw[1] = zv.y; zw[2] = zv.z; zw[3] = zv.w;
+                    }
+                    // (multiplier of D, multiplier of X~) of group gl
+                    auto coef = [&](int gl) -> float2 {
+                        if constexpr (PACKED) {
+                            const float2 s2 = half2_bits_to_float2(sw[gl >> 1]);
+                            const float2 z2 = half2_bits_to_float2(zw[gl >> 1]);
+                            const float sc = (gl & 1) ? s2.y : s2.x, zc = (gl & 1) ? z2.y : z2.x;
+                            return make_float2(16.0f * sc, -sc * (16.0f + zc));
+                        } else {
+                            return rcoef[gl];
+                        }
+                    };
+                    const int xs = (int)(g % tcd::kXSlots);
+                    if (!wait_all(&xfull[xs], (g / tcd::kXSlots) & 1)) {
+                        ok = false;
+                        break;
+                    }
                     const float *tab =
-                        reinterpret_cast<const float *>(xring + s * C::kStride + C::kTab) + m0;
+                        reinterpret_cast<const float *>(xring + xs * C::kStride + C::kTab) + m0;
 #pragma unroll
-                    for (int hs = 0; hs < 2; ++hs) {
-                        if (!wait_all(&done[hs], g & 1)) {
+                    for (int hs = 0; hs < G::kSets; ++hs) {
+                        const uint32_t t = g * G::kSets + hs, b = t & 1, k = t >> 1;
+                        // X~ of the set's groups for this warp's x rows, read into
+                        // registers before the set's tensor-memory loads
+                        float4 tx[SG][MH / 4];
+#pragma unroll
+                        for (int gi = 0; gi < SG; ++gi)
+#pragma unroll
+                            for (int m4 = 0; m4 < MH / 4; ++m4)
+                                tx[gi][m4] =
+                                    reinterpret_cast<const float4 *>(tab + (hs * SG + gi) * MT)[m4];
+                        if (!wait_all(&done[b], k & 1)) {
                             ok = false;
                             break;
                         }
                         tc::fence_after();
 #pragma unroll
-                        for (int pr = 0; pr < 2; ++pr) {
+                        for (int pr = 0; pr < SG / 2; ++pr) {
                             float D[2][MH];
 #pragma unroll
                             for (int e = 0; e < 2; ++e) {
-                                const uint32_t col =
-                                    lane_base + (hs * tcd::kHalf + 2 * pr + e) * NB + m0;
+                                const uint32_t col = lane_base + (b * SG + 2 * pr + e) * NB + m0;
                                 if constexpr (MH == 8) {
-                                    uint32_t a[8], b[8];
-                                    tc::ld8_nw(col, a);
-                                    tc::ld8_nw(col + MT, b);
-                                    tc::wait_ld();
+                                    uint32_t a[8], c2[8];
+                                    tc::ld8x2(col, col + MT, a, c2);
 #pragma unroll
                                     for (int i = 0; i < MH; ++i)
-                                        D[e][i] = __uint_as_float(a[i]) + __uint_as_float(b[i]);
+                                        D[e][i] = __uint_as_float(a[i]) + __uint_as_float(c2[i]);
                                 } else {
-                                    uint32_t a[4], b[4];
-                                    tc::ld4_nw(col, a);
-                                    tc::ld4_nw(col + MT, b);
-                                    tc::wait_ld();
+                                    uint32_t a[4], c2[4];
+                                    tc::ld4x2(col, col + MT, a, c2);
 #pragma unroll
                                     for (int i = 0; i < MH; ++i)
-                                        D[e][i] = __uint_as_float(a[i]) + __uint_as_float(b[i]);
+                                        D[e][i] = __uint_as_float(a[i]) + __uint_as_float(c2[i]);
                                 }
                             }
-                            if (pr == 1) {        // this warp's reads of the D set are done
+                            if (pr == SG / 2 - 1) {   // this warp's reads of the D set are done
                                 tc::fence_before();
                                 __syncwarp();
-                                if (lane == 0) mbar_arrive(smem_u32(&dempty[hs]));
+                                if (lane == 0) mbar_arrive(smem_u32(&dempty[b]));
                             }
 #pragma unroll
                             for (int e = 0; e < 2; ++e) {
-                                const int gl = hs * tcd::kHalf + 2 * pr + e;
-                                const float2 s2 = half2_bits_to_float2(sw[gl >> 1]);
-                                const float2 z2 = half2_bits_to_float2(zw[gl >> 1]);
-                                const float sc = e ? s2.y : s2.x, zc = e ? z2.y : z2.x;
-                                const float s16 = 16.0f * sc, szc = -sc * (16.0f + zc);
-                                const float4 *t4 = reinterpret_cast<const float4 *>(tab + gl * MT);
+                                const int gl = hs * SG + 2 * pr + e;
+                                const float2 cf = coef(gl);
 #pragma unroll
                                 for (int m4 = 0; m4 < MH / 4; ++m4) {
-                                    const float4 X = t4[m4];
+                                    const float4 X = tx[2 * pr + e][m4];
                                     const float Xm[4] = {X.x, X.y, X.z, X.w};
 #pragma unroll
                                     for (int i = 0; i < 4; ++i)
-                                        y[4 * m4 + i] = fmaf(s16, D[e][4 * m4 + i],
-                                                             fmaf(szc, Xm[i], y[4 * m4 + i]));
+                                        y[4 * m4 + i] = fmaf(cf.x, D[e][4 * m4 + i],
+                                                             fmaf(cf.y, Xm[i], y[4 * m4 + i]));
                                 }
                             }
                         }
                     }
                     if (!ok) break;
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&empty[s]));   // scales, X~ read
+                    // every lane releases the slots after its own reads (an
+                    // arrive orders the arriving thread's loads only)
+                    mbar_arrive(smem_u32(&empty[s]));            // scales read
+                    mbar_arrive(smem_u32(&xempty[xs]));          // X~ read
                     if (kc + 1 == kch) {
-                        const int n = (u - J.unit_begin) * kRows + r;
 #pragma unroll
                         for (int i = 0; i < MH; ++i) {
-                            if (m0 + i < P.M && n < J.N) J.y[(int64_t)(m0 + i) * J.N + n] = y[i];
+                            if (m0 + i < P.M && row < J.N) J.y[(int64_t)(m0 + i) * J.N + row] = y[i];
                             y[i] = 0.0f;
                         }
                     }
@@ -1686,7 +1785,7 @@ bc_status launch_one(const StreamParams &P, int grid, int smem, cudaStream_t s) 
     return cuda_status();
 }
 
-template <int MT>
+template <bool PACKED, int MT>
 bc_status launch_tc(const StreamParams &P, int grid, int smem, cudaStream_t s) {
     static std::mutex mu;
     static int attr_smem[64] = {};
@@ -1695,7 +1794,7 @@ bc_status launch_tc(const StreamParams &P, int grid, int smem, cudaStream_t s) {
     {
         std::lock_guard<std::mutex> lock(mu);
         if (smem > attr_smem[dev]) {
-            if (cudaFuncSetAttribute(gemv_tc_kernel<MT>,
+            if (cudaFuncSetAttribute(gemv_tc_kernel<PACKED, MT>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      smem) != cudaSuccess)
                 return BC_ERR_CUDA;
@@ -1712,7 +1811,7 @@ bc_status launch_tc(const StreamParams &P, int grid, int smem, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = P.early ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, gemv_tc_kernel<MT>, P) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, gemv_tc_kernel<PACKED, MT>, P) != cudaSuccess) {
         (void)cudaGetLastError();
         return BC_ERR_CUDA;
     }
@@ -1759,23 +1858,33 @@ size_t xslot_bytes_for(const GemvJob *jobs, int count, int M, bool packed) {
     return (xmax + 127) / 128 * 128;
 }
 
-// Chunk mode: packed launches with 5..16 x rows run the tensor-core decode
-// kernel, which streams x per stage from the workspace.
-bool chunk_mode(int M, bool packed) { return packed && M > kMaxM && M <= kMaxMChunk; }
-int chunk_mt(int M) { return M <= 8 ? 8 : 16; }
-size_t chunk_bytes(int M) {
-    return chunk_mt(M) == 8 ? tcd::Chunk<8>::kBytes : tcd::Chunk<16>::kBytes;
+// Chunk mode: launches with 5..16 x rows (packed, or runtime RTN at 2..8
+// bits) run the tensor-core decode kernel, which streams x per stage from
+// the workspace.
+bool chunk_mode(int M, bool packed, int bits) {
+    return M > kMaxM && M <= kMaxMChunk && (packed || bits <= 8);
 }
-size_t chunk_stride(int M) {
-    return chunk_mt(M) == 8 ? tcd::Chunk<8>::kStride : tcd::Chunk<16>::kStride;
+int chunk_mt(int M) { return M <= 8 ? 8 : 16; }
+size_t chunk_bytes(int M, bool packed) {
+    if (packed)
+        return chunk_mt(M) == 8 ? tcd::Chunk<true, 8>::kBytes : tcd::Chunk<true, 16>::kBytes;
+    return chunk_mt(M) == 8 ? tcd::Chunk<false, 8>::kBytes : tcd::Chunk<false, 16>::kBytes;
+}
+size_t chunk_stride(int M, bool packed) {
+    if (packed)
+        return chunk_mt(M) == 8 ? tcd::Chunk<true, 8>::kStride : tcd::Chunk<true, 16>::kStride;
+    return chunk_mt(M) == 8 ? tcd::Chunk<false, 8>::kStride : tcd::Chunk<false, 16>::kStride;
+}
+int kchunks_mode(int K, bool packed) {
+    return packed ? kchunks_of<true>(K) : kchunks_of<false>(K);
 }
 
 // Workspace layout of the chunk-mode activation digits: each distinct
 // (x, K) of the launch once, in job order; off[i] is job i's offset.  A null
 // x (a size query without pointers) is never shared, which bounds any call.
-size_t xdig_layout(const GemvJob *jobs, int count, int M, std::vector<size_t> *off,
-                   std::vector<int> *first) {
-    const size_t mtb = chunk_bytes(M);
+size_t xdig_layout(const GemvJob *jobs, int count, int M, bool packed,
+                   std::vector<size_t> *off, std::vector<int> *first) {
+    const size_t mtb = chunk_bytes(M, packed);
     size_t total = 0;
     if (off) off->assign(count, 0);
     if (first) first->clear();
@@ -1789,7 +1898,7 @@ size_t xdig_layout(const GemvJob *jobs, int count, int M, std::vector<size_t> *o
         }
         if (off) (*off)[i] = total;
         if (first) first->push_back(i);
-        total += (size_t)kchunks_of<true>((int)jobs[i].K) * mtb;
+        total += (size_t)kchunks_mode((int)jobs[i].K, packed) * mtb;
     }
     return total;
 }
@@ -1853,26 +1962,27 @@ void partition_units(StreamParams &P, int n, bool packed, int grid) {
 
 }  // namespace
 
-bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed,
+bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed, int bits,
                            int max_smem) {
-    const bool xc = chunk_mode(M, packed);
+    const bool xc = chunk_mode(M, packed, bits);
     if (M < 1 || (M > kMaxM && !xc) || count < 1) return false;
     for (int i = 0; i < count; ++i)
         if (jobs[i].N >= (1 << 30) || jobs[i].K >= (1 << 24)) return false;
     const size_t xs = xc ? 0 : xslot_bytes_for(jobs, count, M, packed);
-    const size_t fixed = 2 * xs + kBarBytes + 1024;
-    const size_t per_stage = kStageBytes + (packed ? kSzBytes : 0) +
-                             (xc ? chunk_stride(M) : 0);
+    const size_t fixed =
+        2 * xs + kBarBytes + 1024 + (xc ? tcd::kXSlots * chunk_stride(M, packed) : 0);
+    const size_t per_stage = kStageBytes + (packed ? kSzBytes : 0);
     if (fixed + 2 * per_stage > (size_t)max_smem) return false;
     return tensor_map_encoder() != nullptr;
 }
 
-size_t gemv_stream_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed) {
-    if (!chunk_mode(M, packed)) return 0;
+size_t gemv_stream_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed,
+                                   int bits) {
+    if (!chunk_mode(M, packed, bits)) return 0;
     // launches above kMaxJobs matrices reuse the space batch by batch
     size_t worst = 0;
     for (int b = 0; b < count; b += kMaxJobs)
-        worst = std::max(worst, xdig_layout(jobs + b, std::min(kMaxJobs, count - b), M,
+        worst = std::max(worst, xdig_layout(jobs + b, std::min(kMaxJobs, count - b), M, packed,
                                             nullptr, nullptr));
     return worst ? worst + 256 : 0;
 }
@@ -1896,21 +2006,25 @@ constexpr int kPlanCache = 4;
 bool same_call(const StreamPlan &p, const GemvJob *jobs, int count, int M, int bits,
                bool packed, int dev, bool early, const void *ws) {
     return p.dev == dev && p.M == M && p.bits == bits && p.packed == packed &&
-           (p.P.early != 0) == early && (!chunk_mode(M, packed) || p.ws == ws) &&
+           (p.P.early != 0) == early && (!chunk_mode(M, packed, bits) || p.ws == ws) &&
            (int)p.key.size() == count &&
            std::memcmp(p.key.data(), jobs, sizeof(GemvJob) * count) == 0;
 }
 
 bc_status launch_plan(const StreamPlan &p, cudaStream_t s) {
-    if (chunk_mode(p.M, p.packed)) {
-        if (chunk_mt(p.M) == 8)
-            xpieces_kernel<8><<<p.xgrid, 256, 0, s>>>(p.X);
-        else
-            xpieces_kernel<16><<<p.xgrid, 256, 0, s>>>(p.X);
+    if (chunk_mode(p.M, p.packed, p.bits)) {
+        const int mt = chunk_mt(p.M);
+        if (p.packed && mt == 8) xpieces_kernel<true, 8><<<p.xgrid, 256, 0, s>>>(p.X);
+        if (p.packed && mt == 16) xpieces_kernel<true, 16><<<p.xgrid, 256, 0, s>>>(p.X);
+        if (!p.packed && mt == 8) xpieces_kernel<false, 8><<<p.xgrid, 256, 0, s>>>(p.X);
+        if (!p.packed && mt == 16) xpieces_kernel<false, 16><<<p.xgrid, 256, 0, s>>>(p.X);
         const bc_status st = cuda_status();
         if (st != BC_OK) return st;
-        return chunk_mt(p.M) == 8 ? launch_tc<8>(p.P, p.grid, p.smem, s)
-                                  : launch_tc<16>(p.P, p.grid, p.smem, s);
+        if (p.packed)
+            return mt == 8 ? launch_tc<true, 8>(p.P, p.grid, p.smem, s)
+                           : launch_tc<true, 16>(p.P, p.grid, p.smem, s);
+        return mt == 8 ? launch_tc<false, 8>(p.P, p.grid, p.smem, s)
+                       : launch_tc<false, 16>(p.P, p.grid, p.smem, s);
     }
     if (p.packed)
         return p.M <= 1 ? launch_one<true, 1>(p.P, p.grid, p.smem, s)
@@ -1927,9 +2041,9 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
                              size_t ws_bytes) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BC_ERR_CUDA;
-    const bool xc = chunk_mode(M, packed);
+    const bool xc = chunk_mode(M, packed, bits);
     if (xc) {
-        const size_t need = gemv_stream_workspace_bytes(jobs, count, M, packed);
+        const size_t need = gemv_stream_workspace_bytes(jobs, count, M, packed, bits);
         if (!workspace || ws_bytes < need) return BC_ERR_WORKSPACE;
     }
     thread_local std::vector<std::unique_ptr<StreamPlan>> plans;
@@ -1965,7 +2079,7 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
             const int MT = chunk_mt(M);
             std::vector<size_t> off;
             std::vector<int> first;
-            xdig_layout(jobs + b0, n, M, &off, &first);
+            xdig_layout(jobs + b0, n, M, packed, &off, &first);
             uint8_t *ws = reinterpret_cast<uint8_t *>(
                 (reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255));
             for (int i = 0; i < n; ++i) P.jobs[i].x = reinterpret_cast<const float *>(ws + off[i]);
@@ -1978,14 +2092,14 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
                 X.t[q].out = ws + off[first[q]];
                 X.t[q].K = (int)G0.K;
                 X.t[q].task_begin = tasks;
-                tasks += kchunks_of<true>((int)G0.K) * MT * 2;
+                tasks += kchunks_mode((int)G0.K, packed) * MT * (packed ? 2 : 1);
             }
             X.M = M;
             X.MT = MT;
             X.total = tasks;
             plan->xgrid = std::max(1, std::min((tasks + 7) / 8, 4 * di.sm_count));
             plan->ws = workspace;
-            P.xchunk_bytes = (int)chunk_bytes(M);
+            P.xchunk_bytes = (int)chunk_bytes(M, packed);
         }
         const size_t xs = xc ? 0 : xslot_bytes_for(jobs + b0, n, M, packed);
         const int grid = std::max(1, std::min({units, di.sm_count, kMaxCtas}));
@@ -2004,10 +2118,10 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
             }
             P.max_cta_jobs = most;
         }
-        const int fixed = (int)(2 * xs) + (xc ? 512 : 256) +
+        const int fixed = (int)(2 * xs) +
+                          (xc ? 512 + tcd::kXSlots * (int)chunk_stride(M, packed) : 256) +
                           P.max_cta_jobs * (int)sizeof(StreamJob) + 1024;
-        const int per_stage = kStageBytes + (packed ? kSzBytes : 0) +
-                              (xc ? (int)chunk_stride(M) : 0);
+        const int per_stage = kStageBytes + (packed ? kSzBytes : 0);
         int stages = (di.max_smem_optin - fixed) / per_stage;
         stages = std::min(stages, 6);
         if (stages < 2) return BC_ERR_UNSUPPORTED;

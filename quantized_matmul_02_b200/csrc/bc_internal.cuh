@@ -56,14 +56,15 @@ struct GemvJob {             // one matrix of a launch
     int64_t N, K;
     int64_t group;           // 64 or K
 };
-// Streaming GEMV (bc_gemv_stream.cu): M <= 4 (M <= 16 for packed codes),
-// bulk-copy ring, int8 tensor-core products.  Used for launches large
-// enough to fill the GPU.
-bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed,
+// Streaming decode kernels (bc_gemv_stream.cu): M <= 4 on the mma.sync
+// streaming kernel; M = 5..16 on the tcgen05 decode kernel (packed, or
+// runtime RTN at 2..8 bits).  Used for launches large enough to fill the GPU.
+bool gemv_stream_supported(const GemvJob *jobs, int count, int M, bool packed, int bits,
                            int max_smem);
-// Workspace the streaming kernel needs: the activation digits of packed
-// launches with M > 4 (one copy per distinct non-null x; 0 otherwise).
-size_t gemv_stream_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed);
+// Workspace the streaming kernels need: the activation pieces of launches
+// with M > 4 (one copy per distinct non-null x; 0 otherwise).
+size_t gemv_stream_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed,
+                                   int bits);
 // early_start: programmatic dependent launch (weights known not to be
 // written by pending work; x / y accesses wait for the previous kernel).
 bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,

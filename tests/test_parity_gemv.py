@@ -392,3 +392,39 @@ def test_chunked_activation_workspace(cuda_lib):
         ref = oracle.matmul_q(xk[W.shape[1]], W, 4, 64, "packed")
         assert_close(host(items[i][4]), ref["y"], ref["A"], TOL_FP32, f"matrix {i}")
     assert cuda_lib.device_timeouts() == 0
+
+
+@pytest.mark.parametrize("bits,M", [(3, 16), (5, 8), (8, 11)])
+def test_tc_runtime_ties_take_exact_path(cuda_lib, bits, M):
+    """The tensor-core decode kernel (runtime RTN, 5..16 x rows) on weights
+    with exact half-way points: its transform warps must take the exact
+    quotient for these, like the other decode kernels.  A grouped launch of
+    copies of one grid-valued matrix, large enough for the streaming path."""
+    rng = np.random.default_rng(140 + bits)
+    L = (1 << bits) - 1
+    N, K = 512, 512
+    G = K // 64
+    e = rng.integers(4, 10, size=(N, G))
+    z = rng.integers(1, L, size=(N, G))
+    h = rng.integers(0, L, size=(N, K)) + 0.5 * rng.integers(0, 2, size=(N, K))
+    h[:, 0::64] = 0
+    h[:, 1::64] = L
+    w = (h - np.repeat(z, 64, axis=1)) * np.repeat(np.ldexp(1.0, -e), 64, axis=1)
+    W = w.astype(np.float16)
+    assert np.array_equal(W.astype(np.float64), w)
+    x = wl.activation(14, bits, "x", M, K)
+    xd, Wd = dev(x), dev(W)
+    s, zz = cuda_lib.group_params(Wd, bits, 64, torch.float32)
+    items = [(xd, Wd, s, zz, torch.full((M, N), float("nan"), device="cuda"))
+             for _ in range(24)]
+    cuda_lib.matmul_q_batched(cuda_lib.make_descs(items), M, bits, 64,
+                              cuda_lib.BC_MODE_RUNTIME)
+    torch.cuda.synchronize()
+    ref = oracle.matmul_q(x, W, bits, 64, "runtime")
+    for i in (0, 23):
+        assert_close(host(items[i][4]), ref["y"], ref["A"], TOL_FP32, f"ties bits={bits} #{i}")
+    assert cuda_lib.device_timeouts() == 0
+
+
+def test_batched_qwen3_8b_one_layer_m16_runtime(cuda_lib):
+    _layer_set_case(cuda_lib, "qwen3-8b", 1, 4, "runtime", 3, 64, M=16)
