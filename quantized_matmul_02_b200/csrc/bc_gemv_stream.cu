@@ -1424,12 +1424,12 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
         for (int s = 0; s < S; ++s) {
             // loader, plus every lane of the two scale/zero stagers (packed)
             mbar_init(smem_u32(&full[s]), PACKED ? 1 + 2 * 32 : 1);
-            // transform warps (one arrival each), epilogue threads
-            mbar_init(smem_u32(&empty[s]), tcd::kTrWarps + tcd::kEpWarps * 32);
+            // one arrival per transform and epilogue warp
+            mbar_init(smem_u32(&empty[s]), tcd::kTrWarps + tcd::kEpWarps);
         }
         for (int b = 0; b < tcd::kXSlots; ++b) {
             mbar_init(smem_u32(&xfull[b]), 1);
-            mbar_init(smem_u32(&xempty[b]), 1 + tcd::kEpWarps * 32);   // MMAs + epilogue threads
+            mbar_init(smem_u32(&xempty[b]), 1 + tcd::kEpWarps);   // MMAs + epilogue warps
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&afull[b]), tcd::kTrWarps);
@@ -1723,10 +1723,11 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
                         }
                     }
                     if (!ok) break;
-                    // every lane releases the slots after its own reads (an
-                    // arrive orders the arriving thread's loads only)
-                    mbar_arrive(smem_u32(&empty[s]));            // scales read
-                    mbar_arrive(smem_u32(&xempty[xs]));          // X~ read
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(smem_u32(&empty[s]));        // scales read
+                        mbar_arrive(smem_u32(&xempty[xs]));      // X~ read
+                    }
                     if (kc + 1 == kch) {
 #pragma unroll
                         for (int i = 0; i < MH; ++i) {
