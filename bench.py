@@ -231,7 +231,15 @@ def parse_args(argv=None):
                     help="weight copies rotated between steps (0 = enough to "
                          "exceed 4x the L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args(argv)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="run only the first N layers of the workload (a smaller "
+                         "case of the same kernels, e.g. for a profiler capture)")
+    args = ap.parse_args(argv)
+    if args.layers:
+        w = list(WORKLOADS[args.workload])
+        w[1] = min(w[1], args.layers)
+        WORKLOADS[args.workload] = tuple(w)
+    return args
 
 
 # ---------------------------------------------------------------------------
