@@ -87,8 +87,8 @@ typedef enum bc_mode {
 
 /*
  * bc_group_params -- per-group scale/zero precompute (BITCRUSH BC-06,
- * "Under the hood": the per-group scale/zero precompute kernel; a lever
- * move reruns it once, then decoding uses one uniform).
+ * "Under the hood": the per-group scale/zero precompute kernel; a change
+ * of bit width reruns it once, then decoding only passes the new bits).
  *   W          fp16 [N][K], device
  *   bits       2..8
  *   group      64, or K / 0 for per-channel
@@ -140,8 +140,11 @@ BC_API bc_status bc_pack_int4(const void *W, const void *scales_f16,
  *   workspace    device scratch of at least bc_workspace_size() bytes
  *                (may be NULL when that size is 0); its contents on entry
  *                do not matter; overlapping calls must not share it
- * Decode shapes (M < 64, fp32 x) use the fused dequant GEMV; M >= 64 with
- * bf16 x uses the tcgen05 tensor-core GEMM.
+ * Decode shapes (M < 64, fp32 x) use the fused dequant GEMV: launches that
+ * can fill the GPU run the streaming decode kernels (M <= 4 on the int8
+ * tensor cores; M = 5..16 on the tcgen05 decode kernel, packed or runtime at
+ * 2..8 bits, whose workspace holds the split activations of each x); M >= 64
+ * with bf16 x uses the tcgen05 tensor-core GEMM.
  */
 BC_API bc_status bc_matmul_q(const void *x, bc_dtype x_dtype, const void *W_or_packed,
                       const void *scales, const void *zeros, int64_t M,
@@ -187,7 +190,7 @@ BC_API bc_status bc_matmul_q_batched(const bc_matmul_desc *descs, int count,
  * that name the same non-null x (and K) share scratch, and a size computed
  * with x = NULL holds for any x pointers of a later call with the same N, K.
  * Returns 0 for arguments the call would reject, and for calls that need no
- * scratch (bf16 x, and the decode kernel for fp16 weights or M <= 4).
+ * scratch (bf16 x, and the streaming decode kernel at M <= 4).
  */
 BC_API size_t bc_workspace_size_batched(const bc_matmul_desc *descs, int count,
                                  int64_t M, bc_mode mode, bc_dtype x_dtype);
@@ -226,7 +229,8 @@ BC_API bc_status bc_matmul_q_batched_ex(const bc_matmul_desc *descs, int count,
  * deployment variant of the same computation.
  *   Arguments mean what they mean for bc_matmul_q with x_dtype = BC_F32.
  *   Scratch: instead of a caller workspace, the split-K partial sums and
- *   tickets live in a fixed 4 MiB array inside the library (a __device__
+ *   tickets (and the split activations of the tcgen05 decode kernel) live
+ *   in a fixed 4 MiB array inside the library (a __device__
  *   object that every GPU loading the library holds until process exit).
  *   Shapes whose scratch would exceed it are rejected with
  *   BC_ERR_WORKSPACE before anything is enqueued.  The call allocates

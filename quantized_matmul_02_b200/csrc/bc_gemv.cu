@@ -4,8 +4,8 @@
 // stream in (BITCRUSH BC-06, "Under the hood": matmul_q computes the
 // group-wise affine RTN inline as weights are read; Enargeia, "Four bits per
 // weight": int4 codes unpacked in registers and never written back).
-// Decode "reads every weight in the model to write one word" (Enargeia), so
-// the kernel is an HBM stream: 16-byte vector loads that skip L1, one
+// A decode step touches every weight once for one output row (Enargeia's
+// point about decode), so the kernel is an HBM stream: 16-byte vector loads that skip L1, one
 // 16-byte chunk per lane per step (8 fp16 weights, or 32 int4 codes),
 // `lpr` lanes per weight row, 8 warps per CTA, a persistent grid over a
 // work list that spans every matrix of a grouped launch (Enargeia, "One

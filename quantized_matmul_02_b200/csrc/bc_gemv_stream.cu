@@ -1,7 +1,7 @@
 // bc_gemv_stream.cu -- streaming fused dequant GEMV for decode (M <= 4).
 //
-// Decode "reads every weight in the model to write one word" (Enargeia):
-// the matmul is one pass over HBM.  The kernel is a TMA pipeline that keeps
+// A decode step touches every weight once to produce a single output row
+// (Enargeia makes this point about decode): the matmul is one pass over HBM.  The kernel is a TMA pipeline that keeps
 // ~130-200 KB per SM in flight, with the arithmetic per weight cut down until
 // the stream, not the issue slots, sets the pace.
 //
@@ -344,13 +344,13 @@ __device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
 // One launch before the tensor-core kernel prepares every distinct x of the
 // call per stage chunk (see xpieces_kernel); tasks are numbered per x from
 // task_begin.
-struct XdigTask {
+struct XpreTask {
     const float *x;
     uint8_t *out;
     int K, task_begin;
 };
-struct XdigParams {
-    XdigTask t[kMaxJobs];
+struct XpreParams {
+    XpreTask t[kMaxJobs];
     int count, M, MT, total;
 };
 // One x row of a runtime-mode slot: fp32, zero past K.
@@ -1274,7 +1274,7 @@ template <int MT> __host__ __device__ __forceinline__ int brow_off(int gl, int m
 // up to 4 groups of 64 k, 8 lanes per group, 8 k per lane (one 16-byte piece
 // of a B row).  Rows m >= M and groups past K/64 are zero.
 template <bool PACKED, int MT>
-__global__ void __launch_bounds__(256) xpieces_kernel(const __grid_constant__ XdigParams P) {
+__global__ void __launch_bounds__(256) xpieces_kernel(const __grid_constant__ XpreParams P) {
     using C = tcd::Chunk<PACKED, MT>;
     constexpr int Q = (C::kGroups + 3) / 4;          // quads per chunk
     const int lane = threadIdx.x & 31, j = lane & 7;
@@ -1285,7 +1285,7 @@ __global__ void __launch_bounds__(256) xpieces_kernel(const __grid_constant__ Xd
             const int mid = (lo + hi + 1) >> 1;
             if (P.t[mid].task_begin <= task) lo = mid; else hi = mid - 1;
         }
-        const XdigTask &T = P.t[lo];
+        const XpreTask &T = P.t[lo];
         int r = task - T.task_begin;
         const int quad = r % Q;
         r /= Q;
@@ -1880,10 +1880,10 @@ int kchunks_mode(int K, bool packed) {
     return packed ? kchunks_of<true>(K) : kchunks_of<false>(K);
 }
 
-// Workspace layout of the chunk-mode activation digits: each distinct
+// Workspace layout of the chunk-mode activation pieces: each distinct
 // (x, K) of the launch once, in job order; off[i] is job i's offset.  A null
 // x (a size query without pointers) is never shared, which bounds any call.
-size_t xdig_layout(const GemvJob *jobs, int count, int M, bool packed,
+size_t xpieces_layout(const GemvJob *jobs, int count, int M, bool packed,
                    std::vector<size_t> *off, std::vector<int> *first) {
     const size_t mtb = chunk_bytes(M, packed);
     size_t total = 0;
@@ -1983,7 +1983,7 @@ size_t gemv_stream_workspace_bytes(const GemvJob *jobs, int count, int M, bool p
     // launches above kMaxJobs matrices reuse the space batch by batch
     size_t worst = 0;
     for (int b = 0; b < count; b += kMaxJobs)
-        worst = std::max(worst, xdig_layout(jobs + b, std::min(kMaxJobs, count - b), M, packed,
+        worst = std::max(worst, xpieces_layout(jobs + b, std::min(kMaxJobs, count - b), M, packed,
                                             nullptr, nullptr));
     return worst ? worst + 256 : 0;
 }
@@ -1999,7 +1999,7 @@ struct StreamPlan {
     const void *ws = nullptr;    // chunk mode: the workspace the chunk pointers point into
     StreamParams P;
     int grid = 0, smem = 0;
-    XdigParams X;                // chunk mode: the pre-pass over the distinct x
+    XpreParams X;                // chunk mode: the pre-pass over the distinct x
     int xgrid = 0;
 };
 constexpr int kPlanCache = 4;
@@ -2080,11 +2080,11 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
             const int MT = chunk_mt(M);
             std::vector<size_t> off;
             std::vector<int> first;
-            xdig_layout(jobs + b0, n, M, packed, &off, &first);
+            xpieces_layout(jobs + b0, n, M, packed, &off, &first);
             uint8_t *ws = reinterpret_cast<uint8_t *>(
                 (reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255));
             for (int i = 0; i < n; ++i) P.jobs[i].x = reinterpret_cast<const float *>(ws + off[i]);
-            XdigParams &X = plan->X;
+            XpreParams &X = plan->X;
             int tasks = 0;
             X.count = (int)first.size();
             for (int q = 0; q < X.count; ++q) {
