@@ -428,3 +428,36 @@ def test_tc_runtime_ties_take_exact_path(cuda_lib, bits, M):
 
 def test_batched_qwen3_8b_one_layer_m16_runtime(cuda_lib):
     _layer_set_case(cuda_lib, "qwen3-8b", 1, 4, "runtime", 3, 64, M=16)
+
+
+@pytest.mark.parametrize("mode,bits", [("packed", 4), ("runtime", 5)])
+def test_tc_decode_more_matrices_than_one_launch(cuda_lib, mode, bits):
+    """More matrices than one launch of the tensor-core decode kernel takes
+    (168): the call runs in batches that reuse the activation workspace one
+    after the other; every matrix, first and last batch, must be right."""
+    rng = np.random.default_rng(160 + bits)
+    M, count = 8, 200
+    shapes = [(256, 512), (128, 448), (384, 256)]
+    xs = {K: wl.activation(90, K, "x", M, K) for _, K in shapes}
+    xd = {K: dev(v) for K, v in xs.items()}
+    items, Ws = [], []
+    for i in range(count):
+        N, K = shapes[i % len(shapes)]
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+        Wd = dev(W)
+        if mode == "packed":
+            s, z = cuda_lib.group_params(Wd, 4, 64, torch.float16)
+            Wk = cuda_lib.pack_int4(Wd, s, z)
+        else:
+            s, z = cuda_lib.group_params(Wd, bits, 64, torch.float32)
+            Wk = Wd
+        items.append((xd[K], Wk, s, z, torch.full((M, N), float("nan"), device="cuda")))
+        Ws.append(W)
+    mid = cuda_lib.BC_MODE_PACKED_INT4 if mode == "packed" else cuda_lib.BC_MODE_RUNTIME
+    cuda_lib.matmul_q_batched(cuda_lib.make_descs(items), M, bits, 64, mid)
+    torch.cuda.synchronize()
+    for i in (0, 1, 2, 166, 167, 168, 169, 198, 199):
+        W = Ws[i]
+        ref = oracle.matmul_q(xs[W.shape[1]], W, bits, 64, mode)
+        assert_close(host(items[i][4]), ref["y"], ref["A"], TOL_FP32, f"matrix {i}")
+    assert cuda_lib.device_timeouts() == 0
