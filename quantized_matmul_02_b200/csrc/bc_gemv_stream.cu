@@ -1,4 +1,6 @@
-// bc_gemv_stream.cu -- streaming fused dequant GEMV for decode (M <= 4).
+// bc_gemv_stream.cu -- streaming decode kernels for launches that fill the
+// GPU: gemv_stream_kernel (M <= 4, int8 mma.sync) described here, and the
+// tcgen05 decode kernel for M = 5..16 further below (gemv_tc_kernel).
 //
 // A decode step touches every weight once to produce a single output row
 // (Enargeia makes this point about decode): the matmul is one pass over HBM.  The kernel is a TMA pipeline that keeps
