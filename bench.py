@@ -118,8 +118,8 @@ def launches_per_step(name: str, count: int) -> int:
     return -(-M // 16) * -(-count // 368)
 
 
-KERNEL_SOURCES = {"decode": ("bc_gemv_stream.cu", "bc_gemv.cu", "bc_internal.cuh"),
-                  "prefill": ("bc_gemm_sm100.cu", "bc_internal.cuh")}
+KERNEL_SOURCES = {"decode": ("bc_gemv_stream.cu", "bc_gemv.cu", "bc_internal.cuh", "bc_tc.cuh"),
+                  "prefill": ("bc_gemm_sm100.cu", "bc_internal.cuh", "bc_tc.cuh")}
 
 
 def kernel_source_digest(kind: str = "decode") -> str:
