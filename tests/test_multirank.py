@@ -92,3 +92,32 @@ def test_traffic_needs_matching_digest(tmp_path, monkeypatch):
     assert bench.recorded_traffic("w") == 123
     (csrc / "bc_gemv_stream.cu").write_text("changed")
     assert bench.recorded_traffic("w") is None
+
+
+def test_decode_kernel_choice_and_launch_counts():
+    """The bench's claim of kernels per step mirrors the library's dispatch:
+    the streaming kernel for M <= 4 (168 matrices per launch), the tcgen05
+    decode kernel plus its pre-pass for M = 5..16 (packed, or runtime below
+    16 bits), the tensor-core GEMM for prefill (80 matrices per launch)."""
+    assert bench.decode_kernel("qwen2.5-0.5b-int4-decode") == "stream"
+    assert bench.decode_kernel("qwen3-8b-int4-decode-m16") == "tc"
+    assert bench.decode_kernel("qwen3-8b-rtn3-decode-m16") == "tc"
+    assert bench.launches_per_step("qwen2.5-0.5b-int4-decode", 168) == 1
+    assert bench.launches_per_step("qwen3-8b-int4-decode", 252) == 2
+    assert bench.launches_per_step("qwen3-8b-int4-decode-m16", 252) == 4
+    assert bench.launches_per_step("qwen2.5-0.5b-int4-prefill-m2048", 168) == 3
+
+
+def test_traffic_digest_covers_the_tcgen05_header(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    os.makedirs(tmp_path / "profiles")
+    csrc = tmp_path / "quantized_matmul_02_b200" / "csrc"
+    os.makedirs(csrc)
+    for f in ("bc_gemv.cu", "bc_gemv_stream.cu", "bc_internal.cuh", "bc_tc.cuh"):
+        (csrc / f).write_text(f)
+    d = bench.kernel_source_digest()
+    (tmp_path / "profiles" / "traffic_w.txt").write_text(
+        f"source_digest: {d}\ndram_bytes_per_launch: 7\n")
+    assert bench.recorded_traffic("w") == 7
+    (csrc / "bc_tc.cuh").write_text("changed")
+    assert bench.recorded_traffic("w") is None
