@@ -2,6 +2,9 @@
 codes and packed bytes must be bit-exact (BITCRUSH BC-06 "Under the hood":
 per-group scale/zero precompute and RTN codes; Enargeia "Four bits per
 weight": int4 packing)."""
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -30,13 +33,21 @@ def _edge_matrix(seed=5):
     rows.append(rng.standard_normal(K) * 300.0)                    # large range
     rows.append(np.concatenate([np.full(64, -2.0 ** -24), np.full(64, 65504.0),
                                 rng.standard_normal(64)]))
+    # group 0: fp16 scale below 2^-25, floored to 2^-24; group 1: single-sign
+    # group near 1000 whose zero (|z| > 2048) is rounded to fp16
+    r = np.zeros(K)
+    r[0:4] = np.array([-2, 5, 0, -1]) * 2.0 ** -24
+    r[64:128] = 1000.0 + 0.5 * rng.integers(0, 3, 64)
+    r[64], r[65] = 1000.0, 1001.0
+    r[128:] = rng.standard_normal(64) * 0.02
+    rows.append(r)
     for _ in range(29):
-        rows.append(rng.standard_normal(K) * 0.02)                 # 37 rows total
+        rows.append(rng.standard_normal(K) * 0.02)                 # 38 rows total
     return np.array(rows).astype(np.float16)
 
 
 CASES = [("cfg1_1024", lambda: wl.weight(0, 0, "single", 1024, 1024, 0.02)),
-         ("edges_37x192", _edge_matrix),
+         ("edges_38x192", _edge_matrix),
          ("tiny_1x64", lambda: wl.weight(9, 0, "single", 64, 1, 0.02))]
 
 
@@ -82,3 +93,32 @@ def test_pack_full_qwen25_layer(cuda_lib):
         Wd = dev(W)
         s, z = cuda_lib.group_params(Wd, 4, 64, torch.float16)
         np.testing.assert_array_equal(host(cuda_lib.pack_int4(Wd, s, z)), p_ref)
+
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "rtn_worked_groups.json")
+SINGLE = [c for c in json.load(open(GOLDEN))["cases"] if "w" in c]
+
+
+@pytest.mark.parametrize("case", SINGLE, ids=lambda c: c["name"])
+def test_golden_groups_on_gpu(cuda_lib, case):
+    """The hand-worked groups straight through the GPU kernels (not via the
+    oracle): stored scale and zero, codes and packed bytes as derived by
+    hand from the definitions."""
+    K = case["K"]
+    w = np.full(K, case["fill"], np.float64)
+    w[:len(case["w"])] = case["w"]
+    Wd = dev(w.astype(np.float16)[None, :])
+    packed = case["mode"] == "packed"
+    s, z = cuda_lib.group_params(Wd, case["bits"], case["group"],
+                                 torch.float16 if packed else torch.float32)
+    assert host(s).astype(np.float64).ravel().tolist() == case["scales"]
+    assert host(z).astype(np.float64).ravel().tolist() == case["zeros"]
+    q = host(cuda_lib.quantize_codes(Wd, s, z, case["bits"], case["group"])).ravel()
+    exp_q = np.full(K, case["codes_fill"])
+    exp_q[:len(case["codes"])] = case["codes"]
+    assert q.tolist() == exp_q.tolist()
+    if packed:
+        p = host(cuda_lib.pack_int4(Wd, s, z)).ravel()
+        exp_p = np.full(K // 2, case["packed_fill"])
+        exp_p[:len(case["packed"])] = case["packed"]
+        assert p.tolist() == exp_p.tolist()
