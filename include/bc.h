@@ -243,6 +243,10 @@ BC_API bc_status bc_matmul_q_batched_ex(const bc_matmul_desc *descs, int count,
  *   call).  Calls that can overlap on the GPU -- on different streams, or
  *   from different threads without ordering -- race on the array and give
  *   wrong results; serialise them (e.g. one stream).
+ *   Device reset: the looked-up address belongs to the device's context at
+ *   the time of the first call; after cudaDeviceReset on that device this
+ *   entry point (like the library's other cached per-device state, such as
+ *   kernel shared-memory attributes) is not valid in this process.
  */
 BC_API bc_status bc_matmul_q_noalloc(const void *x, const void *W_or_packed,
                                      const void *scales, const void *zeros,

@@ -226,6 +226,15 @@ def matmul_q_noalloc(x: torch.Tensor, W: torch.Tensor,
     `y` must be supplied; nothing is allocated by this call."""
     M, K = x.shape
     N = W.shape[0]
+    # The C call reads x as fp32 [M][K] and writes y as fp32 [M][N]: anything
+    # else would be read or written out of bounds, so refuse it here.
+    if x.dtype != torch.float32 or y.dtype != torch.float32:
+        raise ValueError("matmul_q_noalloc: x and y must be float32")
+    if tuple(y.shape) != (M, N):
+        raise ValueError(f"matmul_q_noalloc: y must have shape {(M, N)}")
+    devs = {t.device for t in (x, W, y, scales, zeros) if t is not None}
+    if len(devs) != 1 or not next(iter(devs)).type == "cuda":
+        raise ValueError("matmul_q_noalloc: all tensors must be on one CUDA device")
     _check(lib.bc_matmul_q_noalloc(_ptr(x), _ptr(W), _ptr(scales), _ptr(zeros),
                                    M, N, K, bits, group, mode, _ptr(y),
                                    _stream(stream)), "bc_matmul_q_noalloc")
