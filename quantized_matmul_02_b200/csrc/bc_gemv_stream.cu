@@ -56,6 +56,7 @@
 // so a single lane arriving for its warp could let the producer overwrite a
 // slot while other lanes' loads are still in flight.
 #include "bc_internal.cuh"
+#include "bc_rtn.cuh"
 #include "bc_tc.cuh"
 
 #include <cuda.h>
@@ -70,6 +71,9 @@
 namespace bc {
 
 __device__ unsigned int g_gemv_timeouts = 0;
+// Limit of the pipeline waits, in clock64 cycles (bc_set_wait_limit);
+// the drains after an abort keep the fixed ~2 s limit.
+__device__ long long g_gemv_wait_limit = 4000000000LL;
 
 namespace {
 
@@ -114,6 +118,7 @@ struct __align__(64) StreamParams {
     int xslot_bytes, stages, max_cta_jobs;
     int early;                    // launched as a programmatic dependent launch
     int xchunk_bytes;             // tensor-core kernel: bytes of one stage's x chunk
+    int range;                    // runtime mode: (scale, zero) from stored ranges
 };
 static_assert(sizeof(StreamParams) <= 32000, "kernel parameter space");
 
@@ -129,12 +134,22 @@ template <bool PACKED> __host__ __device__ __forceinline__ int kpad_of(int K) {
 }
 // Packed x row: digit words [digit d][lane t][unit U][parity] with a row
 // stride of dig_rs words (= 4 mod 32, so the 8 rows a quarter-warp reads sit
-// in distinct banks), then [parity][group] float2 (f, X~) tables.
+// in distinct banks), then [parity][group] float2 (f, T) tables, then per
+// group the values of its side pair (float2: even k, odd k) and one side byte
+// (0: none; 1 + p: exactly one side pair, pair p = k 64g + 2p, 2p + 1;
+// 0xFF: more than one), eight bytes to a stage chunk.
 __host__ __device__ __forceinline__ int dig_rs(int kchunks) { return 32 * kchunks + 4; }
-// Bytes of one x row in a slot.  Runtime: x[kp] f32.
+__host__ __device__ __forceinline__ int side_val_off(int kchunks) {
+    return 64 * dig_rs(kchunks) + 16 * (8 * kchunks);
+}
+__host__ __device__ __forceinline__ int side_flag_off(int kchunks) {
+    return side_val_off(kchunks) + 8 * (8 * kchunks);
+}
+constexpr uint8_t kSideMany = 0xFF;
+// Bytes of one x row in a slot (a multiple of 16).  Runtime: x[kp] f32.
 template <bool PACKED> __host__ __device__ __forceinline__ int xrow_bytes(int K) {
     const int kc = kchunks_of<PACKED>(K);
-    return PACKED ? 64 * dig_rs(kc) + 16 * (8 * kc) : 4 * kpad_of<false>(K);
+    return PACKED ? (side_flag_off(kc) + 8 * kc + 15) / 16 * 16 : 4 * kpad_of<false>(K);
 }
 
 // ---- PTX helpers -------------------------------------------------------------
@@ -164,10 +179,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int *abort_flag) {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
+    const long long limit = *(volatile long long *)&g_gemv_wait_limit;
     while (true) {
         if (mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             if (atomicExch((int *)abort_flag, 1) == 0)
                 atomicAdd(&g_gemv_timeouts, 1u);
             return false;
@@ -237,6 +253,18 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t v) {
     *reinterpret_cast<uint32_t *>(&h) = v;
     return __half22float2(h);
 }
+// Two integer-valued fp16 (zero points) as ints.
+__device__ __forceinline__ int2 half2_bits_to_int2(uint32_t v) {
+    __half2 h;
+    *reinterpret_cast<uint32_t *>(&h) = v;
+    return make_int2(__half2int_rn(__low2half(h)), __half2int_rn(__high2half(h)));
+}
+// (float)(v - z t), the difference exact: in int32 when |z| <= 45 (|v| < 2^30,
+// |t| < 2^25), else in int64 (single-sign groups, whose zero lies far out).
+__device__ __forceinline__ float exact_dot(int v, int z, int t) {
+    if (abs(z) <= 45) return (float)(v - z * t);
+    return (float)((long long)v - (long long)z * (long long)t);
+}
 
 // Units are visited in increasing order, so the owning job only moves forward.
 __device__ __forceinline__ int next_job(const StreamJob *jobs, int count, int j, int unit) {
@@ -263,37 +291,91 @@ __device__ __forceinline__ void transpose4(const uint32_t (&w)[4], uint32_t (&o)
 // Digits of one 64-group held by 8 lanes (lane j has k = 8j .. 8j+7 of it):
 // the digit words of this lane's even-k values (te) and odd-k slots (to,
 // carrying X_odd - X_even), byte i of each at k = 8j + 2i; and, on every
-// lane of the 8, the group's f = 2^(E-30) and X~ = f * sum(X_e + 16 X_o).
+// lane of the 8, the group's f = 2^(E-30), its zero-point sums T01 / T23
+// and the mask of its side elements.
+//
+// Side elements.  The integer grid of a group is 2^(E-30) at even k and
+// 2^(E-26) at odd k, so an element keeps a relative error of at most 2^-14
+// only if |x| >= 2^(E-17) (even) or 2^(E-13) (odd).  Nonzero elements below
+// those bounds are left out of the digits (staged as 0) and flagged; the
+// consumers add their products exactly, in fp32.  The values of a group's
+// side pair are kept beside the digits (a group holds one side pair or none
+// on almost every input; groups with more take a slower exact path that
+// reads x from global memory).
+// When the odd element of a (2i, 2i+1) pair is a side element, its even
+// partner is one too: the odd slot then carries no part of the even value,
+// which keeps every digit pair's sum below free of carries from elements
+// the integers do not hold (see the epilogue).
+//
+// Zero-point sums.  With A = z in place of the codes (17 z in the raw-byte
+// even slot, 16 z in the odd slot) the MMA would give, per digit d,
+// T_d = sum over pairs (17 d(X_e) + 16 d(X_o - X_e)); the consumer forms
+// C_d - z T_d, which is exactly sum (q - z) d(...).  Per digit pair
+// (0,1) and (2,3): T01 = T_0 + 256 T_1, T23 = T_2 + 256 T_3, |T| < 2^25.
+// max|x| < 2^E for a group with largest magnitude amax; E >= -96 keeps
+// every scale below a normal float.
+__device__ __forceinline__ int group_exponent(float amax) {
+    const int E = amax > 0.0f ? (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126 : 0;
+    return max(E, -96);
+}
+// Side elements of the pair (ve, vo) by the staging rules of a group with
+// grid exponent E (as group_digits decides them).
+__device__ __forceinline__ void side_pair(float ve, float vo, int E, bool &se, bool &so) {
+    const float thr_e = __uint_as_float((uint32_t)(127 + E - 17) << 23);
+    const float thr_o = __uint_as_float((uint32_t)(127 + E - 13) << 23);
+    so = vo != 0.0f && fabsf(vo) < thr_o;
+    se = ve != 0.0f && (so || fabsf(ve) < thr_e);
+}
+__device__ __forceinline__ int lo16(int v) {          // d0 + 256 d1 of digits4(v)
+    return (int)(((uint32_t)v + 0x8080u) & 0xFFFFu) - 0x8080;
+}
 __device__ __forceinline__ void group_digits(const float (&v)[8], uint32_t (&te)[4],
-                                             uint32_t (&to)[4], float &f, float &xt) {
+                                             uint32_t (&to)[4], float &f, int &t01,
+                                             int &t23, uint32_t &sidepairs, int &Eg) {
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-    // max|x| < 2^E; E >= -96 keeps every scale below a normal float
-    int E = amax > 0.0f ? (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126 : 0;
-    E = max(E, -96);
+    const int E = group_exponent(amax);
     const float sc_e = __uint_as_float((uint32_t)(127 + kXP + 4 - E) << 23);
     const float sc_o = __uint_as_float((uint32_t)(127 + kXP - E) << 23);
     uint32_t de[4], dq[4];
-    long long sum = 0;
+    uint32_t lm = 0;
+    int s01 = 0, s23 = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int xe = __float2int_rn(v[2 * i] * sc_e);      // |xe| <= 2^30
-        const int xo = __float2int_rn(v[2 * i + 1] * sc_o);  // |xo| <= 2^26
-        sum += (long long)xe + 16ll * xo;
+        const float ve = v[2 * i], vo = v[2 * i + 1];
+        bool se, so;
+        side_pair(ve, vo, E, se, so);
+        lm |= ((se || so) ? 1u : 0u) << i;
+        const int xe = se ? 0 : __float2int_rn(ve * sc_e);   // |xe| <= 2^30
+        const int xo = so ? 0 : __float2int_rn(vo * sc_o);   // |xo| <= 2^26
+        const int dv = xo - xe;       // odd slots carry X_odd - X_even (raw-byte A)
         de[i] = digits4(xe);
-        dq[i] = digits4(xo - xe);     // odd slots carry X_odd - X_even (raw-byte A)
+        dq[i] = digits4(dv);
+        const int le = lo16(xe), ld = lo16(dv);
+        s01 += 17 * le + 16 * ld;
+        s23 += 17 * ((xe - le) >> 16) + 16 * ((dv - ld) >> 16);
     }
     transpose4(de, te);
     transpose4(dq, to);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+    s01 += __shfl_xor_sync(0xffffffffu, s01, 1);
+    s01 += __shfl_xor_sync(0xffffffffu, s01, 2);
+    s01 += __shfl_xor_sync(0xffffffffu, s01, 4);
+    s23 += __shfl_xor_sync(0xffffffffu, s23, 1);
+    s23 += __shfl_xor_sync(0xffffffffu, s23, 2);
+    s23 += __shfl_xor_sync(0xffffffffu, s23, 4);
+    t01 = s01;
+    t23 = s23;
+    // side pairs of the group: bit 4j + i <-> pair (8j + 2i, 8j + 2i + 1)
+    sidepairs = lm << (4 * (threadIdx.x & 7));
+    sidepairs |= __shfl_xor_sync(0xffffffffu, sidepairs, 1);
+    sidepairs |= __shfl_xor_sync(0xffffffffu, sidepairs, 2);
+    sidepairs |= __shfl_xor_sync(0xffffffffu, sidepairs, 4);
     f = __uint_as_float((uint32_t)(127 + E - kXP - 4) << 23);
-    xt = (float)((double)f * (double)sum);
+    Eg = E;
 }
 
 // One x row of a packed-mode slot, by warp `widx` of `nw` working together.
@@ -327,16 +409,37 @@ __device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
             const float v[8] = {va[b][0].x, va[b][0].y, va[b][0].z, va[b][0].w,
                                 va[b][1].x, va[b][1].y, va[b][1].z, va[b][1].w};
             uint32_t te[4], to[4];
-            float f, xt;
-            group_digits(v, te, to, f, xt);
+            float f;
+            int t01, t23;
+            uint32_t sp;
+            int E;
+            group_digits(v, te, to, f, t01, t23, sp, E);
             const int U = 2 * g + (j >> 2), tt = j & 3;
 #pragma unroll
             for (int d = 0; d < 4; ++d)
                 *reinterpret_cast<uint2 *>(dig + (d * 4 + tt) * rs + 2 * U) =
                     make_uint2(te[d], to[d]);
             if (j == 0) {
-                tab[g] = make_float2(f, xt);
-                tab[gpad + g] = make_float2(f * 65536.0f, 0.0f);
+                tab[g] = make_float2(f, __int_as_float(t01));
+                tab[gpad + g] = make_float2(f * 65536.0f, __int_as_float(t23));
+                xm[side_flag_off(kch) + g] =
+                    sp == 0 ? 0 : (__popc(sp) == 1 ? (uint8_t)(__ffs(sp)) : kSideMany);
+            }
+            if (sp != 0 && __popc(sp) == 1 && ((__ffs(sp) - 1) >> 2) == j) {
+                // the lane holding the group's one side pair stores its values
+                // (0 for a member the integers hold)
+                const int i = (__ffs(sp) - 1) & 3;
+                float ve = 0.0f, vo = 0.0f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (q == i) {
+                        ve = v[2 * q];
+                        vo = v[2 * q + 1];
+                    }
+                bool se, so;
+                side_pair(ve, vo, E, se, so);
+                reinterpret_cast<float2 *>(xm + side_val_off(kch))[g] =
+                    make_float2(se ? ve : 0.0f, so ? vo : 0.0f);
             }
         }
     }
@@ -513,6 +616,39 @@ __device__ __forceinline__ void sz_store(const StreamJob *jobs, const SzWalk &a,
 // tensor-core math and epilogue, so the wait and load latency of one stage
 // hide behind the arithmetic of the other.  A step reads the activation slot
 // only for its own stage, before the next stage may move to another slot.
+// Side products of group `sub` of a stage window (its 128-byte swizzled rows
+// start at `box`), for one weight row, with the group's scale s and zero z.
+// Fast path (info = 1 + p): the group's one side pair p, its values from the
+// x slot, both codes from one byte of the row.
+__device__ __forceinline__ float side_fast(uint32_t info, float2 vals, const uint8_t *box,
+                                           int row, int sub, float s, float z) {
+    const int byte = 32 * sub + (int)info - 1;
+    const uint32_t b = box[row * 128 + (((byte >> 4) ^ (row & 7)) << 4) + (byte & 15)];
+    return s * fmaf((float)(b >> 4) - z, vals.y, ((float)(b & 15u) - z) * vals.x);
+}
+// Slow path (more than one side pair in the group): the side elements are
+// found again from the group's x in global memory (xg = its first element)
+// by the staging rules, and their products added exactly.
+__device__ __noinline__ float side_slow(const float *__restrict__ xg, const uint8_t *box,
+                                        int row, int sub, float s, float z) {
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(xg) + i);
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+    const int E = group_exponent(amax);
+    float acc = 0.0f;
+    for (int p = 0; p < 32; ++p) {
+        const float2 v = __ldg(reinterpret_cast<const float2 *>(xg) + p);
+        bool se, so;
+        side_pair(v.x, v.y, E, se, so);
+        if (se || so) acc += side_fast((uint32_t)p + 1, make_float2(se ? v.x : 0.0f,
+                                                                    so ? v.y : 0.0f),
+                                       box, row, sub, s, z);
+    }
+    return acc;
+}
+
 struct StageA {
     uint32_t R[2][4][4];   // [window][j] ldmatrix fragments
     uint32_t s[2][2], z[2][2];   // [row ra / ra+8][window] fp16 pair (2eh, 2eh+1)
@@ -564,6 +700,41 @@ __device__ __forceinline__ void consume_packed_m1(
     auto step = [&](StageA &cur, StageA &nxt) -> bool {
         const StreamJob &J = jobs[k.jidx];
         const int kch = kchunks_of<true>(J.K);
+        {
+            // side elements of this stage's 8 groups (about one stage in ten
+            // on Gaussian activations): this lane takes groups 2eh, 2eh + 1 of
+            // each window for row ra (ep = 0) or ra + 8 (ep = 1), before the
+            // stage is released
+            const uint2 fl = *reinterpret_cast<const uint2 *>(xc.xs + side_flag_off(kch) +
+                                                               8 * k.kc);
+            if (fl.x | fl.y) {
+                const float2 *sv =
+                    reinterpret_cast<const float2 *>(xc.xs + side_val_off(kch)) + 8 * k.kc;
+                const uint8_t *st = smem + k.sidx * kStageBytes;
+                const int row = ra + 8 * ep;
+                float v = 0.0f;
+#pragma unroll
+                for (int w = 0; w < 2; ++w) {
+                    const uint32_t fw = w ? fl.y : fl.x;
+                    if (!fw) continue;
+                    const float2 s2 = half2_bits_to_float2(ep ? cur.s[1][w] : cur.s[0][w]);
+                    const float2 z2 = half2_bits_to_float2(ep ? cur.z[1][w] : cur.z[0][w]);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int sub = 2 * eh + e;
+                        const uint32_t info = (fw >> (8 * sub)) & 0xffu;
+                        if (!info) continue;
+                        const float sc = e ? s2.y : s2.x, zc = e ? z2.y : z2.x;
+                        v += info != kSideMany
+                                 ? side_fast(info, sv[4 * w + sub], st + w * kBoxBytes, row, sub,
+                                             sc, zc)
+                                 : side_slow(J.x + 512 * k.kc + 64 * (4 * w + sub),
+                                             st + w * kBoxBytes, row, sub, sc, zc);
+                    }
+                }
+                if (ep) yb += v; else ya += v;
+            }
+        }
         // stage released: the arrive's release semantics order this warp's
         // ldmatrix reads (made visible to lane 0 by the warp sync) before it
         __syncwarp();
@@ -592,17 +763,21 @@ __device__ __forceinline__ void consume_packed_m1(
                 mma_i8(C, R[0] & 0xF0F0F0F0u, R[1] & 0xF0F0F0F0u, R[2] & 0xF0F0F0F0u,
                        R[3] & 0xF0F0F0F0u, bu & m0, bu & m1);
             }
-            // digits (2ep, 2ep+1) of rows ra, ra+8 for groups 4w+2eh (A) and +1 (B)
+            // digits (2ep, 2ep+1) of rows ra, ra+8 for groups 4w+2eh (A) and +1 (B):
+            // y += s f (C - z T), the integer part exact
             const float2 sa = half2_bits_to_float2(cur.s[0][w]);
             const float2 sb = half2_bits_to_float2(cur.s[1][w]);
-            const float2 za = half2_bits_to_float2(cur.z[0][w]);
-            const float2 zb = half2_bits_to_float2(cur.z[1][w]);
-            const float vAa = (float)(CA[0] + 256 * CA[1]), vAb = (float)(CA[2] + 256 * CA[3]);
-            const float vBa = (float)(CB[0] + 256 * CB[1]), vBb = (float)(CB[2] + 256 * CB[3]);
-            ya = fmaf(sa.x, fmaf(tb.x, vAa, -za.x * tb.y), ya);
-            yb = fmaf(sb.x, fmaf(tb.x, vAb, -zb.x * tb.y), yb);
-            ya = fmaf(sa.y, fmaf(tb.z, vBa, -za.y * tb.w), ya);
-            yb = fmaf(sb.y, fmaf(tb.z, vBb, -zb.y * tb.w), yb);
+            const int2 za = half2_bits_to_int2(cur.z[0][w]);
+            const int2 zb = half2_bits_to_int2(cur.z[1][w]);
+            const int TA = __float_as_int(tb.y), TB = __float_as_int(tb.w);
+            const float rAa = exact_dot(CA[0] + 256 * CA[1], za.x, TA);
+            const float rAb = exact_dot(CA[2] + 256 * CA[3], zb.x, TA);
+            const float rBa = exact_dot(CB[0] + 256 * CB[1], za.y, TB);
+            const float rBb = exact_dot(CB[2] + 256 * CB[3], zb.y, TB);
+            ya = fmaf(sa.x * tb.x, rAa, ya);
+            yb = fmaf(sb.x * tb.x, rAb, yb);
+            ya = fmaf(sa.y * tb.z, rBa, ya);
+            yb = fmaf(sb.y * tb.z, rBb, yb);
         }
         if (n.kc == 0 || !more) {      // unit done: four lanes per row
             ya += __shfl_xor_sync(0xffffffffu, ya, 1);
@@ -680,6 +855,50 @@ __device__ __forceinline__ void consume_packed_mx(
                 zu[1][w] = *reinterpret_cast<const uint2 *>(sz + kSzBytes / 2 + 128 + 8 * w);
             }
         }
+        // side elements of the stage's groups, per x row (rows past M hold
+        // stale data and are skipped); before the stage is released
+#pragma unroll
+        for (int mp = 0; mp < MP; ++mp) {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int m = 2 * mp + h2;
+                if (m >= P.M) continue;
+                const uint8_t *xr = xb + m * mb;
+                const uint2 fl = *reinterpret_cast<const uint2 *>(xr + side_flag_off(kch) +
+                                                                   8 * k.kc);
+                if (!(fl.x | fl.y)) continue;
+                const float2 *sv =
+                    reinterpret_cast<const float2 *>(xr + side_val_off(kch)) + 8 * k.kc;
+                const uint8_t *st = smem + k.sidx * kStageBytes;
+                const int row = ra + 8 * ep;
+                float v = 0.0f;
+#pragma unroll
+                for (int w = 0; w < 2; ++w) {
+                    const uint32_t fw = w ? fl.y : fl.x;
+                    if (!fw) continue;
+                    // lanes of x row parity eh = h2; ep = 0 row ra, 1 row ra + 8
+                    const uint2 svw = ep ? su[1][w] : su[0][w];
+                    const uint2 zvw = ep ? zu[1][w] : zu[0][w];
+#pragma unroll 1
+                    for (int sub = 0; sub < 4; ++sub) {
+                        const uint32_t info = (fw >> (8 * sub)) & 0xffu;
+                        if (!info) continue;
+                        const float2 s2 = half2_bits_to_float2(sub < 2 ? svw.x : svw.y);
+                        const float2 z2 = half2_bits_to_float2(sub < 2 ? zvw.x : zvw.y);
+                        const float sc = (sub & 1) ? s2.y : s2.x, zc = (sub & 1) ? z2.y : z2.x;
+                        v += info != kSideMany
+                                 ? side_fast(info, sv[4 * w + sub], st + w * kBoxBytes, row, sub,
+                                             sc, zc)
+                                 : side_slow(J.x + (int64_t)m * J.K + 512 * k.kc +
+                                                 64 * (4 * w + sub),
+                                             st + w * kBoxBytes, row, sub, sc, zc);
+                    }
+                }
+                if (eh == h2) {
+                    if (ep) yb[mp] += v; else ya[mp] += v;
+                }
+            }
+        }
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
             uint32_t R[4][4];
@@ -694,13 +913,14 @@ __device__ __forceinline__ void consume_packed_mx(
                 __syncwarp();
                 mbar_arrive(smem_u32(&empty[k.sidx]));   // stage consumed (every lane)
             }
-            float sa[4], sb[4], za[4], zb[4];
+            float sa[4], sb[4];
+            int za[4], zb[4];
 #pragma unroll
             for (int p = 0; p < 2; ++p) {
                 const float2 a2 = half2_bits_to_float2(p ? su[0][w].y : su[0][w].x);
                 const float2 b2 = half2_bits_to_float2(p ? su[1][w].y : su[1][w].x);
-                const float2 c2 = half2_bits_to_float2(p ? zu[0][w].y : zu[0][w].x);
-                const float2 d2 = half2_bits_to_float2(p ? zu[1][w].y : zu[1][w].x);
+                const int2 c2 = half2_bits_to_int2(p ? zu[0][w].y : zu[0][w].x);
+                const int2 d2 = half2_bits_to_int2(p ? zu[1][w].y : zu[1][w].x);
                 sa[2 * p] = a2.x; sa[2 * p + 1] = a2.y;
                 sb[2 * p] = b2.x; sb[2 * p + 1] = b2.y;
                 za[2 * p] = c2.x; za[2 * p + 1] = c2.y;
@@ -727,13 +947,14 @@ __device__ __forceinline__ void consume_packed_mx(
                 const float4 t01 = reinterpret_cast<const float4 *>(tb)[0];
                 const float4 t23 = reinterpret_cast<const float4 *>(tb)[1];
                 const float f[4] = {t01.x, t01.z, t23.x, t23.z};
-                const float X[4] = {t01.y, t01.w, t23.y, t23.w};
+                const int T[4] = {__float_as_int(t01.y), __float_as_int(t01.w),
+                                  __float_as_int(t23.y), __float_as_int(t23.w)};
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
-                    const float va = (float)(C[g][0] + 256 * C[g][1]);
-                    const float vb = (float)(C[g][2] + 256 * C[g][3]);
-                    ya[mp] = fmaf(sa[g], fmaf(f[g], va, -za[g] * X[g]), ya[mp]);
-                    yb[mp] = fmaf(sb[g], fmaf(f[g], vb, -zb[g] * X[g]), yb[mp]);
+                    const float ra = exact_dot(C[g][0] + 256 * C[g][1], za[g], T[g]);
+                    const float rb = exact_dot(C[g][2] + 256 * C[g][3], zb[g], T[g]);
+                    ya[mp] = fmaf(sa[g] * f[g], ra, ya[mp]);
+                    yb[mp] = fmaf(sb[g] * f[g], rb, yb[mp]);
                 }
             }
         }
@@ -791,8 +1012,14 @@ __device__ __forceinline__ void consume_runtime(
         o = make_float2(1.0f, 0.0f);
         if (pass || row >= J.N || k0 >= J.K) return;
         const int64_t gi = (int64_t)row * (J.K / J.group) + k0 / J.group;
-        o.x = __ldg(reinterpret_cast<const float *>(J.s) + gi);
-        o.y = __ldg(reinterpret_cast<const float *>(J.z) + gi);
+        if (P.range) {
+            const float2 r =
+                range_of_word(__ldg(reinterpret_cast<const uint32_t *>(J.s) + gi));
+            o = rtn_params_from_range(r.x, r.y, P.bits);
+        } else {
+            o.x = __ldg(reinterpret_cast<const float *>(J.s) + gi);
+            o.y = __ldg(reinterpret_cast<const float *>(J.z) + gi);
+        }
     };
     float2 sz_a, sz_b = make_float2(1.0f, 0.0f);
     load_sz(k, sz_a);
@@ -1351,7 +1578,7 @@ __device__ __forceinline__ void unpack_a(uint32_t w, uint32_t *o) {
 // could reach a rounding boundary (then the chunk takes the exact quotient);
 // q = (q - z) + z in exact integer arithmetic.
 __device__ __forceinline__ void rtn_codes8(uint4 raw, float s, float z, float L,
-                                           uint32_t *o) {
+                                           bool centered, uint32_t *o) {
     const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
     float wv[8];
 #pragma unroll
@@ -1377,12 +1604,24 @@ __device__ __forceinline__ void rtn_codes8(uint4 raw, float s, float z, float L,
 #pragma unroll
         for (int i = 0; i < 8; ++i) cq[i] = centered_code_exact(wv[i], s, z, L);
     }
+    const float zb = centered ? 0.0f : z;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 p = __floats2bfloat162_rn(cq[i] + z, cq[i + 4] + z);
+        const __nv_bfloat162 p = __floats2bfloat162_rn(cq[i] + zb, cq[i + 4] + zb);
         o[i] = *reinterpret_cast<const uint32_t *>(&p);
     }
 }
+// The A operand holds centred codes q - z (bf16) when they are exact in bf16
+// (|q - z| <= 256 for every code, i.e. max(|z|, |L - z|) <= 256; packed:
+// |z| <= 224, where 1 + z/16 and (q - z)/16 are exact as well), so that
+// D = sum (q - z) x~ and an activation that meets q = z adds exactly
+// nothing.  Otherwise (a single-sign group whose zero lies far outside
+// [0, L]) A holds q (packed: 1 + q/16) and the epilogue subtracts z X~; then
+// |z| X~ is within a small factor of sum |q - z| |x~| and loses nothing.
+__device__ __forceinline__ bool centered_rt(float z, float L) {
+    return fmaxf(fabsf(z), fabsf(L - z)) <= 256.0f;
+}
+__device__ __forceinline__ bool centered_pk(float z) { return fabsf(z) <= 224.0f; }
 
 template <bool PACKED, int MT>
 __global__ void __launch_bounds__(tcd::kThreads, 1)
@@ -1426,12 +1665,15 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
         for (int s = 0; s < S; ++s) {
             // loader, plus every lane of the two scale/zero stagers (packed)
             mbar_init(smem_u32(&full[s]), PACKED ? 1 + 2 * 32 : 1);
-            // one arrival per transform and epilogue warp
-            mbar_init(smem_u32(&empty[s]), tcd::kTrWarps + tcd::kEpWarps);
+            // one arrival per transform warp (its reads of the stage are
+            // consumed by its tensor-memory stores, which it waits for), and
+            // one per epilogue lane (each lane's own scale/zero reads)
+            mbar_init(smem_u32(&empty[s]), tcd::kTrWarps + 32 * tcd::kEpWarps);
         }
         for (int b = 0; b < tcd::kXSlots; ++b) {
             mbar_init(smem_u32(&xfull[b]), 1);
-            mbar_init(smem_u32(&xempty[b]), 1 + tcd::kEpWarps);   // MMAs + epilogue warps
+            // the MMAs' commit + every epilogue lane (each lane's own X~ reads)
+            mbar_init(smem_u32(&xempty[b]), 1 + 32 * tcd::kEpWarps);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&afull[b]), tcd::kTrWarps);
@@ -1455,6 +1697,11 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
     auto rt_sz = [&](const StreamJob &J, int row, int gg) -> float2 {
         if (row >= J.N || 64 * gg >= J.K) return make_float2(0.0f, 0.0f);
         const int64_t gi = (int64_t)row * (J.K / J.group) + (64 * gg) / J.group;
+        if (P.range) {
+            const float2 r =
+                range_of_word(__ldg(reinterpret_cast<const uint32_t *>(J.s) + gi));
+            return rtn_params_from_range(r.x, r.y, P.bits);
+        }
         return make_float2(__ldg(reinterpret_cast<const float *>(J.s) + gi),
                            __ldg(reinterpret_cast<const float *>(J.z) + gi));
     };
@@ -1581,6 +1828,20 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
                                 unpack_a(v1.y, o + 20);
                                 unpack_a(v1.z, o + 24);
                                 unpack_a(v1.w, o + 28);
+                                // centred: (1 + q/16) - (1 + z/16) = (q - z)/16, exact
+                                const float zc = __half2float(__ushort_as_half(
+                                    reinterpret_cast<const unsigned short *>(
+                                        szring + s * kSzBytes + kSzBytes / 2 +
+                                        r * 16)[hs * SG + gi]));
+                                if (centered_pk(zc)) {
+                                    const __nv_bfloat162 zz = __float2bfloat162_rn(1.0f + zc * 0.0625f);
+#pragma unroll
+                                    for (int c = 0; c < 32; ++c) {
+                                        const __nv_bfloat162 a =
+                                            __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&o[c]), zz);
+                                        o[c] = *reinterpret_cast<const uint32_t *>(&a);
+                                    }
+                                }
                             } else {
                                 // group gi is the stage's box gi: 64 fp16 of row r
                                 const uint8_t *box = st + gi * kBoxBytes + r * 128;
@@ -1588,7 +1849,8 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
                                 for (int c = 0; c < 8; ++c) {
                                     const uint4 raw =
                                         *reinterpret_cast<const uint4 *>(box + ((c ^ (r & 7)) << 4));
-                                    rtn_codes8(raw, szv[i].x, szv[i].y, L, o + 4 * c);
+                                    rtn_codes8(raw, szv[i].x, szv[i].y, L,
+                                               centered_rt(szv[i].y, L), o + 4 * c);
                                 }
                             }
                             // tcgen05.st is warp-collective: reconverge after
@@ -1630,10 +1892,11 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
                     uint32_t sw[4], zw[4];
                     float2 rcoef[PACKED ? 1 : G::kGroups];
                     if constexpr (!PACKED) {
+                        const float L = (float)((1 << P.bits) - 1);
 #pragma unroll
                         for (int gl = 0; gl < G::kGroups; ++gl) {
                             const float2 v = rt_sz(J, row, G::kGroups * kc + gl);
-                            rcoef[gl] = make_float2(v.x, -v.x * v.y);
+                            rcoef[gl] = make_float2(v.x, centered_rt(v.y, L) ? 0.0f : -v.x * v.y);
                         }
                     }
                     if (!wait_all(&full[s], (g / S) & 1)) {
@@ -1654,7 +1917,8 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
                             const float2 s2 = half2_bits_to_float2(sw[gl >> 1]);
                             const float2 z2 = half2_bits_to_float2(zw[gl >> 1]);
                             const float sc = (gl & 1) ? s2.y : s2.x, zc = (gl & 1) ? z2.y : z2.x;
-                            return make_float2(16.0f * sc, -sc * (16.0f + zc));
+                            return make_float2(16.0f * sc,
+                                               centered_pk(zc) ? 0.0f : -sc * (16.0f + zc));
                         } else {
                             return rcoef[gl];
                         }
@@ -1725,11 +1989,12 @@ gemv_tc_kernel(const __grid_constant__ StreamParams P) {
                         }
                     }
                     if (!ok) break;
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(smem_u32(&empty[s]));        // scales read
-                        mbar_arrive(smem_u32(&xempty[xs]));      // X~ read
-                    }
+                    // every lane releases the slots after its own reads: an
+                    // arrive orders only the arriving thread's accesses, and a
+                    // lane's shared-memory load may still be in flight when
+                    // another lane of the warp arrives
+                    mbar_arrive(smem_u32(&empty[s]));        // scales read
+                    mbar_arrive(smem_u32(&xempty[xs]));      // X~ read
                     if (kc + 1 == kch) {
 #pragma unroll
                         for (int i = 0; i < MH; ++i) {
@@ -2130,6 +2395,7 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
         if (stages < 2) return BC_ERR_UNSUPPORTED;
         P.M = M;
         P.bits = bits;
+        P.range = (int)jobs[0].range;
         P.xslot_bytes = (int)xs;
         P.stages = stages;
         P.early = early_start ? 1 : 0;
@@ -2147,6 +2413,12 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
         plans.insert(plans.begin(), std::move(plan));
         if ((int)plans.size() > kPlanCache) plans.pop_back();
     }
+    return BC_OK;
+}
+
+bc_status gemv_set_wait_limit(long long cycles) {
+    if (cudaMemcpyToSymbol(g_gemv_wait_limit, &cycles, sizeof(cycles)) != cudaSuccess)
+        return BC_ERR_CUDA;
     return BC_OK;
 }
 

@@ -461,3 +461,47 @@ def test_tc_decode_more_matrices_than_one_launch(cuda_lib, mode, bits):
         ref = oracle.matmul_q(xs[W.shape[1]], W, bits, 64, mode)
         assert_close(host(items[i][4]), ref["y"], ref["A"], TOL_FP32, f"matrix {i}")
     assert cuda_lib.device_timeouts() == 0
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8])
+@pytest.mark.parametrize("big", [3.0e3, 1.0e5, 1.0e6])
+def test_stream_outliers_where_weights_are_zero(cuda_lib, M, big):
+    """Activation outliers placed where every row's dequantized weight is 0
+    (the weight column is zero, so its code equals the zero point): the
+    outlier adds nothing to y or to A = sum |x w'|, but it sets the group's
+    integer grid and enters the zero-point term.  Neighbours 3000, 10^5 and
+    10^6 times smaller, and 1e-30 values, must still meet the fp32 bar.  A grouped launch of 160 matrices (large
+    enough for the streaming kernels); M = 8 takes the tensor-core decode."""
+    rng = np.random.default_rng(int(big) % 1000 + M)
+    K, N = 896, 896
+    G = K // 64
+    x = wl.activation(81, M, "x", M, K).astype(np.float64)
+    cols = set()
+    for m in range(M):
+        for g in range(G):
+            k_big = 64 * g + (7 + 2 * m if g % 2 else 10 + 2 * m)   # odd, even k
+            x[m, k_big] = big * (1 if (g + m) % 2 else -1)
+            x[m, 64 * g + 21 + m] = 1.0e-30
+            cols.add(k_big)
+    x = x.astype(np.float32)
+    items, refs = [], []
+    xd = dev(x)
+    for i in range(160):
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+        W[:, sorted(cols)] = 0.0
+        Wd = dev(W)
+        s, z = cuda_lib.group_params(Wd, 4, 64, torch.float16)
+        Wk = cuda_lib.pack_int4(Wd, s, z)
+        y = torch.full((M, N), float("nan"), device="cuda")
+        items.append((xd, Wk, s, z, y))
+        if i < 3 or i == 159:
+            refs.append((i, oracle.matmul_q(x, W, 4, 64, "packed")))
+    cuda_lib.matmul_q_batched(cuda_lib.make_descs(items), M, 4, 64,
+                              cuda_lib.BC_MODE_PACKED_INT4)
+    torch.cuda.synchronize()
+    for i, ref in refs:
+        # the outliers meet w' = 0 exactly: they must not show up in A
+        assert np.all(ref["A"] < 1.0e3)
+        assert_close(host(items[i][4]), ref["y"], ref["A"], TOL_FP32,
+                     f"outlier {big:g} M={M} matrix {i}")
+    assert cuda_lib.device_timeouts() == 0
