@@ -1,31 +1,44 @@
 // bc_gemm_sm100.cu -- prefill GEMM on the 5th-generation tensor cores.
 //
-// y[m,n] = sum_k x[m,k] * w'[n,k] for M >= 64 prompt rows, bf16 x, packed
-// int4 W with fp16 scale/zero per 64-block along K (Enargeia, "Four bits per
-// weight": int4 weights unpacked on chip, never written back to memory;
-// Enargeia's benchmark table: prefill at 128 and 2048 tokens; the tiled
-// matmul ladder on the same page: tiling and register blocking decide
-// matmul speed).
+// y[m,n] = sum_k x[m,k] * w'[n,k] for M >= 64 prompt rows, bf16 x, and
+// weights in either form of the method:
+//   * packed int4 with fp16 scale/zero per 64-block along K (Enargeia,
+//     "Four bits per weight": int4 weights unpacked on chip, never written
+//     back; its benchmark table measures prefill at 128 and 2048 tokens);
+//   * fp16 weights re-quantized as they are read, group-wise (64) or per
+//     channel, at 2..8 bits or passed through at 16 (BITCRUSH BC-06, "Under
+//     the hood": matmul_q computes the RTN codes inline at any lever
+//     position, so a prompt can be prefilled at any precision).
+// Enargeia's tiled-matmul ladder: tiling and register blocking decide
+// matmul speed; here the tiles feed tcgen05 from shared memory and TMEM.
 //
 // Tile = 128 weight rows (the MMA's M, i.e. TMEM lanes) x BNX activation
 // rows (the MMA's N) x 64 along K (one quantization block, one 128-byte
 // swizzle atom row of bf16).  Per 64-block of K:
-//   * one thread (warp 0) issues two TMA loads into a smem stage: the bf16
-//     x tile (128B-swizzled, K-major) and the 128 x 32-byte packed codes;
-//   * eight dequant warps turn the codes into bf16 w' = (q - z) * s in the
-//     same 128B-swizzled K-major layout the MMA reads (exact q - z in bf16
-//     arithmetic, one rounding for the scale), then fence the generic-proxy
-//     writes for the tensor core;
+//   * one thread (warp 0) issues the TMA loads of a stage: the bf16 x tile
+//     (128B-swizzled, K-major) and the weights -- 128 x 32 bytes of packed
+//     codes, or the 128 x 64 fp16 weights themselves, landed 128B-swizzled
+//     in the stage's A tile;
+//   * eight dequant warps form bf16 w' = (q - z) * s in the same
+//     128B-swizzled K-major layout the MMA reads (packed: exact q - z in
+//     bf16 arithmetic and one rounding for the scale; runtime: the exact RTN
+//     code of each fp16 weight, then one rounding of (q - z) s, written over
+//     the weight it came from), then fence the generic-proxy writes for the
+//     tensor core;
 //   * one thread (warp 1) issues four tcgen05.mma.kind::f16 (K = 16 each)
 //     accumulating fp32 in TMEM, and tcgen05.commit frees the stage;
 //   * four epilogue warps drain the finished accumulator (tcgen05.ld) and
 //     store y with 128-byte coalesced rows, while the next tile accumulates
 //     into the second TMEM buffer.
-// The kernel is persistent (one CTA per SM, tiles strided over the grid)
-// and spans every matrix of a grouped launch.  All waits are bounded: a
-// wait that runs out records a timeout, the CTA stops, waits (bounded) for
-// its own TMA copies in flight and frees its TMEM.
+// The kernel is persistent (one CTA per SM) and spans every matrix of a
+// grouped launch.  Each CTA owns a contiguous range of tiles chosen on the
+// host so that the ranges cost about the same (a tile costs its K/64 stages
+// plus its epilogue), instead of a round-robin stride that leaves SMs idle
+// when matrices of very different K share a launch.  All waits are bounded:
+// a wait that runs out records a timeout, the CTA stops, waits (bounded) for
+// its own copies and MMAs in flight and frees its TMEM.
 #include "bc_internal.cuh"
+#include "bc_rtn.cuh"
 #include "bc_tc.cuh"
 
 #include <cuda.h>
@@ -38,6 +51,9 @@
 namespace bc {
 
 __device__ unsigned int g_gemm_timeouts = 0;
+// Limit of the pipeline waits, in clock64 cycles (bc_set_wait_limit);
+// the drains after an abort keep the fixed ~2 s limit.
+__device__ long long g_gemm_wait_limit = 4000000000LL;
 
 namespace {
 
@@ -48,36 +64,46 @@ constexpr int kDqWarp0 = 2, kDqWarps = 8;   // warps 2..9
 constexpr int kEpWarp0 = 10, kEpWarps = 4;  // warps 10..13
 constexpr int kThreads = 32 * (kEpWarp0 + kEpWarps);
 constexpr int kMaxJobs = 80;
+constexpr int kMaxCtas = 160;
 constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 2 GHz
 
+// Weight forms.
+constexpr int kPacked = 0;    // int4 codes, fp16 scale/zero per 64-block
+constexpr int kRuntime = 1;   // fp16 W, RTN inline (fp32 scale/zero or ranges)
+
 struct GemmJobDev {
-    const __half *s;
-    const __half *z;
+    const void *s;         // packed: fp16 [N][K/64]; runtime: fp32 [N][K/g] or ranges
+    const void *z;         // packed: fp16; runtime: fp32 (unused with ranges)
     float *y;
-    int N, K;
+    int N, K, group;       // group: 64, or K (runtime per channel)
     int tile_begin;
     int xblocks;           // ceil(M / BNX)
 };
 
 struct __align__(64) GemmParams {
     CUtensorMap xmap[kMaxJobs];     // bf16 x [M][K], box {64, BNX}, SW128
-    CUtensorMap cmap[kMaxJobs];     // u8 packed [N][K/2], box {32, 128}
+    CUtensorMap wmap[kMaxJobs];     // packed u8 [N][K/2] box {32, 128}; fp16 W [N][K] box {64, 128} SW128
     GemmJobDev jobs[kMaxJobs];
+    int cta_begin[kMaxCtas + 1];    // tile range of each CTA
     int count, total_tiles, M;
+    int bits;                       // runtime: 2..8 or 16 (passthrough)
+    int range;                      // runtime: s holds per-group ranges
 };
 static_assert(sizeof(GemmParams) <= 32000, "kernel parameter space");
 
-template <int BNX> struct Cfg {
-    static constexpr int kABytes = kBM * 128;          // 16 KB
+template <int BNX, int WF> struct Cfg {
+    static constexpr int kABytes = kBM * 128;          // 16 KB (runtime: W lands here)
     static constexpr int kBBytes = BNX * 128;
-    static constexpr int kCBytes = kBM * 32;           // 4 KB
-    static constexpr int kStageBytes = kABytes + kBBytes + kCBytes;
-    static constexpr int kStages = BNX == 256 ? 4 : 6;
-    static constexpr int kTmemCols = 2 * BNX;
+    static constexpr int kCBytes = WF == kPacked ? kBM * 32 : 0;   // 4 KB of codes
+    static constexpr int kStageBytes = kABytes + kBBytes + kCBytes;  // multiple of 1024
     static constexpr int kBarBytes = 4096;     // barriers + job table copy
+    static constexpr int kStages =
+        std::min(6, (227 * 1024 - kBarBytes - 1024) / kStageBytes);
+    static constexpr int kTmemCols = 2 * BNX;
     static constexpr int kSmem = kStages * kStageBytes + kBarBytes + 1024;
     // instruction descriptor: D f32, A/B bf16, K-major both, N, M = 128
     static constexpr uint32_t kIdesc = tc::idesc_bf16(kBM, BNX);
+    static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 };
 
 // ---- small PTX wrappers ----------------------------------------------------
@@ -103,16 +129,29 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
+// The same test, letting the thread sleep (up to a hint of 20 us) until the
+// phase completes: a waiting warp then takes no issue slots from the warps
+// doing the work.
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity), "r"(20000u) : "memory");
+    return ok != 0;
+}
 // Bounded wait; false (and a recorded timeout, once per CTA) if it ran out
 // or if another role of this CTA already gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int *abort_flag) {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
+    const long long limit = *(volatile long long *)&g_gemm_wait_limit;
     while (true) {
-        if (mbar_try(bar, parity)) return true;
+        if (mbar_try_sleep(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             if (atomicExch((int *)abort_flag, 1) == 0)
                 atomicAdd(&g_gemm_timeouts, 1u);
             return false;
@@ -126,6 +165,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         " [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
+}
+// Bring one weight box of a later tile into L2 (no shared memory, no
+// barrier): the TMA of that stage then meets L2 instead of HBM latency.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -175,6 +223,26 @@ __device__ __noinline__ uint4 dequant8_wide(uint32_t w, float z, float s) {
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
+// Runtime mode: 8 fp16 weights -> 8 bf16 w' = (q - z) s (or w itself at 16
+// bits), k order kept.
+__device__ __forceinline__ uint4 requant8(uint4 raw, float s, float z, float L, bool pass) {
+    uint32_t o[4];
+    if (pass) {
+        const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(h[i]);
+            o[i] = bf2_as_u32(__floats2bfloat162_rn(f.x, f.y));
+        }
+    } else {
+        float c[8];
+        rtn_centered8(raw, s, z, L, c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            o[i] = bf2_as_u32(__floats2bfloat162_rn(c[2 * i] * s, c[2 * i + 1] * s));
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
 
 // Job descriptors are read from a shared-memory copy (sjobs): dynamically
 // indexed reads of the parameter block miss the constant cache.
@@ -190,13 +258,14 @@ __device__ __forceinline__ int find_job(const GemmJobDev *jobs, int count, int t
 constexpr int kLook = 4;     // scale/zero look-ahead, in 64-blocks of K
 
 // Walks the (tile, 64-block) sequence a dequant thread consumes and loads
-// the scale/zero of its weight row for each position.
-struct SzCursor {
-    int tile, kb, kblocks;
-    const __half *srow, *zrow;
+// the scale and zero of its weight row for each position.
+template <int WF> struct SzCursor {
+    int tile, t_end, kb, kblocks, group;
+    const void *srow;
+    const void *zrow;
     const GemmJobDev *jobs;
     __device__ __forceinline__ void bind(const GemmParams &P, int r) {
-        if (tile >= P.total_tiles) {
+        if (tile >= t_end) {
             srow = zrow = nullptr;
             kblocks = 1;
             return;
@@ -205,42 +274,60 @@ struct SzCursor {
         const int nb = (tile - J.tile_begin) / J.xblocks;
         const int row = nb * kBM + r;
         kblocks = J.K / kBK;
+        group = J.group;
+        const int64_t G = J.K / J.group;
         if (row < J.N) {
-            srow = J.s + (int64_t)row * kblocks;
-            zrow = J.z + (int64_t)row * kblocks;
+            const size_t es = (WF == kPacked) ? 2 : 4;
+            srow = static_cast<const uint8_t *>(J.s) + (int64_t)row * G * es;
+            zrow = J.z ? static_cast<const uint8_t *>(J.z) + (int64_t)row * G * es : nullptr;
         } else {
             srow = zrow = nullptr;
         }
     }
-    __device__ __forceinline__ void init(const GemmParams &P, const GemmJobDev *sj,
-                                         int first, int, int r) {
+    __device__ __forceinline__ void init(const GemmParams &P, const GemmJobDev *sj, int first,
+                                         int last, int r) {
         jobs = sj;
         tile = first;
+        t_end = last;
         kb = 0;
         bind(P, r);
     }
-    __device__ __forceinline__ void advance(const GemmParams &P, int stride, int r) {
+    __device__ __forceinline__ void advance(const GemmParams &P, int r) {
         if (++kb == kblocks) {
             kb = 0;
-            tile += stride;
+            ++tile;
             bind(P, r);
         }
     }
-    __device__ __forceinline__ void load(float &s, float &z) const {
-        if (srow) {
-            s = __half2float(__ldg(srow + kb));
-            z = __half2float(__ldg(zrow + kb));
+    // (s, z) of the current position
+    __device__ __forceinline__ void load(const GemmParams &P, float &s, float &z) const {
+        s = 0.0f;
+        z = 0.0f;
+        if (!srow) return;
+        if constexpr (WF == kPacked) {
+            s = __half2float(__ldg(static_cast<const __half *>(srow) + kb));
+            z = __half2float(__ldg(static_cast<const __half *>(zrow) + kb));
         } else {
-            s = 0.0f;
-            z = 0.0f;
+            if (P.bits == 16) return;
+            const int gi = (kb * kBK) / group;
+            if (P.range) {
+                const float2 rg =
+                    range_of_word(__ldg(static_cast<const uint32_t *>(srow) + gi));
+                const float2 sz = rtn_params_from_range(rg.x, rg.y, P.bits);
+                s = sz.x;
+                z = sz.y;
+            } else {
+                s = __ldg(static_cast<const float *>(srow) + gi);
+                z = __ldg(static_cast<const float *>(zrow) + gi);
+            }
         }
     }
 };
 
-template <int BNX>
+template <int BNX, int WF>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_packed_kernel(const __grid_constant__ GemmParams P) {
-    using C = Cfg<BNX>;
+gemm_kernel(const __grid_constant__ GemmParams P) {
+    using C = Cfg<BNX, WF>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -262,6 +349,7 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
     }
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t_begin = P.cta_begin[blockIdx.x], t_end = P.cta_begin[blockIdx.x + 1];
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -284,43 +372,70 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int K_tiles_dummy = 0;
-    (void)K_tiles_dummy;
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
             uint32_t g = 0;                       // k-block counter over tiles
             uint32_t armed = 0;                   // stages with a load issued
-            for (int tile = blockIdx.x; tile < P.total_tiles && !*abort_flag;
-                 tile += gridDim.x) {
+            for (int tile = t_begin; tile < t_end && !*abort_flag; ++tile) {
                 const int j = find_job(sjobs, P.count, tile);
                 const GemmJobDev &J = sjobs[j];
                 const int local = tile - J.tile_begin;
                 const int nb = local / J.xblocks, xb = local % J.xblocks;
                 const int kblocks = J.K / kBK;
+                if (tile + 1 < t_end) {
+                    // the next tile's weights (and their scales/zeros) to L2
+                    // while this one streams, unless it reuses these rows
+                    const int j2 = find_job(sjobs, P.count, tile + 1);
+                    const GemmJobDev &J2 = sjobs[j2];
+                    const int nb2 = (tile + 1 - J2.tile_begin) / J2.xblocks;
+                    if (j2 != j || nb2 != nb) {
+                        const int kb2 = J2.K / kBK;
+                        for (int q = 0; q < kb2; ++q)
+                            tma_prefetch_2d(&P.wmap[j2], WF == kPacked ? q * (kBK / 2) : q * kBK,
+                                            nb2 * kBM);
+                        const int64_t G2 = J2.K / J2.group;
+                        const int rows = min(kBM, J2.N - nb2 * kBM);
+                        const int64_t es = WF == kPacked ? 2 : 4;
+                        const int64_t bytes = rows * G2 * es;
+                        const char *sb = static_cast<const char *>(J2.s) + (int64_t)nb2 * kBM * G2 * es;
+                        const char *zb = J2.z ? static_cast<const char *>(J2.z) +
+                                                    (int64_t)nb2 * kBM * G2 * es
+                                              : nullptr;
+                        for (int64_t o = 0; o < bytes; o += 128) {
+                            if (P.bits != 16 || WF == kPacked) {
+                                prefetch_l2(sb + o);
+                                if (zb) prefetch_l2(zb + o);
+                            }
+                        }
+                    }
+                }
                 for (int kb = 0; kb < kblocks; ++kb, ++g) {
                     const int s = g % C::kStages;
                     const uint32_t ph = (g / C::kStages) & 1;
                     if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag)) break;
                     uint8_t *st = smem + s * C::kStageBytes;
                     const uint32_t fb = smem_u32(&full_tma[s]);
-                    mbar_expect_tx(fb, C::kBBytes + C::kCBytes);
-                    tma_load_2d(smem_u32(st + C::kABytes), &P.xmap[j], kb * kBK,
-                                xb * BNX, fb);
-                    tma_load_2d(smem_u32(st + C::kABytes + C::kBBytes), &P.cmap[j],
-                                kb * (kBK / 2), nb * kBM, fb);
+                    if constexpr (WF == kPacked) {
+                        mbar_expect_tx(fb, C::kBBytes + C::kCBytes);
+                        tma_load_2d(smem_u32(st + C::kABytes + C::kBBytes), &P.wmap[j],
+                                    kb * (kBK / 2), nb * kBM, fb);
+                    } else {
+                        mbar_expect_tx(fb, C::kBBytes + C::kABytes);
+                        tma_load_2d(smem_u32(st), &P.wmap[j], kb * kBK, nb * kBM, fb);
+                    }
+                    tma_load_2d(smem_u32(st + C::kABytes), &P.xmap[j], kb * kBK, xb * BNX, fb);
                     armed |= 1u << s;
                 }
             }
             // drain: every load this thread issued has landed before exit
             // (on the normal path each stage was consumed, so these pass)
-            for (uint32_t q = 0; q < (uint32_t)C::kStages; ++q) {
+            for (uint32_t q = 0; q < (uint32_t)C::kStages && g > 0; ++q) {
                 if (!(armed & (1u << q))) continue;
                 // the last use of stage q had index g_last = largest g' < g with
                 // g' % kStages == q
-                if (g == 0) break;
-                uint32_t gl = (g - 1) - (((g - 1) % C::kStages + C::kStages - q) %
-                                         C::kStages);
+                const uint32_t gl = (g - 1) - (((g - 1) % C::kStages + C::kStages - q) %
+                                               C::kStages);
                 const long long t0 = clock64();
                 while (!mbar_try(smem_u32(&full_tma[q]), (gl / C::kStages) & 1) &&
                        clock64() - t0 < kWaitCycles) {
@@ -337,9 +452,8 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
         const uint64_t bdesc0 = tc::sw128_desc(smem_u32(smem + C::kABytes));
         uint32_t g = 0;
         int lt = 0;
-        for (int tile = blockIdx.x;
-             tile < P.total_tiles && !__shfl_sync(0xffffffffu, (int)*abort_flag, 0);
-             tile += gridDim.x, ++lt) {
+        for (int tile = t_begin;
+             tile < t_end && !__shfl_sync(0xffffffffu, (int)*abort_flag, 0); ++tile, ++lt) {
             const int j = find_job(sjobs, P.count, tile);
             const int kblocks = sjobs[j].K / kBK;
             const int buf = lt & 1;
@@ -390,18 +504,20 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
         // copy waits on a load that is still in flight.
         const int t = threadIdx.x - 32 * kDqWarp0;
         const int r = t & (kBM - 1), h = t >> 7;
-        SzCursor la;                        // look-ahead cursor
-        la.init(P, sjobs, blockIdx.x, gridDim.x, r);
+        const float L = (float)((1 << (P.bits & 15)) - 1);
+        const bool pass = WF == kRuntime && P.bits == 16;
+        SzCursor<WF> la;                    // look-ahead cursor
+        la.init(P, sjobs, t_begin, t_end, r);
         float sq[kLook], zq[kLook];
 #pragma unroll
         for (int i = 0; i < kLook; ++i) {
-            la.load(sq[i], zq[i]);
-            la.advance(P, gridDim.x, r);
+            la.load(P, sq[i], zq[i]);
+            la.advance(P, r);
         }
-        int tile = blockIdx.x, kb = 0, kblocks = 1;
+        int tile = t_begin, kb = 0, kblocks = 1;
         bool valid = false;
         auto bind = [&]() {
-            if (tile >= P.total_tiles) return;
+            if (tile >= t_end) return;
             const GemmJobDev &J = sjobs[find_job(sjobs, P.count, tile)];
             const int nb = (tile - J.tile_begin) / J.xblocks;
             kblocks = J.K / kBK;
@@ -410,13 +526,13 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
         bind();
         uint32_t g = 0;
         bool ok = true;
-        while (ok && tile < P.total_tiles && !*abort_flag) {
+        while (ok && tile < t_end && !*abort_flag) {
 #pragma unroll
             for (int j = 0; j < kLook; ++j) {
-                if (tile >= P.total_tiles) break;
+                if (tile >= t_end) break;
                 const float sf = sq[j], zf = zq[j];
-                la.load(sq[j], zq[j]);             // refill slot j, kLook ahead
-                la.advance(P, gridDim.x, r);
+                la.load(P, sq[j], zq[j]);          // refill slot j, kLook ahead
+                la.advance(P, r);
                 const int s = g % C::kStages;
                 const uint32_t ph = (g / C::kStages) & 1;
                 if (!mbar_wait(smem_u32(&full_tma[s]), ph, abort_flag)) {
@@ -424,9 +540,6 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
                     break;
                 }
                 uint8_t *st = smem + s * C::kStageBytes;
-                const uint4 codes = *reinterpret_cast<const uint4 *>(
-                    st + C::kABytes + C::kBBytes + r * 32 + h * 16);
-                const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
                 uint8_t *arow = st + (r >> 3) * 1024 + (r & 7) * 128;
                 if (!valid) {
 #pragma unroll
@@ -435,23 +548,35 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
                         *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) =
                             make_uint4(0, 0, 0, 0);
                     }
-                } else if (fabsf(zf) <= 128.0f) {
-                    const __nv_bfloat16 zb1 = __float2bfloat16_rn(128.0f + zf);
-                    const __nv_bfloat16 sb1 = __float2bfloat16_rn(sf);
-                    const __nv_bfloat162 zb = __halves2bfloat162(zb1, zb1);
-                    const __nv_bfloat162 sb = __halves2bfloat162(sb1, sb1);
+                } else if constexpr (WF == kRuntime) {
+                    // the 8 fp16 of each chunk are replaced by their 8 bf16 w'
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int chunk = h * 4 + i;
-                        *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) =
-                            dequant8(cw[i], zb, sb);
+                        uint4 *p = reinterpret_cast<uint4 *>(arow + (((h * 4 + i) ^ (r & 7)) << 4));
+                        *p = requant8(*p, sf, zf, L, pass);
                     }
                 } else {
+                    const uint4 codes = *reinterpret_cast<const uint4 *>(
+                        st + C::kABytes + C::kBBytes + r * 32 + h * 16);
+                    const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
+                    if (fabsf(zf) <= 128.0f) {
+                        const __nv_bfloat16 zb1 = __float2bfloat16_rn(128.0f + zf);
+                        const __nv_bfloat16 sb1 = __float2bfloat16_rn(sf);
+                        const __nv_bfloat162 zb = __halves2bfloat162(zb1, zb1);
+                        const __nv_bfloat162 sb = __halves2bfloat162(sb1, sb1);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int chunk = h * 4 + i;
-                        *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) =
-                            dequant8_wide(cw[i], zf, sf);
+                        for (int i = 0; i < 4; ++i) {
+                            const int chunk = h * 4 + i;
+                            *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) =
+                                dequant8(cw[i], zb, sb);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int chunk = h * 4 + i;
+                            *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) =
+                                dequant8_wide(cw[i], zf, sf);
+                        }
                     }
                 }
                 fence_proxy_async_smem();
@@ -460,7 +585,7 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
                 ++g;
                 if (++kb == kblocks) {
                     kb = 0;
-                    tile += gridDim.x;
+                    ++tile;
                     bind();
                 }
             }
@@ -469,8 +594,7 @@ gemm_packed_kernel(const __grid_constant__ GemmParams P) {
         // epilogue: warp quarter q reads TMEM lanes 32q..32q+31 (weight rows)
         const int q = warp & 3;
         int lt = 0;
-        for (int tile = blockIdx.x; tile < P.total_tiles && !*abort_flag;
-             tile += gridDim.x, ++lt) {
+        for (int tile = t_begin; tile < t_end && !*abort_flag; ++tile, ++lt) {
             const int j = find_job(sjobs, P.count, tile);
             const GemmJobDev &J = sjobs[j];
             const int local = tile - J.tile_begin;
@@ -535,51 +659,114 @@ bool encode_x(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m,
 }
 
 bool encode_codes(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m,
-                  const uint8_t *w, int64_t N, int64_t K) {
+                  const void *w, int64_t N, int64_t K) {
     cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
     cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
     cuuint32_t box[2] = {(cuuint32_t)(kBK / 2), (cuuint32_t)kBM};
     cuuint32_t es[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void *)w, dims, strides, box,
-               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(w), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BNX>
-bc_status launch_bnx(const GemmJob *jobs, int count, int64_t M, cudaStream_t s,
-                     int sm_count) {
-    using C = Cfg<BNX>;
+// fp16 W [N][K], box 64 x 128 rows, 128B swizzle (the A tile's layout)
+bool encode_w16(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const void *w,
+                int64_t N, int64_t K) {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBM};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(w), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Contiguous tile ranges per CTA that minimise the costliest range (binary
+// search on the bound, greedy fill).  A tile costs its K/64 stages plus a
+// fixed share for its epilogue.
+void partition_tiles(GemmParams &P, const std::vector<double> &tcost, int grid) {
+    const int n = (int)tcost.size();
+    double total = 0, tmax = 0;
+    for (double c : tcost) {
+        total += c;
+        tmax = std::max(tmax, c);
+    }
+    auto fill = [&](double T, bool out) -> int {
+        int ctas = 1;
+        double cur = 0;
+        if (out) P.cta_begin[0] = 0;
+        for (int i = 0; i < n; ++i) {
+            if (cur > 0 && cur + tcost[i] > T) {
+                if (out && ctas < grid) P.cta_begin[ctas] = i;
+                ++ctas;
+                cur = 0;
+            }
+            cur += tcost[i];
+        }
+        return ctas;
+    };
+    double lo = std::max(tmax, total / grid), hi = total + tmax;
+    for (int it = 0; it < 60 && hi - lo > 0.5; ++it) {
+        const double mid = 0.5 * (lo + hi);
+        if (fill(mid, false) <= grid) hi = mid; else lo = mid;
+    }
+    const int used = std::min(fill(hi, true), grid);
+    for (int c = used; c <= grid; ++c) P.cta_begin[c] = n;
+}
+
+template <int BNX, int WF>
+bc_status launch_cfg(const GemmJob *jobs, int count, int64_t M, int bits, bool range,
+                     cudaStream_t s, int sm_count) {
+    using C = Cfg<BNX, WF>;
     auto enc = get_encoder();
     if (!enc) return BC_ERR_CUDA;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_packed_kernel<BNX>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        C::kSmem);
-    });
-    if (attr_err != cudaSuccess) return BC_ERR_CUDA;
+    static std::mutex mu;
+    static int attr_set[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return BC_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(gemm_kernel<BNX, WF>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     C::kSmem) != cudaSuccess)
+                return BC_ERR_CUDA;
+            attr_set[dev] = 1;
+        }
+    }
     thread_local GemmParams *Pp = nullptr;
     if (!Pp) Pp = new GemmParams();
     GemmParams &P = *Pp;
+    std::vector<double> tcost;
     for (int b = 0; b < count; b += kMaxJobs) {
         const int n = std::min(kMaxJobs, count - b);
         int tiles = 0;
         const int xblocks = (int)((M + BNX - 1) / BNX);
+        tcost.clear();
         for (int i = 0; i < n; ++i) {
             const GemmJob &J = jobs[b + i];
-            if (!encode_x(enc, &P.xmap[i], J.x, M, J.K, BNX) ||
-                !encode_codes(enc, &P.cmap[i], J.w, J.N, J.K))
-                return BC_ERR_CUDA;
-            P.jobs[i] = GemmJobDev{J.s, J.z, J.y, (int)J.N, (int)J.K, tiles, xblocks};
-            tiles += (int)((J.N + kBM - 1) / kBM) * xblocks;
+            if (!encode_x(enc, &P.xmap[i], J.x, M, J.K, BNX)) return BC_ERR_CUDA;
+            const bool ok = WF == kPacked ? encode_codes(enc, &P.wmap[i], J.w, J.N, J.K)
+                                          : encode_w16(enc, &P.wmap[i], J.w, J.N, J.K);
+            if (!ok) return BC_ERR_CUDA;
+            P.jobs[i] = GemmJobDev{J.s, J.z, J.y, (int)J.N, (int)J.K, (int)J.group, tiles,
+                                   xblocks};
+            const int nt = (int)((J.N + kBM - 1) / kBM) * xblocks;
+            tiles += nt;
+            // cost in stages: K/64 of MMA plus the epilogue (BNX/32 loads of
+            // 32 columns and their stores), about two stages' worth
+            tcost.insert(tcost.end(), nt, (double)(J.K / kBK) + 2.0 * BNX / 128.0);
         }
         P.count = n;
         P.total_tiles = tiles;
         P.M = (int)M;
-        const int grid = std::max(1, std::min(tiles, sm_count));
-        gemm_packed_kernel<BNX><<<grid, kThreads, C::kSmem, s>>>(P);
+        P.bits = bits;
+        P.range = range ? 1 : 0;
+        const int grid = std::max(1, std::min({tiles, sm_count, kMaxCtas}));
+        partition_tiles(P, tcost, grid);
+        gemm_kernel<BNX, WF><<<grid, kThreads, C::kSmem, s>>>(P);
         bc_status st = cuda_status();
         if (st != BC_OK) return st;
     }
@@ -588,8 +775,8 @@ bc_status launch_bnx(const GemmJob *jobs, int count, int64_t M, cudaStream_t s,
 
 }  // namespace
 
-bc_status launch_gemm_packed(const GemmJob *jobs, int count, int64_t M,
-                             cudaStream_t s) {
+bc_status launch_gemm(const GemmJob *jobs, int count, int64_t M, bool packed, int bits,
+                      bool range, cudaStream_t s) {
     DeviceInfo di;
     if (!device_info(&di)) return BC_ERR_CUDA;
     if (di.cc_major != 10) return BC_ERR_UNSUPPORTED;
@@ -599,8 +786,17 @@ bc_status launch_gemm_packed(const GemmJob *jobs, int count, int64_t M,
         if (xa % 16 || wa % 16) return BC_ERR_ALIGNMENT;
         if (M >= (int64_t)1 << 31) return BC_ERR_UNSUPPORTED;
     }
-    if (M <= 128) return launch_bnx<128>(jobs, count, M, s, di.sm_count);
-    return launch_bnx<256>(jobs, count, M, s, di.sm_count);
+    if (packed)
+        return M <= 128 ? launch_cfg<128, kPacked>(jobs, count, M, bits, false, s, di.sm_count)
+                        : launch_cfg<256, kPacked>(jobs, count, M, bits, false, s, di.sm_count);
+    return M <= 128 ? launch_cfg<128, kRuntime>(jobs, count, M, bits, range, s, di.sm_count)
+                    : launch_cfg<256, kRuntime>(jobs, count, M, bits, range, s, di.sm_count);
+}
+
+bc_status gemm_set_wait_limit(long long cycles) {
+    if (cudaMemcpyToSymbol(g_gemm_wait_limit, &cycles, sizeof(cycles)) != cudaSuccess)
+        return BC_ERR_CUDA;
+    return BC_OK;
 }
 
 unsigned gemm_timeouts() {
