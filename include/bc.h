@@ -79,7 +79,12 @@ typedef enum bc_dtype { BC_F32 = 0, BC_F16 = 1, BC_BF16 = 2 } bc_dtype;
 
 typedef enum bc_mode {
     BC_MODE_RUNTIME = 0,      /* fp16 W re-quantized inline to `bits` (2..8), or 16 = passthrough */
-    BC_MODE_PACKED_INT4 = 1   /* pre-packed int4 codes, fp16 scale/zero per 64-block */
+    BC_MODE_PACKED_INT4 = 1,  /* pre-packed codes, fp16 scale/zero per 64-block: int4, or
+                                 2, 3 and 8 bits (bc_pack_codes) on the decode path */
+    BC_MODE_PACKED = 1,       /* the same mode under its width-neutral name */
+    BC_MODE_RUNTIME_RANGE = 2 /* as BC_MODE_RUNTIME, but `scales` holds each group's range
+                                 (bc_group_minmax) and the kernel derives scale and zero
+                                 for `bits` itself; `zeros` is unused (may be NULL) */
 } bc_mode;
 
 /* Per-channel grouping may be requested as group == K or group == 0. */
@@ -99,6 +104,22 @@ typedef enum bc_mode {
 BC_API bc_status bc_group_params(const void *W, int64_t N, int64_t K, int bits,
                           int64_t group, bc_dtype out_dtype, void *scales,
                           void *zeros, bc_stream_t stream);
+
+/*
+ * bc_group_minmax -- the bit-width-independent form of the precompute
+ * (BITCRUSH BC-06, "Under the hood": after the precompute, a change of bit
+ * width costs one kernel argument).  Stores each group's range, so that
+ * BC_MODE_RUNTIME_RANGE matmuls derive scale and zero for any `bits` from it
+ * with the fp32 arithmetic of bc_group_params: their codes are bit-identical
+ * to those of the (scale, zero) that bc_group_params(..., bits, ..., BC_F32)
+ * stores, and moving the lever reruns nothing.
+ *   W       fp16 [N][K], device
+ *   group   64, or K / 0 for per-channel
+ *   ranges  uint32 [N][K/group], device, written: fp16 min in the low half,
+ *           fp16 max in the high half (both exact: they are weights)
+ */
+BC_API bc_status bc_group_minmax(const void *W, int64_t N, int64_t K, int64_t group,
+                                 void *ranges, bc_stream_t stream);
 
 /*
  * bc_quantize_codes -- the RTN codes q = clamp(round(w/scale)+zero, 0, L)
@@ -127,14 +148,38 @@ BC_API bc_status bc_pack_int4(const void *W, const void *scales_f16,
                        uint8_t *packed, bc_stream_t stream);
 
 /*
+ * bc_pack_codes -- one-time packing at other code widths (Enargeia,
+ * "Honestly": an int8 tied embedding; BITCRUSH BC-06, "The machine", BRAIN
+ * SIZE: 2-bit weights), so that decode bytes fall with the bit width.
+ *   W                  fp16 [N][K], device
+ *   scales_f16, zeros_f16  fp16 [N][K/64] from bc_group_params(..., bits,
+ *                      64, BC_F16, ...)
+ *   bits               2, 3, 4 or 8
+ *   packed             uint8 [N][K*bits/8], device, written: each row a
+ *                      little-endian bit string, code k at bits
+ *                      [bits*k, bits*k + bits) (bits = 4 is bc_pack_int4's
+ *                      layout; a 64-group takes 8*bits bytes)
+ * Matmuls over these codes use BC_MODE_PACKED with the same `bits`; widths
+ * other than 4 take fp32 x (the decode GEMV, any M).
+ */
+BC_API bc_status bc_pack_codes(const void *W, const void *scales_f16,
+                               const void *zeros_f16, int64_t N, int64_t K, int bits,
+                               uint8_t *packed, bc_stream_t stream);
+
+/*
  * bc_matmul_q -- y = x . deq(W)^T (BITCRUSH BC-06 matmul_q; Enargeia int4
  * weights unpacked in registers).
- *   x, x_dtype   [M][K]: BC_F32 for any M; BC_BF16 only for M >= 64 in
- *                BC_MODE_PACKED_INT4 (tensor-core prefill, fp32 accumulate)
- *   W_or_packed  fp16 W [N][K] (runtime) or packed uint8 [N][K/2] (packed)
+ *   x, x_dtype   [M][K]: BC_F32 for any M; BC_BF16 for M >= 64 in every
+ *                mode (tensor-core prefill, fp32 accumulate: packed codes, or
+ *                fp16 weights re-quantized inline at 2..8 bits / passed
+ *                through at 16)
+ *   W_or_packed  fp16 W [N][K] (runtime) or packed uint8 [N][K*bits/8] (packed)
  *   scales, zeros  fp32 [N][K/group] (runtime) or fp16 [N][K/64] (packed);
+ *                BC_MODE_RUNTIME_RANGE: scales = uint32 ranges [N][K/group]
+ *                from bc_group_minmax, zeros unused;
  *                ignored (may be NULL) when bits == 16
- *   bits         runtime: 2..8 or 16 (fp16 passthrough); packed: 4
+ *   bits         runtime: 2..8 or 16 (fp16 passthrough); packed: 4, or 2, 3, 8
+ *                with fp32 x
  *   group        runtime: 64, or K / 0 (per channel); packed: 64
  *   y            fp32 [M][N], device, written (not accumulated into)
  *   workspace    device scratch of at least bc_workspace_size() bytes
@@ -144,7 +189,7 @@ BC_API bc_status bc_pack_int4(const void *W, const void *scales_f16,
  * can fill the GPU run the streaming decode kernels (M <= 4 on the int8
  * tensor cores; M = 5..16 on the tcgen05 decode kernel, packed or runtime at
  * 2..8 bits, whose workspace holds the split activations of each x); M >= 64
- * with bf16 x uses the tcgen05 tensor-core GEMM.
+ * with bf16 x uses the tcgen05 tensor-core GEMM (no workspace).
  */
 BC_API bc_status bc_matmul_q(const void *x, bc_dtype x_dtype, const void *W_or_packed,
                       const void *scales, const void *zeros, int64_t M,
@@ -255,6 +300,33 @@ BC_API bc_status bc_matmul_q_noalloc(const void *x, const void *W_or_packed,
                                      bc_stream_t stream);
 
 /*
+ * bc_matmul_q_argmax -- greedy token selection: for each row m of
+ * y = x . deq(W)^T, the index n of its largest value (ties go to the lowest
+ * index).  Enargeia ("One decode step"): a decode step ends in a single
+ * GPU -> CPU readback that carries one token id; BITCRUSH BC-06 ("Honest
+ * notes") decodes greedily.  Typically W is the LM head (Qwen3-0.6B's tied
+ * head: K = 1024, N = 151936, fp16 passthrough with bits = 16).
+ *   Arguments other than `token` mean what they mean for bc_matmul_q
+ *   (M <= 65535).
+ *   token      int32 [M], device, written
+ *   workspace  device scratch of at least bc_workspace_size_argmax() bytes,
+ *              256-byte aligned: it holds the logits (M x N fp32), the
+ *              reduction's partials and the matmul's own workspace; its
+ *              contents on entry do not matter
+ * Enqueues the matmul and two reduction kernels on `stream`.
+ */
+BC_API bc_status bc_matmul_q_argmax(const void *x, bc_dtype x_dtype, const void *W_or_packed,
+                                    const void *scales, const void *zeros, int64_t M,
+                                    int64_t N, int64_t K, int bits, int64_t group,
+                                    bc_mode mode, int32_t *token, void *workspace,
+                                    size_t workspace_bytes, bc_stream_t stream);
+
+/* Workspace bytes bc_matmul_q_argmax needs for this shape (0 if the shape
+ * would be rejected). */
+BC_API size_t bc_workspace_size_argmax(int64_t M, int64_t N, int64_t K, bc_mode mode,
+                                       bc_dtype x_dtype);
+
+/*
  * bc_device_timeouts -- number of bounded in-kernel waits (tensor-core
  * pipeline barriers) that ran out on the current device since the library
  * was loaded.  A kernel whose wait runs out stops early, frees its tensor
@@ -263,6 +335,17 @@ BC_API bc_status bc_matmul_q_noalloc(const void *x, const void *W_or_packed,
  * device.  `count` is a HOST pointer.
  */
 BC_API bc_status bc_device_timeouts(unsigned *count);
+
+/*
+ * bc_set_wait_limit -- limit of the bounded in-kernel pipeline waits on the
+ * current device, in SM clock cycles (0 restores the default of about 2 s,
+ * the maximum).  For tests of the failure path: a limit shorter than a
+ * pipeline stage makes the kernels' waits run out, so they record timeouts
+ * (bc_device_timeouts), stop early and leave their outputs incomplete --
+ * after waiting, with the default limit, for their own copies and MMAs in
+ * flight and freeing their tensor memory.  Synchronises the device.
+ */
+BC_API bc_status bc_set_wait_limit(uint64_t cycles);
 
 /* Static description of a status code. */
 BC_API const char *bc_status_string(bc_status status);

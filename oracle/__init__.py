@@ -37,8 +37,10 @@ def _load():
         P = ctypes.c_void_p
         lib.oracle_group_params.argtypes = [P, i64, i64, i32, i64, i32, P, P]
         lib.oracle_codes.argtypes = [P, P, P, i64, i64, i32, i64, P]
+        lib.oracle_group_range.argtypes = [P, i64, i64, i64, P, P]
         lib.oracle_dequant.argtypes = [P, P, P, i64, i64, i64, P]
         lib.oracle_pack_int4.argtypes = [P, i64, i64, P]
+        lib.oracle_pack_codes.argtypes = [P, i64, i64, i32, P]
         lib.oracle_matmul.argtypes = [P, P, i64, i64, i64, P, P]
         lib.oracle_half_rows_to_double.argtypes = [P, i64, P]
         lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
@@ -86,6 +88,17 @@ def group_params(W, bits: int, group: int, f16_storage: bool):
     return s, z
 
 
+def group_range(W, group: int):
+    """Exact (min, max) of every group, float64 arrays [N][K/group]."""
+    Wb = _half_bits(W)
+    N, K = Wb.shape
+    G = K // group
+    lo = np.empty((N, G), np.float64)
+    hi = np.empty((N, G), np.float64)
+    _load().oracle_group_range(_ptr(Wb), N, K, group, _ptr(lo), _ptr(hi))
+    return lo, hi
+
+
 def codes(W, s, z, bits: int, group: int):
     """uint8 codes [N][K] = clamp(rne(w/s) + z, 0, 2^bits-1)."""
     Wb = _half_bits(W)
@@ -114,6 +127,16 @@ def pack_int4(q):
     N, K = q.shape
     out = np.empty((N, K // 2), np.uint8)
     _load().oracle_pack_int4(_ptr(q), N, K, _ptr(out))
+    return out
+
+
+def pack_codes(q, bits: int):
+    """Packed bytes [N][K*bits/8]: each row a little-endian bit string, code
+    k at bits [bits*k, bits*k + bits)."""
+    q = np.ascontiguousarray(q, np.uint8)
+    N, K = q.shape
+    out = np.empty((N, K * bits // 8), np.uint8)
+    _load().oracle_pack_codes(_ptr(q), N, K, bits, _ptr(out))
     return out
 
 
@@ -150,7 +173,8 @@ def matmul_q(x, W, bits: int, group: int, mode: str):
 
     mode 'runtime': fp32 scale/zero recomputed from fp16 W (bits 2..8, or 16
                     for the fp16 passthrough);
-    mode 'packed' : int4 codes with fp16 scale/zero per 64-block.
+    mode 'packed' : packed codes (bits 2, 3, 4 or 8) with fp16 scale/zero per
+                    64-block.
     Returns dict with y, A (tolerance scale), codes, s, z, packed (packed
     mode only).
     """
@@ -164,7 +188,7 @@ def matmul_q(x, W, bits: int, group: int, mode: str):
         wq = dequant(q, s, z, group)
         out.update(s=s, z=z, codes=q)
         if f16:
-            out["packed"] = pack_int4(q)
+            out["packed"] = pack_int4(q) if bits == 4 else pack_codes(q, bits)
     y, a = matmul(x, wq)
     out.update(y=y, A=a, wq=wq)
     return out

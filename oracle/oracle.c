@@ -137,6 +137,33 @@ void oracle_group_params(const uint16_t *W, int64_t N, int64_t K, int bits,
     }
 }
 
+/* ---- step 1 alone: the group range ---------------------------------------- */
+/*
+ * The bit-width-independent precompute (BITCRUSH BC-06, "Under the hood":
+ * after the precompute a change of bit width costs one argument): the
+ * exact (min, max) of every group, from which steps 2-4 give the scale and
+ * zero of any bit width.
+ * lo, hi : [N][K/group] doubles (exact fp16 values)
+ */
+void oracle_group_range(const uint16_t *W, int64_t N, int64_t K, int64_t group,
+                        double *lo_out, double *hi_out)
+{
+    const int64_t G = K / group;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t j = 0; j < G; ++j) {
+            double lo = INFINITY, hi = -INFINITY;
+            for (int64_t k = j * group; k < (j + 1) * group; ++k) {
+                double w = oracle_half_to_double(W[n * K + k]);
+                if (w < lo) lo = w;
+                if (w > hi) hi = w;
+            }
+            lo_out[n * G + j] = lo;
+            hi_out[n * G + j] = hi;
+        }
+    }
+}
+
 /* ---- step 5: codes ------------------------------------------------------ */
 /* q = clamp(round-half-even(w / s) + z, 0, L) with the exact quotient. */
 void oracle_codes(const uint16_t *W, const double *s, const double *z,
@@ -178,6 +205,30 @@ void oracle_pack_int4(const uint8_t *q, int64_t N, int64_t K, uint8_t *packed)
         for (int64_t k = 0; k < K; k += 2)
             packed[n * (K / 2) + k / 2] =
                 (uint8_t)((q[n * K + k] & 0xf) | ((q[n * K + k + 1] & 0xf) << 4));
+}
+
+/* ---- step 9, any width: packed codes of `bits` bits ------------------------ */
+/*
+ * Other packed widths (Enargeia, "Honestly": an int8 tied embedding;
+ * BITCRUSH BC-06, "The machine", BRAIN SIZE: 2-bit weights): each row is one
+ * little-endian bit string in which code k occupies bits [bits*k,
+ * bits*k + bits).  For bits = 4 this is the int4 layout above (low nibble =
+ * even k); for bits = 8 one byte per code; a 64-group takes 8*bits bytes.
+ * packed : [N][K*bits/8]
+ */
+void oracle_pack_codes(const uint8_t *q, int64_t N, int64_t K, int bits, uint8_t *packed)
+{
+    const int64_t rb = K * bits / 8;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t b = 0; b < rb; ++b) packed[n * rb + b] = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            for (int i = 0; i < bits; ++i) {
+                const int64_t bit = k * bits + i;               /* position in the row */
+                if ((q[n * K + k] >> i) & 1)
+                    packed[n * rb + bit / 8] |= (uint8_t)(1u << (bit % 8));
+            }
+        }
+    }
 }
 
 /* ---- step 8: y = x . w'^T in fp64, plus the tolerance scale A ----------- */

@@ -23,16 +23,19 @@ LIB_PATH = os.path.join(_HERE, "libbc.so")
 BC_OK, BC_ERR_INVALID_ARG, BC_ERR_UNSUPPORTED, BC_ERR_ALIGNMENT, \
     BC_ERR_WORKSPACE, BC_ERR_CUDA = range(6)
 BC_F32, BC_F16, BC_BF16 = 0, 1, 2
-BC_MODE_RUNTIME, BC_MODE_PACKED_INT4 = 0, 1
+BC_MODE_RUNTIME, BC_MODE_PACKED_INT4, BC_MODE_RUNTIME_RANGE = 0, 1, 2
+BC_MODE_PACKED = BC_MODE_PACKED_INT4
 GROUP_PER_CHANNEL = 0
 BC_FLAG_STATIC_WEIGHTS = 1
 
 # Every symbol include/bc.h declares.
-EXPORTS = ("bc_group_params", "bc_quantize_codes", "bc_pack_int4",
+EXPORTS = ("bc_group_params", "bc_group_minmax", "bc_quantize_codes", "bc_pack_int4",
+           "bc_pack_codes",
            "bc_matmul_q", "bc_workspace_size", "bc_matmul_q_batched",
            "bc_matmul_q_batched_ex",
            "bc_workspace_size_batched", "bc_matmul_q_noalloc",
-           "bc_device_timeouts",
+           "bc_matmul_q_argmax", "bc_workspace_size_argmax",
+           "bc_device_timeouts", "bc_set_wait_limit",
            "bc_status_string", "bc_version")
 
 
@@ -58,7 +61,11 @@ def _load() -> ctypes.CDLL:
     P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     lib.bc_group_params.argtypes = [P, i64, i64, i32, i64, i32, P, P, P]
     lib.bc_quantize_codes.argtypes = [P, P, P, i32, i64, i64, i32, i64, P, P]
+    lib.bc_group_minmax.argtypes = [P, i64, i64, i64, P, P]
+    lib.bc_group_minmax.restype = i32
     lib.bc_pack_int4.argtypes = [P, P, P, i64, i64, P, P]
+    lib.bc_pack_codes.argtypes = [P, P, P, i64, i64, i32, P, P]
+    lib.bc_pack_codes.restype = i32
     lib.bc_matmul_q.argtypes = [P, i32, P, P, P, i64, i64, i64, i32, i64, i32,
                                 P, P, sz, P]
     lib.bc_workspace_size.argtypes = [i64, i64, i64, i32]
@@ -73,6 +80,13 @@ def _load() -> ctypes.CDLL:
     lib.bc_matmul_q_noalloc.argtypes = [P, P, P, P, i64, i64, i64, i32, i64,
                                         i32, P, P]
     lib.bc_matmul_q_noalloc.restype = i32
+    lib.bc_matmul_q_argmax.argtypes = [P, i32, P, P, P, i64, i64, i64, i32, i64, i32,
+                                       P, P, sz, P]
+    lib.bc_matmul_q_argmax.restype = i32
+    lib.bc_workspace_size_argmax.argtypes = [i64, i64, i64, i32, i32]
+    lib.bc_workspace_size_argmax.restype = sz
+    lib.bc_set_wait_limit.argtypes = [ctypes.c_uint64]
+    lib.bc_set_wait_limit.restype = i32
     lib.bc_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     lib.bc_device_timeouts.restype = i32
     lib.bc_status_string.argtypes = [i32]
@@ -130,6 +144,19 @@ def group_params(W: torch.Tensor, bits: int, group: int, out_dtype=torch.float32
     return scales, zeros
 
 
+def group_minmax(W: torch.Tensor, group: int, ranges: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """Per-group range of fp16 W [N][K] as int32 words [N][K/group] (fp16 min
+    in the low half, fp16 max in the high half), for BC_MODE_RUNTIME_RANGE."""
+    N, K = W.shape
+    g = K if group in (0, K) else group
+    if ranges is None:
+        ranges = torch.empty((N, K // g), dtype=torch.int32, device=W.device)
+    _check(lib.bc_group_minmax(_ptr(W), N, K, group, _ptr(ranges), _stream(stream)),
+           "bc_group_minmax")
+    return ranges
+
+
 def quantize_codes(W: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
                    bits: int, group: int, codes: Optional[torch.Tensor] = None,
                    stream=None) -> torch.Tensor:
@@ -150,6 +177,17 @@ def pack_int4(W: torch.Tensor, scales_f16: torch.Tensor, zeros_f16: torch.Tensor
         packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
     _check(lib.bc_pack_int4(_ptr(W), _ptr(scales_f16), _ptr(zeros_f16), N, K,
                             _ptr(packed), _stream(stream)), "bc_pack_int4")
+    return packed
+
+
+def pack_codes(W: torch.Tensor, scales_f16: torch.Tensor, zeros_f16: torch.Tensor,
+               bits: int, packed: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Packed codes of `bits` (2, 3, 4, 8) bits: uint8 [N][K*bits/8]."""
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty((N, K * bits // 8), dtype=torch.uint8, device=W.device)
+    _check(lib.bc_pack_codes(_ptr(W), _ptr(scales_f16), _ptr(zeros_f16), N, K, bits,
+                             _ptr(packed), _stream(stream)), "bc_pack_codes")
     return packed
 
 
@@ -217,6 +255,11 @@ def device_timeouts() -> int:
     return int(c.value)
 
 
+def set_wait_limit(cycles: int) -> None:
+    """bc_set_wait_limit: the in-kernel wait limit in cycles (0 = default)."""
+    _check(lib.bc_set_wait_limit(int(cycles)), "bc_set_wait_limit")
+
+
 def matmul_q_noalloc(x: torch.Tensor, W: torch.Tensor,
                      scales: Optional[torch.Tensor], zeros: Optional[torch.Tensor],
                      bits: int, group: int, mode: int, y: torch.Tensor,
@@ -239,3 +282,27 @@ def matmul_q_noalloc(x: torch.Tensor, W: torch.Tensor,
                                    M, N, K, bits, group, mode, _ptr(y),
                                    _stream(stream)), "bc_matmul_q_noalloc")
     return y
+
+
+def workspace_size_argmax(M: int, N: int, K: int, mode: int, x_dtype: int = BC_F32) -> int:
+    return int(lib.bc_workspace_size_argmax(M, N, K, mode, x_dtype))
+
+
+def matmul_q_argmax(x: torch.Tensor, W: torch.Tensor, scales: Optional[torch.Tensor],
+                    zeros: Optional[torch.Tensor], bits: int, group: int, mode: int,
+                    token: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """bc_matmul_q_argmax: int32 [M], per row of x the index of the largest
+    output of x . deq(W)^T (lowest index among equal values)."""
+    M, K = x.shape
+    N = W.shape[0]
+    if token is None:
+        token = torch.empty((M,), dtype=torch.int32, device=x.device)
+    need = workspace_size_argmax(M, N, K, mode, _DT[x.dtype])
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    _check(lib.bc_matmul_q_argmax(_ptr(x), _DT[x.dtype], _ptr(W), _ptr(scales), _ptr(zeros),
+                                  M, N, K, bits, group, mode, _ptr(token), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(),
+                                  _stream(stream)), "bc_matmul_q_argmax")
+    return token

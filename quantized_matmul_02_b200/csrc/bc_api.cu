@@ -4,6 +4,7 @@
 // caller's stream.  Nothing here allocates device memory or synchronises.
 #include "bc_internal.cuh"
 
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
@@ -45,13 +46,19 @@ namespace {
 bc_status check_matmul_common(int64_t M, int bits, int64_t group_norm,
                               bc_mode mode, bc_dtype x_dtype) {
     if (M <= 0 || M > (int64_t)1 << 24) return BC_ERR_INVALID_ARG;
-    if (mode == BC_MODE_RUNTIME) {
+    if (mode == BC_MODE_RUNTIME || mode == BC_MODE_RUNTIME_RANGE) {
         if (!((bits >= 2 && bits <= 8) || bits == 16)) return BC_ERR_UNSUPPORTED;
-        if (x_dtype != BC_F32) return BC_ERR_UNSUPPORTED;
-    } else if (mode == BC_MODE_PACKED_INT4) {
-        if (bits != 4 || group_norm != 64) return BC_ERR_UNSUPPORTED;
         if (x_dtype == BC_BF16) {
             if (M < 64) return BC_ERR_UNSUPPORTED;
+        } else if (x_dtype != BC_F32) {
+            return BC_ERR_UNSUPPORTED;
+        }
+    } else if (mode == BC_MODE_PACKED_INT4) {
+        // packed codes: int4 everywhere; 2, 3 and 8 bits on the decode GEMV
+        if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8) || group_norm != 64)
+            return BC_ERR_UNSUPPORTED;
+        if (x_dtype == BC_BF16) {
+            if (M < 64 || bits != 4) return BC_ERR_UNSUPPORTED;
         } else if (x_dtype != BC_F32) {
             return BC_ERR_UNSUPPORTED;
         }
@@ -80,14 +87,15 @@ bc_status check_matmul_ptrs(const void *x, bc_dtype x_dtype, const void *w,
                             const void *s, const void *z, const float *y,
                             int bits, bc_mode mode) {
     if (!x || !w || !y) return BC_ERR_INVALID_ARG;
-    const bool need_sz = !(mode == BC_MODE_RUNTIME && bits == 16);
-    if (need_sz && (!s || !z)) return BC_ERR_INVALID_ARG;
+    const bool need_sz = !(mode != BC_MODE_PACKED_INT4 && bits == 16);
+    const bool need_z = need_sz && mode != BC_MODE_RUNTIME_RANGE;   // ranges: one array
+    if ((need_sz && !s) || (need_z && !z)) return BC_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(w, 16) || !aligned(y, 4))
         return BC_ERR_ALIGNMENT;
     (void)x_dtype;
     if (need_sz) {
-        const size_t a = mode == BC_MODE_RUNTIME ? 4 : 2;
-        if (!aligned(s, a) || !aligned(z, a)) return BC_ERR_ALIGNMENT;
+        const size_t a = mode == BC_MODE_PACKED_INT4 ? 2 : 4;
+        if (!aligned(s, a) || (need_z && !aligned(z, a))) return BC_ERR_ALIGNMENT;
     }
     return BC_OK;
 }
@@ -122,6 +130,15 @@ bc_status bc_device_timeouts(unsigned *count) {
     return BC_OK;
 }
 
+bc_status bc_set_wait_limit(uint64_t cycles) {
+    const long long v = cycles == 0 ? 4000000000LL
+                                    : (long long)std::min<uint64_t>(cycles, 4000000000ull);
+    if (cudaDeviceSynchronize() != cudaSuccess) return BC_ERR_CUDA;
+    bc_status st = gemv_set_wait_limit(v);
+    if (st == BC_OK) st = gemm_set_wait_limit(v);
+    return st;
+}
+
 bc_status bc_group_params(const void *W, int64_t N, int64_t K, int bits,
                           int64_t group, bc_dtype out_dtype, void *scales,
                           void *zeros, bc_stream_t stream) {
@@ -137,6 +154,18 @@ bc_status bc_group_params(const void *W, int64_t N, int64_t K, int bits,
         return BC_ERR_ALIGNMENT;
     return launch_group_params(static_cast<const __half *>(W), N, K, bits, g,
                                out_dtype == BC_F16, scales, zeros,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+bc_status bc_group_minmax(const void *W, int64_t N, int64_t K, int64_t group,
+                          void *ranges, bc_stream_t stream) {
+    if (!W || !ranges) return BC_ERR_INVALID_ARG;
+    bc_status st = check_nk(N, K);
+    if (st != BC_OK) return st;
+    const int64_t g = normalize_group(group, K);
+    if (g < 0) return BC_ERR_UNSUPPORTED;
+    if (!aligned(W, 16) || !aligned(ranges, 4)) return BC_ERR_ALIGNMENT;
+    return launch_group_minmax(static_cast<const __half *>(W), N, K, g, ranges,
                                reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -173,6 +202,21 @@ bc_status bc_pack_int4(const void *W, const void *scales_f16,
                             static_cast<const __half *>(scales_f16),
                             static_cast<const __half *>(zeros_f16), N, K,
                             packed, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bc_status bc_pack_codes(const void *W, const void *scales_f16, const void *zeros_f16,
+                        int64_t N, int64_t K, int bits, uint8_t *packed, bc_stream_t stream) {
+    if (!W || !scales_f16 || !zeros_f16 || !packed) return BC_ERR_INVALID_ARG;
+    bc_status st = check_nk(N, K);
+    if (st != BC_OK) return st;
+    if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8)) return BC_ERR_UNSUPPORTED;
+    if (!aligned(W, 16) || !aligned(scales_f16, 2) || !aligned(zeros_f16, 2) ||
+        !aligned(packed, 16))
+        return BC_ERR_ALIGNMENT;
+    return launch_pack_codes(static_cast<const __half *>(W),
+                             static_cast<const __half *>(scales_f16),
+                             static_cast<const __half *>(zeros_f16), N, K, bits, packed,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t bc_workspace_size_batched(const bc_matmul_desc *descs, int count,
@@ -230,13 +274,12 @@ bc_status bc_matmul_q_batched_ex(const bc_matmul_desc *descs, int count,
         std::vector<GemmJob> jobs(count);
         for (int i = 0; i < count; ++i) {
             const bc_matmul_desc &d = descs[i];
-            jobs[i] = GemmJob{static_cast<const __nv_bfloat16 *>(d.x),
-                              static_cast<const uint8_t *>(d.W_or_packed),
-                              static_cast<const __half *>(d.scales),
-                              static_cast<const __half *>(d.zeros), d.y, d.N,
-                              d.K};
+            jobs[i] = GemmJob{static_cast<const __nv_bfloat16 *>(d.x), d.W_or_packed,
+                              d.scales, d.zeros, d.y, d.N, d.K,
+                              group == 64 ? (int64_t)64 : d.K};
         }
-        return launch_gemm_packed(jobs.data(), count, M, s);
+        return launch_gemm(jobs.data(), count, M, mode == BC_MODE_PACKED_INT4, bits,
+                           mode == BC_MODE_RUNTIME_RANGE, s);
     }
     if (workspace_bytes && !workspace) return BC_ERR_INVALID_ARG;
     if (workspace && !aligned(workspace, 256)) return BC_ERR_ALIGNMENT;
@@ -245,8 +288,11 @@ bc_status bc_matmul_q_batched_ex(const bc_matmul_desc *descs, int count,
         const bc_matmul_desc &d = descs[i];
         jobs[i] = GemvJob{static_cast<const float *>(d.x), d.W_or_packed,
                           d.scales, d.zeros, d.y, d.N, d.K,
-                          group == 64 ? (int64_t)64 : d.K};
+                          group == 64 ? (int64_t)64 : d.K,
+                          mode == BC_MODE_RUNTIME_RANGE ? (int64_t)1 : (int64_t)0};
     }
+    if (mode == BC_MODE_PACKED_INT4 && bits != 4)
+        return launch_gemv_packed(jobs.data(), count, (int)M, bits, s);
     return launch_gemv(jobs.data(), count, (int)M, bits,
                        mode == BC_MODE_PACKED_INT4, workspace, workspace_bytes,
                        s, (flags & BC_FLAG_STATIC_WEIGHTS) != 0);
@@ -265,6 +311,39 @@ bc_status bc_matmul_q(const void *x, bc_dtype x_dtype, const void *W_or_packed,
     return bc_matmul_q_batched(&d, 1, M, bits,
                                g == 64 ? 64 : BC_GROUP_PER_CHANNEL, mode,
                                x_dtype, workspace, workspace_bytes, stream);
+}
+
+size_t bc_workspace_size_argmax(int64_t M, int64_t N, int64_t K, bc_mode mode,
+                                bc_dtype x_dtype) {
+    if (M <= 0 || M > 65535 || N <= 0 || K <= 0 || check_nk(N, K) != BC_OK) return 0;
+    const size_t yb = ((size_t)M * N * 4 + 255) / 256 * 256;
+    const size_t gemv = x_dtype == BC_F32 ? bc_workspace_size(M, N, K, mode) : 0;
+    return yb + argmax_partials_bytes(M, N) + gemv;
+}
+
+bc_status bc_matmul_q_argmax(const void *x, bc_dtype x_dtype, const void *W_or_packed,
+                             const void *scales, const void *zeros, int64_t M,
+                             int64_t N, int64_t K, int bits, int64_t group,
+                             bc_mode mode, int32_t *token, void *workspace,
+                             size_t workspace_bytes, bc_stream_t stream) {
+    if (!token) return BC_ERR_INVALID_ARG;
+    if (!aligned(token, 4)) return BC_ERR_ALIGNMENT;
+    bc_status st = check_nk(N, K);
+    if (st != BC_OK) return st;
+    if (M <= 0 || M > 65535) return BC_ERR_INVALID_ARG;
+    const size_t need = bc_workspace_size_argmax(M, N, K, mode, x_dtype);
+    if (!workspace || workspace_bytes < need) return BC_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BC_ERR_ALIGNMENT;
+    // scratch: logits y [M][N], then the reduction's partials, then the
+    // matmul's own workspace
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const size_t yb = ((size_t)M * N * 4 + 255) / 256 * 256;
+    const size_t pb = argmax_partials_bytes(M, N);
+    float *y = reinterpret_cast<float *>(ws);
+    st = bc_matmul_q(x, x_dtype, W_or_packed, scales, zeros, M, N, K, bits, group, mode, y,
+                     ws + yb + pb, workspace_bytes - yb - pb, stream);
+    if (st != BC_OK) return st;
+    return launch_argmax(y, M, N, ws + yb, token, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

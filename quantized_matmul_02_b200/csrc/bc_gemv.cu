@@ -22,6 +22,7 @@
 // to the caller's workspace; the last CTA to finish a row block (ticket
 // counter) sums the partials in split order, so results are deterministic.
 #include "bc_internal.cuh"
+#include "bc_rtn.cuh"
 
 #include <algorithm>
 #include <vector>
@@ -51,6 +52,7 @@ struct JobDev {
 
 struct GemvParams {
     int count, total_items, M, bits;
+    int range;             // runtime mode: (scale, zero) derived from stored ranges
     float *ws_partial;
     unsigned *ws_ticket;
     JobDev jobs[kMaxJobs];
@@ -208,8 +210,16 @@ gemv_kernel(const __grid_constant__ GemvParams P) {
                     } else {
                         float s = 1.0f, z = 0.0f;
                         if (!passthrough) {
-                            s = __ldg(reinterpret_cast<const float *>(J.s) + gi);
-                            z = __ldg(reinterpret_cast<const float *>(J.z) + gi);
+                            if (P.range) {
+                                const float2 r = range_of_word(
+                                    __ldg(reinterpret_cast<const uint32_t *>(J.s) + gi));
+                                const float2 sz = rtn_params_from_range(r.x, r.y, P.bits);
+                                s = sz.x;
+                                z = sz.y;
+                            } else {
+                                s = __ldg(reinterpret_cast<const float *>(J.s) + gi);
+                                z = __ldg(reinterpret_cast<const float *>(J.z) + gi);
+                            }
                         }
                         float cq[8];
                         runtime_codes(raw[u], s, z, L, passthrough, cq);
@@ -424,6 +434,7 @@ bc_status launch_gemv(const GemvJob *jobs, int count, int M, int bits,
             Q.total_items = p.total_items;
             Q.M = mrows;
             Q.bits = bits;
+            Q.range = (int)jobs[0].range;
             Q.ws_partial = reinterpret_cast<float *>(workspace);
             Q.ws_ticket = nullptr;
             if (p.tickets) {

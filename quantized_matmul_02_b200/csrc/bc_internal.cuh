@@ -36,6 +36,9 @@ inline bc_status cuda_status() {
 bc_status launch_group_params(const __half *W, int64_t N, int64_t K, int bits,
                               int64_t group, bool f16_out, void *scales,
                               void *zeros, cudaStream_t s);
+// Per-group range (fp16 min, fp16 max) as one 32-bit word per group.
+bc_status launch_group_minmax(const __half *W, int64_t N, int64_t K, int64_t group,
+                              void *minmax, cudaStream_t s);
 bc_status launch_quantize_codes(const __half *W, const void *scales,
                                 const void *zeros, bool f16_sz, int64_t N,
                                 int64_t K, int bits, int64_t group,
@@ -43,6 +46,9 @@ bc_status launch_quantize_codes(const __half *W, const void *scales,
 bc_status launch_pack_int4(const __half *W, const __half *scales,
                            const __half *zeros, int64_t N, int64_t K,
                            uint8_t *packed, cudaStream_t s);
+// Packed codes of 2, 3, 4 or 8 bits (row = little-endian bit string).
+bc_status launch_pack_codes(const __half *W, const __half *scales, const __half *zeros,
+                            int64_t N, int64_t K, int bits, uint8_t *packed, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Fused dequant GEMV (bc_gemv.cu), M < 64, fp32 x
@@ -55,6 +61,8 @@ struct GemvJob {             // one matrix of a launch
     float *y;                // [M][N]
     int64_t N, K;
     int64_t group;           // 64 or K
+    int64_t range;           // runtime mode: s holds per-group ranges (fp16 min|max)
+                             // and z is unused; the same for every job of a call
 };
 // Streaming decode kernels (bc_gemv_stream.cu): M <= 4 on the mma.sync
 // streaming kernel; M = 5..16 on the tcgen05 decode kernel (packed, or
@@ -71,6 +79,10 @@ bc_status launch_gemv_stream(const GemvJob *jobs, int count, int M, int bits,
                              bool packed, cudaStream_t s, bool early_start, void *workspace,
                              size_t ws_bytes);
 unsigned gemv_timeouts();
+bc_status gemv_set_wait_limit(long long cycles);
+// Decode GEMV over packed codes of 2, 3 or 8 bits (bc_gemv_packed.cu;
+// fp32 x, any M).
+bc_status launch_gemv_packed(const GemvJob *jobs, int count, int M, int bits, cudaStream_t s);
 // Bytes of split-K scratch a launch over these jobs needs.
 size_t gemv_workspace_bytes(const GemvJob *jobs, int count, int M, bool packed,
                             int sm_count);
@@ -79,19 +91,31 @@ bc_status launch_gemv(const GemvJob *jobs, int count, int M, int bits,
                       cudaStream_t s, bool early_start = false);
 
 // ---------------------------------------------------------------------------
-// tcgen05 prefill GEMM (bc_gemm_sm100.cu), packed int4 W, bf16 x, M >= 64
+// Greedy token selection (bc_argmax.cu): per row of y [M][N] the index of
+// the largest value, ties to the lowest index.
+// ---------------------------------------------------------------------------
+// Scratch of the reduction (partials), 256-byte multiple.
+size_t argmax_partials_bytes(int64_t M, int64_t N);
+bc_status launch_argmax(const float *y, int64_t M, int64_t N, void *partials,
+                        int32_t *token, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// tcgen05 prefill GEMM (bc_gemm_sm100.cu), bf16 x, M >= 64: packed int4 W,
+// or fp16 W re-quantized inline (runtime mode)
 // ---------------------------------------------------------------------------
 struct GemmJob {
     const __nv_bfloat16 *x;  // [M][K]
-    const uint8_t *w;        // packed [N][K/2]
-    const __half *s;         // [N][K/64]
-    const __half *z;
+    const void *w;           // packed [N][K/2] or fp16 [N][K]
+    const void *s;           // fp16 [N][K/64] | fp32 [N][K/group] | ranges
+    const void *z;           // fp16 | fp32 | unused (ranges)
     float *y;                // [M][N]
     int64_t N, K;
+    int64_t group;           // 64, or K (runtime per channel)
 };
-bc_status launch_gemm_packed(const GemmJob *jobs, int count, int64_t M,
-                             cudaStream_t s);
+bc_status launch_gemm(const GemmJob *jobs, int count, int64_t M, bool packed, int bits,
+                      bool range, cudaStream_t s);
 // Bounded waits of the GEMM that ran out on the current device since load.
 unsigned gemm_timeouts();
+bc_status gemm_set_wait_limit(long long cycles);
 
 }  // namespace bc

@@ -11,6 +11,7 @@
 // read).  Each lane moves 16-byte vectors; a 64-weight group is 128 bytes,
 // i.e. 8 lanes, so one warp covers four groups per load.
 #include "bc_internal.cuh"
+#include "bc_rtn.cuh"
 
 namespace bc {
 namespace {
@@ -42,10 +43,7 @@ __device__ __forceinline__ void half8_to_float(const uint4 &v, float (&f)[8]) {
 __device__ __forceinline__ void rtn_params(float lo, float hi, int bits,
                                            bool f16, float &s, float &z) {
     const float L = (float)((1 << bits) - 1);
-    if (hi == lo)
-        s = (lo == 0.0f) ? 1.0f : fabsf(lo);
-    else
-        s = __fdiv_rn(__fsub_rn(hi, lo), L);
+    s = rtn_scale(lo, hi, L);
     if (f16) {
         s = __half2float(__float2half_rn(s));
         if (s < 5.9604644775390625e-08f) s = 5.9604644775390625e-08f;  // 2^-24
@@ -64,7 +62,9 @@ __device__ __forceinline__ int rtn_code_exact(float w, float s, float z, int L) 
 }
 
 // LPG lanes share one group; lane handles chunks (lane % LPG) + LPG*i.
-template <int LPG>
+// RANGE: store the group's range instead (fp16 min | fp16 max << 16 in one
+// word of `scales`; bits, f16 and zeros unused).
+template <int LPG, bool RANGE>
 __global__ void __launch_bounds__(kThreads)
 group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t K,
                     int64_t group, int bits, bool f16, void *scales,
@@ -94,6 +94,13 @@ group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t K,
     for (int off = LPG / 2; off > 0; off >>= 1) {
         lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
         hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (RANGE) {
+        if (valid && sub == 0) {
+            const __half2 r = __halves2half2(__float2half_rn(lo), __float2half_rn(hi));
+            reinterpret_cast<__half2 *>(scales)[gi] = r;      // exact: fp16 values
+        }
+        return;
     }
     if (valid && sub == 0) {
         float s, z;
@@ -164,6 +171,51 @@ pack_int4_kernel(const __half *__restrict__ W, const __half *__restrict__ S,
     *reinterpret_cast<uint2 *>(packed + e / 2) = make_uint2(w0, w1);
 }
 
+// Packed codes of 2, 3 or 8 bits: one thread per 64-group.  The row is a
+// little-endian bit string, code k at bits [BITS k, BITS k + BITS); the
+// group's 8 BITS bytes are built as 2 BITS words and stored with aligned
+// vector stores (8-byte for 3 bits, 16-byte otherwise).
+template <int BITS>
+__global__ void __launch_bounds__(kThreads)
+pack_codes_kernel(const __half *__restrict__ W, const __half *__restrict__ S,
+                  const __half *__restrict__ Z, int64_t N, int64_t K,
+                  uint8_t *__restrict__ packed) {
+    const int64_t gi = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    const int64_t G = K / 64;
+    if (gi >= N * G) return;
+    const int64_t n = gi / G, g = gi % G;
+    const float s = __half2float(S[gi]);
+    const float z = __half2float(Z[gi]);
+    constexpr int L = (1 << BITS) - 1;
+    uint32_t w[2 * BITS];
+#pragma unroll
+    for (int i = 0; i < 2 * BITS; ++i) w[i] = 0;
+    const __half *src = W + n * K + g * 64;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        float f[8];
+        half8_to_float(ld_stream(src + 8 * c), f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int k = 8 * c + i, pos = BITS * k, wi = pos >> 5, sh = pos & 31;
+            const uint32_t q = (uint32_t)rtn_code_exact(f[i], s, z, L);
+            w[wi] |= q << sh;
+            if (sh + BITS > 32) w[wi + 1] |= q >> (32 - sh);
+        }
+    }
+    uint8_t *dst = packed + n * (K / 8) * BITS + g * 8 * BITS;
+    if constexpr (BITS == 3) {
+#pragma unroll
+        for (int i = 0; i < 3; ++i)
+            reinterpret_cast<uint2 *>(dst)[i] = make_uint2(w[2 * i], w[2 * i + 1]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < BITS / 2; ++i)
+            reinterpret_cast<uint4 *>(dst)[i] =
+                make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    }
+}
+
 inline unsigned blocks_for(int64_t threads) {
     return (unsigned)((threads + kThreads - 1) / kThreads);
 }
@@ -175,11 +227,24 @@ bc_status launch_group_params(const __half *W, int64_t N, int64_t K, int bits,
                               void *zeros, cudaStream_t s) {
     const int64_t ngroups = N * (K / group);
     if (group == 64) {
-        group_params_kernel<8><<<blocks_for(ngroups * 8), kThreads, 0, s>>>(
+        group_params_kernel<8, false><<<blocks_for(ngroups * 8), kThreads, 0, s>>>(
             W, N, K, group, bits, f16_out, scales, zeros);
     } else {
-        group_params_kernel<32><<<blocks_for(ngroups * 32), kThreads, 0, s>>>(
+        group_params_kernel<32, false><<<blocks_for(ngroups * 32), kThreads, 0, s>>>(
             W, N, K, group, bits, f16_out, scales, zeros);
+    }
+    return cuda_status();
+}
+
+bc_status launch_group_minmax(const __half *W, int64_t N, int64_t K, int64_t group,
+                              void *minmax, cudaStream_t s) {
+    const int64_t ngroups = N * (K / group);
+    if (group == 64) {
+        group_params_kernel<8, true><<<blocks_for(ngroups * 8), kThreads, 0, s>>>(
+            W, N, K, group, 2, false, minmax, nullptr);
+    } else {
+        group_params_kernel<32, true><<<blocks_for(ngroups * 32), kThreads, 0, s>>>(
+            W, N, K, group, 2, false, minmax, nullptr);
     }
     return cuda_status();
 }
@@ -190,6 +255,19 @@ bc_status launch_quantize_codes(const __half *W, const void *scales,
                                 uint8_t *codes, cudaStream_t s) {
     codes_kernel<<<blocks_for(N * K / 8), kThreads, 0, s>>>(
         W, scales, zeros, f16_sz, N, K, group, bits, codes);
+    return cuda_status();
+}
+
+bc_status launch_pack_codes(const __half *W, const __half *scales, const __half *zeros,
+                            int64_t N, int64_t K, int bits, uint8_t *packed, cudaStream_t s) {
+    if (bits == 4) return launch_pack_int4(W, scales, zeros, N, K, packed, s);
+    const unsigned blocks = blocks_for(N * (K / 64));
+    if (bits == 2)
+        pack_codes_kernel<2><<<blocks, kThreads, 0, s>>>(W, scales, zeros, N, K, packed);
+    else if (bits == 3)
+        pack_codes_kernel<3><<<blocks, kThreads, 0, s>>>(W, scales, zeros, N, K, packed);
+    else
+        pack_codes_kernel<8><<<blocks, kThreads, 0, s>>>(W, scales, zeros, N, K, packed);
     return cuda_status();
 }
 

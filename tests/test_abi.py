@@ -52,14 +52,20 @@ FAKE = 0x10000  # 16-byte aligned non-null address: never dereferenced
     ((FAKE, 0, FAKE, FAKE, FAKE, 1, 8, 96, 4, 64, 0, FAKE, None, 0, None), 1),
     # bits 9 (the lever goes 16 -> 2; 9..15 are not offered)
     ((FAKE, 0, FAKE, FAKE, FAKE, 1, 8, 64, 9, 64, 0, FAKE, None, 0, None), 2),
-    # packed mode with bits != 4
-    ((FAKE, 0, FAKE, FAKE, FAKE, 1, 8, 64, 3, 64, 1, FAKE, None, 0, None), 2),
+    # packed mode at a width that is not packed (2, 3, 4 and 8 are)
+    ((FAKE, 0, FAKE, FAKE, FAKE, 1, 8, 64, 5, 64, 1, FAKE, None, 0, None), 2),
     # group 32 is not offered
     ((FAKE, 0, FAKE, FAKE, FAKE, 1, 8, 128, 4, 32, 0, FAKE, None, 0, None), 2),
     # bf16 x below M=64
     ((FAKE, 2, FAKE, FAKE, FAKE, 8, 8, 64, 4, 64, 1, FAKE, None, 0, None), 2),
-    # bf16 x in runtime mode
-    ((FAKE, 2, FAKE, FAKE, FAKE, 128, 8, 64, 4, 64, 0, FAKE, None, 0, None), 2),
+    # fp16 x is not offered (fp32 decode, bf16 prefill)
+    ((FAKE, 1, FAKE, FAKE, FAKE, 128, 8, 64, 4, 64, 0, FAKE, None, 0, None), 2),
+    # bf16 x in runtime mode below M = 64
+    ((FAKE, 2, FAKE, FAKE, FAKE, 32, 8, 64, 4, 64, 0, FAKE, None, 0, None), 2),
+    # range mode without the ranges
+    ((FAKE, 0, FAKE, None, None, 1, 8, 64, 4, 64, 2, FAKE, None, 0, None), 1),
+    # no such mode
+    ((FAKE, 0, FAKE, FAKE, FAKE, 1, 8, 64, 4, 64, 7, FAKE, None, 0, None), 2),
     # misaligned x
     ((FAKE + 4, 0, FAKE, FAKE, FAKE, 1, 8, 64, 4, 64, 0, FAKE, None, 0, None), 3),
     # misaligned fp32 scales
@@ -83,3 +89,11 @@ def test_other_calls_reject_on_host(qmm):
     assert L.bc_pack_int4(FAKE, FAKE, FAKE, 8, 64, None, None) == 1
     assert L.bc_pack_int4(FAKE, FAKE, FAKE, -1, 64, FAKE, None) == 1
     assert L.bc_matmul_q_batched(None, 1, 1, 4, 64, 1, 0, None, 0, None) == 1
+    assert L.bc_group_minmax(None, 8, 64, 64, FAKE, None) == 1
+    assert L.bc_group_minmax(FAKE, 8, 64, 32, FAKE, None) == 2
+    assert L.bc_group_minmax(FAKE, 8, 64, 64, FAKE + 2, None) == 3
+    # argmax: no token buffer; workspace smaller than the logits
+    assert L.bc_matmul_q_argmax(FAKE, 0, FAKE, None, None, 1, 8, 64, 16, 64, 0, None,
+                                FAKE, 4096, None) == 1
+    assert L.bc_matmul_q_argmax(FAKE, 0, FAKE, None, None, 1, 1 << 20, 64, 16, 64, 0, FAKE,
+                                FAKE, 4096, None) == 4

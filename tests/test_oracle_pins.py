@@ -339,3 +339,49 @@ def test_algorithmic_bytes_qwen25_int4_set():
     tot = sum(wl.gemv_bytes(m.K, m.N, 1, "packed", 4, 64)
               for m in wl.layer_set("qwen2.5-0.5b"))
     assert tot == 203476992
+
+
+def test_group_range_is_the_library_min_max():
+    """The bit-width-independent precompute (BITCRUSH BC-06, "Under the
+    hood") stores each group's exact range; numpy's own reductions over the
+    fp16 groups must give the same values, per group and per channel."""
+    rng = np.random.default_rng(12)
+    W = (rng.standard_normal((9, 192)) * np.exp(rng.uniform(-8, 4, (9, 1)))).astype(np.float16)
+    W[0] = 0.75
+    W[1, :64] = -2.0 ** -24
+    for group in (64, 192):
+        lo, hi = oracle.group_range(W, group)
+        g = W.astype(np.float64).reshape(9, 192 // group, group)
+        assert np.array_equal(lo, g.min(axis=2))
+        assert np.array_equal(hi, g.max(axis=2))
+
+
+def test_pack_codes_hand_worked_bytes():
+    """Other packed widths: each row is a little-endian bit string with code
+    k at bits [bits*k, bits*k + bits).  Hand-worked bytes:
+    3-bit codes 1,2,3,4,5,6,7,0: byte0 = 1 | 2<<3 | (3&3)<<6 = 209,
+    byte1 = 3>>2 | 4<<1 | 5<<4 | (6&1)<<7 = 88, byte2 = 6>>1 | 7<<2 | 0<<5 = 31;
+    2-bit codes 1,2,3,0,3,3,0,1: 1 | 2<<2 | 3<<4 | 0<<6 = 57 and
+    3 | 3<<2 | 0<<4 | 1<<6 = 79."""
+    q3 = np.zeros((1, 64), np.uint8)
+    q3[0, :8] = [1, 2, 3, 4, 5, 6, 7, 0]
+    assert oracle.pack_codes(q3, 3)[0, :4].tolist() == [209, 88, 31, 0]
+    q2 = np.zeros((1, 64), np.uint8)
+    q2[0, :8] = [1, 2, 3, 0, 3, 3, 0, 1]
+    assert oracle.pack_codes(q2, 2)[0, :3].tolist() == [57, 79, 0]
+    q8 = np.arange(64, dtype=np.uint8)[None, :] * 3
+    assert np.array_equal(oracle.pack_codes(q8, 8), q8)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_pack_codes_matches_numpy_bit_string(bits):
+    """Against numpy's own bit packing of the row bit strings (little-endian
+    bit order); for 4 bits it is also the int4 packing."""
+    rng = np.random.default_rng(bits)
+    q = rng.integers(0, 1 << bits, size=(5, 192)).astype(np.uint8)
+    bitsarr = ((q[:, :, None] >> np.arange(bits)) & 1).astype(np.uint8).reshape(5, -1)
+    expect = np.packbits(bitsarr, axis=1, bitorder="little")
+    got = oracle.pack_codes(q, bits)
+    assert np.array_equal(got, expect)
+    if bits == 4:
+        assert np.array_equal(got, oracle.pack_int4(q))

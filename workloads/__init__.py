@@ -38,11 +38,18 @@ SHAPE_SETS: Dict[str, List[Tuple[str, int, int]]] = {
                  ("o", 4096, 4096), ("gate", 4096, 12288), ("up", 4096, 12288),
                  ("down", 12288, 4096)],
 }
-LAYERS = {"qwen2.5-0.5b": 24, "qwen3-0.6b": 28, "qwen3-8b": 36}
-SIGMA = {"qwen2.5-0.5b": 0.02, "qwen3-0.6b": 0.02, "qwen3-8b": 0.015}
+# Single-matrix sets: the 1024 x 1024 single layer (BITCRUSH BC-06's lever
+# on one matrix) and Qwen3-0.6B's tied LM head (1024 -> vocabulary).
+SHAPE_SETS["single-1024"] = [("single", 1024, 1024)]
+SHAPE_SETS["qwen3-0.6b-lmhead"] = [("lm_head", 1024, 151936)]
+LAYERS = {"qwen2.5-0.5b": 24, "qwen3-0.6b": 28, "qwen3-8b": 36,
+          "single-1024": 1, "qwen3-0.6b-lmhead": 1}
+SIGMA = {"qwen2.5-0.5b": 0.02, "qwen3-0.6b": 0.02, "qwen3-8b": 0.015,
+         "single-1024": 0.02, "qwen3-0.6b-lmhead": 0.02}
 # Which activation each matrix reads inside a layer.
 X_TAG = {"q": "x_attn", "k": "x_attn", "v": "x_attn", "o": "x_o",
-         "gate": "x_mlp", "up": "x_mlp", "down": "x_down"}
+         "gate": "x_mlp", "up": "x_mlp", "down": "x_down", "single": "x",
+         "lm_head": "x"}
 _MAT_ID = {"q": 0, "k": 1, "v": 2, "o": 3, "gate": 4, "up": 5, "down": 6,
            "lm_head": 7, "single": 8}
 _TAG_ID = {"W": 0, "x_attn": 1, "x_o": 2, "x_mlp": 3, "x_down": 4, "x": 5}
@@ -140,12 +147,15 @@ def model_bytes(shape_set: str, bits: int) -> int:
 def gemv_bytes(K: int, N: int, M: int, mode: str, bits: int, group: int,
                x_bytes_per_elem: int = 4) -> int:
     """Algorithmic bytes of one matmul: weights (codes or fp16), scale/zero,
-    x and y.  Runtime mode reads fp16 W whatever the bits; packed mode reads
-    int4 codes and fp16 scale/zero per 64-block."""
+    x and y.  Runtime mode reads fp16 W whatever the bits, with fp32 scale
+    and zero per group ("range": one fp16 (min, max) word per group); packed
+    mode reads int4 codes and fp16 scale/zero per 64-block."""
     if mode == "packed":
         w = N * K // 2 + N * (K // 64) * 2 * 2
     elif bits == 16:
         w = N * K * 2
+    elif mode == "range":      # one 4-byte (min, max) word per group
+        w = N * K * 2 + N * (K // group) * 4
     else:
         w = N * K * 2 + N * (K // group) * 4 * 2
     return w + M * K * x_bytes_per_elem + M * N * 4
