@@ -48,10 +48,38 @@ WORKLOADS = {
     "qwen3-8b-int4-decode-m16": ("qwen3-8b", 36, "packed", 4, 64, 16, 4),
     "qwen3-8b-rtn3-decode": ("qwen3-8b", 36, "runtime", 3, 64, 1, 4),
     "qwen3-8b-rtn3-decode-m16": ("qwen3-8b", 36, "runtime", 3, 64, 16, 4),
-    # prefill: bf16 x, packed int4 W, tcgen05 tensor-core GEMM
+    # prefill: bf16 x, tcgen05 tensor-core GEMM; packed int4 W, or fp16 W
+    # re-quantized inline (runtime RTN at 3 bits, and the fp16 passthrough)
     "qwen2.5-0.5b-int4-prefill-m128": ("qwen2.5-0.5b", 24, "packed", 4, 64, 128, 3),
     "qwen2.5-0.5b-int4-prefill-m2048": ("qwen2.5-0.5b", 24, "packed", 4, 64, 2048, 3),
+    "qwen2.5-0.5b-rtn3-prefill-m128": ("qwen2.5-0.5b", 24, "runtime", 3, 64, 128, 3),
+    "qwen2.5-0.5b-rtn3-prefill-m2048": ("qwen2.5-0.5b", 24, "runtime", 3, 64, 2048, 3),
+    "qwen2.5-0.5b-fp16-prefill-m2048": ("qwen2.5-0.5b", 24, "runtime", 16, 64, 2048, 3),
+    # the bit-width-independent precompute: ranges stored, scale/zero in-kernel
+    "qwen3-0.6b-rtn3range-decode": ("qwen3-0.6b", 28, "range", 3, 64, 1, 2),
+    # Qwen3-0.6B's tied LM head (fp16 passthrough) reduced to a token id
+    "qwen3-0.6b-lmhead-argmax": ("qwen3-0.6b-lmhead", 1, "runtime", 16, 64, 1, 2),
 }
+# The lever sweep 16 -> 2 of the Qwen3-0.6B set, per group and per channel.
+for _b in (2, 4, 5, 6, 7, 8):
+    WORKLOADS[f"qwen3-0.6b-rtn{_b}-decode"] = ("qwen3-0.6b", 28, "runtime", _b, 64, 1, 2)
+for _b in (2, 4, 5, 6, 7, 8):
+    WORKLOADS[f"qwen3-0.6b-rtn{_b}-channel-decode"] = ("qwen3-0.6b", 28, "runtime", _b, 0, 1, 2)
+# The 1024 x 1024 single layer (seed 0) at bits {2, 3, 4, 8}, per group and
+# per channel: one matmul per step, L2 flushed before each timed step.
+for _b in (2, 3, 4, 8):
+    WORKLOADS[f"single-1024-rtn{_b}-decode"] = ("single-1024", 1, "runtime", _b, 64, 1, 0)
+    WORKLOADS[f"single-1024-rtn{_b}-channel-decode"] = ("single-1024", 1, "runtime", _b, 0, 1, 0)
+
+
+def is_argmax(name: str) -> bool:
+    return WORKLOADS[name][0] == "qwen3-0.6b-lmhead"
+
+
+def is_tiny(name: str) -> bool:
+    """Workloads far smaller than L2: each timed step is preceded by an L2
+    flush (outside the timed region) and timed on its own."""
+    return WORKLOADS[name][0] == "single-1024"
 
 
 def is_prefill(name: str) -> bool:
@@ -91,9 +119,13 @@ def workload_flops(name: str) -> int:
 
 
 def decode_kernel(name: str) -> str:
-    """The decode kernel the library picks for a workload's grouped call
-    (all decode workloads here are large enough for the streaming kernels)."""
-    _, _, mode, bits, _, M, _ = WORKLOADS[name]
+    """The decode kernel the library picks for a workload's grouped call:
+    the streaming kernels when the call has at least 74 row blocks of 128
+    (half the SMs), else the general GEMV."""
+    shape_set, layers, mode, bits, _, M, _ = WORKLOADS[name]
+    units = sum(-(-m.N // 128) for m in wl.layer_set(shape_set, layers))
+    if units < 74:
+        return "general"
     if M <= 4:
         return "stream"
     if M <= 16 and (mode == "packed" or bits <= 8):
@@ -110,16 +142,18 @@ def launches_per_step(name: str, count: int) -> int:
     M = WORKLOADS[name][5]
     if is_prefill(name):
         return -(-count // 80)
+    extra = 2 if is_argmax(name) else 0       # the two reduction kernels
     kind = decode_kernel(name)
     if kind == "stream":
-        return -(-count // 168)
+        return -(-count // 168) + extra
     if kind == "tc":
-        return 2 * -(-count // 168)
-    return -(-M // 16) * -(-count // 368)
+        return 2 * -(-count // 168) + extra
+    return -(-M // 16) * -(-count // 368) + extra
 
 
-KERNEL_SOURCES = {"decode": ("bc_gemv_stream.cu", "bc_gemv.cu", "bc_internal.cuh", "bc_tc.cuh"),
-                  "prefill": ("bc_gemm_sm100.cu", "bc_internal.cuh", "bc_tc.cuh")}
+KERNEL_SOURCES = {"decode": ("bc_gemv_stream.cu", "bc_gemv.cu", "bc_internal.cuh", "bc_tc.cuh",
+                             "bc_rtn.cuh"),
+                  "prefill": ("bc_gemm_sm100.cu", "bc_internal.cuh", "bc_tc.cuh", "bc_rtn.cuh")}
 
 
 def kernel_source_digest(kind: str = "decode") -> str:
@@ -302,6 +336,9 @@ def build_workload(qmm, torch, name: str, copies: int):
         elif bits == 16:
             s = z = None
             Wk = W
+        elif mode == "range":
+            s, z = qmm.group_minmax(W, group), None
+            Wk = W
         else:
             s, z = qmm.group_params(W, bits, group, torch.float32)
             Wk = W
@@ -353,7 +390,7 @@ def cpu_baseline_sample(name: str, target_s: float = 12.0):
             s, z = oracle.group_params(W, bits, g, mode == "packed")
             q = oracle.codes(W, s, z, bits, g)
             t0 = time.perf_counter()
-            if mode == "runtime":   # runtime mode re-derives the codes per step
+            if mode != "packed":    # runtime mode re-derives the codes per step
                 s, z = oracle.group_params(W, bits, g, False)
                 q = oracle.codes(W, s, z, bits, g)
             oracle.matmul(x, oracle.dequant(q, s, z, g))
@@ -406,7 +443,7 @@ def _reference_pass(name: str, sample) -> None:
             oracle.matmul(it["x"], oracle.half_to_f64(it["W"]))
             continue
         s, z, q = it["s"], it["z"], it["q"]
-        if mode == "runtime":     # runtime mode re-derives the codes per step
+        if mode != "packed":      # runtime mode re-derives the codes per step
             s, z = oracle.group_params(it["W"], bits, it["g"], False)
             q = oracle.codes(it["W"], s, z, bits, it["g"])
         oracle.matmul(it["x"], oracle.dequant(q, s, z, it["g"]))
@@ -470,18 +507,34 @@ def run_ours(args, rank, world, local_rank):
     step_bytes = workload_bytes(name)
     l2 = torch.cuda.get_device_properties(local_rank).L2_cache_size
     copies = args.copies or max(2, int(np.ceil(4 * l2 / step_bytes)) + 1)
-    copies = min(copies, 8)
+    copies = 1 if is_tiny(name) else min(copies, 8)
     W = build_workload(qmm, torch, name, copies)
-    mode_id = qmm.BC_MODE_PACKED_INT4 if mode == "packed" else qmm.BC_MODE_RUNTIME
+    mode_id = {"packed": qmm.BC_MODE_PACKED_INT4, "range": qmm.BC_MODE_RUNTIME_RANGE,
+               "runtime": qmm.BC_MODE_RUNTIME}[mode]
     prefill = is_prefill(name)
+    argmax = is_argmax(name)
     x_dtype = qmm.BC_BF16 if prefill else qmm.BC_F32
-    ws_bytes = max(qmm.workspace_size_batched(d, M, mode_id, x_dtype) for d in W["descs"])
+    if argmax:
+        m0 = W["mats"][0]
+        ws_bytes = qmm.workspace_size_argmax(M, m0.N, m0.K, mode_id, x_dtype)
+        token = torch.empty((M,), dtype=torch.int32, device="cuda")
+    else:
+        ws_bytes = max(qmm.workspace_size_batched(d, M, mode_id, x_dtype) for d in W["descs"])
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
     # The weights are fixed for the whole run, so decode steps may start while
     # the previous step finishes (BC_FLAG_STATIC_WEIGHTS; x and y still wait).
     def step(i):
+        if argmax:      # the LM head reduced to one token id per x row
+            xx, Wk, s, z, _ = W["per_copy"][i % copies][0]
+            st = qmm.lib.bc_matmul_q_argmax(
+                xx.data_ptr(), x_dtype, Wk.data_ptr(), None if s is None else s.data_ptr(),
+                None if z is None else z.data_ptr(), M, Wk.shape[0], xx.shape[1], bits, group,
+                mode_id, token.data_ptr(), ws.data_ptr(), ws.numel(), stream.cuda_stream)
+            if st != qmm.BC_OK:
+                raise qmm.BCError(st, "bc_matmul_q_argmax")
+            return
         qmm.matmul_q_batched(W["descs"][i % copies], M, bits, group, mode_id,
                              x_dtype=x_dtype, workspace=ws, static_weights=True)
 
@@ -523,6 +576,22 @@ def run_ours(args, rank, world, local_rank):
     time.sleep(0.02)
     sampler.stop()
     elapsed_ms = start.elapsed_time(end)
+    hot_ms = None
+    if is_tiny(name):
+        # far smaller than L2: time each step alone after writing a buffer
+        # larger than L2, and report that; the back-to-back figure is "hot"
+        hot_ms = elapsed_ms
+        flush = torch.empty(4 * l2, dtype=torch.uint8, device="cuda")
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i, (a, b) in enumerate(evs):
+            flush.fill_(i & 0xFF)
+            a.record(stream)
+            step(i)
+            b.record(stream)
+        torch.cuda.synchronize()
+        elapsed_ms = sum(a.elapsed_time(b) for a, b in evs)
+        del flush
     times = [elapsed_ms]
     if dist:
         t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
@@ -539,14 +608,15 @@ def run_ours(args, rank, world, local_rank):
     x_pinned = torch.from_numpy(W["x_all_host"]).pin_memory()
     if prefill:
         x_pinned = x_pinned.view(torch.bfloat16)
-    y_pinned = torch.empty(W["y_all_dev"].shape, dtype=torch.float32).pin_memory()
+    out_dev = token if argmax else W["y_all_dev"]     # argmax: one token id per row
+    y_pinned = torch.empty(out_dev.shape, dtype=out_dev.dtype).pin_memory()
     h2d = x_pinned.numel() * x_pinned.element_size()
-    d2h = y_pinned.numel() * 4
+    d2h = y_pinned.numel() * y_pinned.element_size()
 
-    def e2e_step(i):      # every x of the step in, the step, every y out
+    def e2e_step(i):      # every x of the step in, the step, every output out
         W["x_all_dev"].copy_(x_pinned, non_blocking=True)
         step(i)
-        y_pinned.copy_(W["y_all_dev"], non_blocking=True)
+        y_pinned.copy_(out_dev, non_blocking=True)
 
     for i in range(3):
         e2e_step(i)
@@ -591,7 +661,7 @@ def run_ours(args, rank, world, local_rank):
                                f"{peaks['bf16_tflops_sustained']}",
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                 "hbm_gbs_achieved": step_bytes / (avg_launch_ms / 1e3) / 1e9,
-                "kernel": "gemm_packed_kernel (bc_gemm_sm100.cu)",
+                "kernel": "gemm_kernel (bc_gemm_sm100.cu)",
                 "avg_step_us": avg_launch_ms * 1e3}
     else:
         achieved = step_bytes / (avg_launch_ms / 1e3) / 1e9
@@ -613,16 +683,28 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": name, "shape_set": shape_set, "layers": layers,
                    "matrices": len(W["mats"]), "mode": mode, "bits": bits,
                    "group": group if group else "per-channel", "M": M,
-                   "weights": "int4 packed, fp16 scale/zero per 64-block"
-                   if mode == "packed" else "fp16, runtime RTN",
+                   "weights": {"packed": "int4 packed, fp16 scale/zero per 64-block",
+                               "runtime": "fp16, runtime RTN" if bits != 16
+                               else "fp16 passthrough",
+                               "range": "fp16, runtime RTN from stored group ranges "
+                                        "(scale/zero derived in the kernel)"}[mode],
                    "x": "bf16" if prefill else "fp32", "bytes_per_step": step_bytes,
                    "flops_per_step": step_flops,
-                   "l2": f"inputs larger than L2: {copies} weight copies "
-                         f"({copies * step_bytes / 1e6:.0f} MB) rotated between "
-                         f"steps, L2 {l2 / 1e6:.0f} MB",
-                   "launch": "one grouped launch per step; decode steps launched "
-                             "as programmatic dependent launches (static weights)"},
+                   "l2": (f"L2 flushed ({4 * l2 / 1e6:.0f} MB written) before each timed "
+                          "step; each step timed on its own"
+                          if is_tiny(name) else
+                          f"inputs larger than L2: {copies} weight copies "
+                          f"({copies * step_bytes / 1e6:.0f} MB) rotated between "
+                          f"steps, L2 {l2 / 1e6:.0f} MB"),
+                   "launch": ("one call per step: the GEMV, then two reduction kernels "
+                              "(token id per row)" if argmax else
+                              "one grouped launch per step; decode steps launched "
+                              "as programmatic dependent launches (static weights)")},
         "roofline": roof,
+        **({"hot": {"us_per_step": hot_ms / args.steps * 1e3,
+                    "value": step_units * args.steps / (hot_ms / 1e3), "unit": unit,
+                    "note": "steps back to back, weights resident in L2"}}
+           if hot_ms is not None else {}),
         "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": e_ms / e_steps, "steps": e_steps},
