@@ -135,9 +135,10 @@ template <bool PACKED> __host__ __device__ __forceinline__ int kpad_of(int K) {
 // Packed x row: digit words [digit d][lane t][unit U][parity] with a row
 // stride of dig_rs words (= 4 mod 32, so the 8 rows a quarter-warp reads sit
 // in distinct banks), then [parity][group] float2 (f, T) tables, then per
-// group the values of its side pair (float2: even k, odd k) and one side byte
-// (0: none; 1 + p: exactly one side pair, pair p = k 64g + 2p, 2p + 1;
-// 0xFF: more than one), eight bytes to a stage chunk.
+// group the values of its side pair (float2: even k, odd k; for a group with
+// several side pairs the masks of their even and odd side members) and one
+// side byte (0: none; 1 + p: exactly one side pair, pair p = k 64g + 2p,
+// 2p + 1; 0xFF: more than one), eight bytes to a stage chunk.
 __host__ __device__ __forceinline__ int dig_rs(int kchunks) { return 32 * kchunks + 4; }
 __host__ __device__ __forceinline__ int side_val_off(int kchunks) {
     return 64 * dig_rs(kchunks) + 16 * (8 * kchunks);
@@ -295,9 +296,10 @@ __device__ __forceinline__ void transpose4(const uint32_t (&w)[4], uint32_t (&o)
 // and the mask of its side elements.
 //
 // Side elements.  The integer grid of a group is 2^(E-30) at even k and
-// 2^(E-26) at odd k, so an element keeps a relative error of at most 2^-14
-// only if |x| >= 2^(E-17) (even) or 2^(E-13) (odd).  Nonzero elements below
-// those bounds are left out of the digits (staged as 0) and flagged; the
+// 2^(E-26) at odd k, so an element above 2^(E-17) (even) or 2^(E-13) (odd)
+// is always held within 2^-14 of itself.  Below those bounds an element
+// whose rounding misses it by more than 2^-14 of itself is left out of the
+// digits (staged as 0) and flagged (about half of the small ones); the
 // consumers add their products exactly, in fp32.  The values of a group's
 // side pair are kept beside the digits (a group holds one side pair or none
 // on almost every input; groups with more take a slower exact path that
@@ -319,19 +321,30 @@ __device__ __forceinline__ int group_exponent(float amax) {
     return max(E, -96);
 }
 // Side elements of the pair (ve, vo) by the staging rules of a group with
-// grid exponent E (as group_digits decides them).
+// grid exponent E: an element is a side element when its integer rounding
+// misses it by more than 2^-14 of itself (only possible below 2^(E-17) at
+// even k, 2^(E-13) at odd k); the even element goes with a side odd one.
+__device__ __forceinline__ bool rounds_badly(float v, int E, int bits) {
+    // grid 2^(E-bits); below 2^(E-bits+13) the scaled value is under 2^13,
+    // so rint, the product and the fma residual are all exact
+    if (v == 0.0f) return false;
+    if (fabsf(v) >= __uint_as_float((uint32_t)(127 + E - bits + 13) << 23)) return false;
+    const float sc = __uint_as_float((uint32_t)(127 + bits - E) << 23);
+    const float grid = __uint_as_float((uint32_t)(127 + E - bits) << 23);
+    const float err = fmaf(-rintf(v * sc), grid, v);
+    return fabsf(err) > fabsf(v) * 6.103515625e-05f;             // 2^-14
+}
 __device__ __forceinline__ void side_pair(float ve, float vo, int E, bool &se, bool &so) {
-    const float thr_e = __uint_as_float((uint32_t)(127 + E - 17) << 23);
-    const float thr_o = __uint_as_float((uint32_t)(127 + E - 13) << 23);
-    so = vo != 0.0f && fabsf(vo) < thr_o;
-    se = ve != 0.0f && (so || fabsf(ve) < thr_e);
+    so = rounds_badly(vo, E, kXP);
+    se = ve != 0.0f && (so || rounds_badly(ve, E, kXP + 4));
 }
 __device__ __forceinline__ int lo16(int v) {          // d0 + 256 d1 of digits4(v)
     return (int)(((uint32_t)v + 0x8080u) & 0xFFFFu) - 0x8080;
 }
 __device__ __forceinline__ void group_digits(const float (&v)[8], uint32_t (&te)[4],
                                              uint32_t (&to)[4], float &f, int &t01,
-                                             int &t23, uint32_t &sidepairs, int &Eg) {
+                                             int &t23, uint32_t &side_e, uint32_t &side_o,
+                                             int &Eg) {
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
@@ -342,14 +355,15 @@ __device__ __forceinline__ void group_digits(const float (&v)[8], uint32_t (&te)
     const float sc_e = __uint_as_float((uint32_t)(127 + kXP + 4 - E) << 23);
     const float sc_o = __uint_as_float((uint32_t)(127 + kXP - E) << 23);
     uint32_t de[4], dq[4];
-    uint32_t lm = 0;
+    uint32_t lme = 0, lmo = 0;
     int s01 = 0, s23 = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const float ve = v[2 * i], vo = v[2 * i + 1];
         bool se, so;
         side_pair(ve, vo, E, se, so);
-        lm |= ((se || so) ? 1u : 0u) << i;
+        lme |= (se ? 1u : 0u) << i;
+        lmo |= (so ? 1u : 0u) << i;
         const int xe = se ? 0 : __float2int_rn(ve * sc_e);   // |xe| <= 2^30
         const int xo = so ? 0 : __float2int_rn(vo * sc_o);   // |xo| <= 2^26
         const int dv = xo - xe;       // odd slots carry X_odd - X_even (raw-byte A)
@@ -369,11 +383,15 @@ __device__ __forceinline__ void group_digits(const float (&v)[8], uint32_t (&te)
     s23 += __shfl_xor_sync(0xffffffffu, s23, 4);
     t01 = s01;
     t23 = s23;
-    // side pairs of the group: bit 4j + i <-> pair (8j + 2i, 8j + 2i + 1)
-    sidepairs = lm << (4 * (threadIdx.x & 7));
-    sidepairs |= __shfl_xor_sync(0xffffffffu, sidepairs, 1);
-    sidepairs |= __shfl_xor_sync(0xffffffffu, sidepairs, 2);
-    sidepairs |= __shfl_xor_sync(0xffffffffu, sidepairs, 4);
+    // side members of the group's pairs: bit 4j + i <-> pair (8j + 2i,
+    // 8j + 2i + 1), even members in side_e, odd members in side_o
+    side_e = lme << (4 * (threadIdx.x & 7));
+    side_o = lmo << (4 * (threadIdx.x & 7));
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+        side_e |= __shfl_xor_sync(0xffffffffu, side_e, o);
+        side_o |= __shfl_xor_sync(0xffffffffu, side_o, o);
+    }
     f = __uint_as_float((uint32_t)(127 + E - kXP - 4) << 23);
     Eg = E;
 }
@@ -411,9 +429,10 @@ __device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
             uint32_t te[4], to[4];
             float f;
             int t01, t23;
-            uint32_t sp;
+            uint32_t sme, smo;
             int E;
-            group_digits(v, te, to, f, t01, t23, sp, E);
+            group_digits(v, te, to, f, t01, t23, sme, smo, E);
+            const uint32_t sp = sme | smo;
             const int U = 2 * g + (j >> 2), tt = j & 3;
 #pragma unroll
             for (int d = 0; d < 4; ++d)
@@ -424,6 +443,8 @@ __device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
                 tab[gpad + g] = make_float2(f * 65536.0f, __int_as_float(t23));
                 xm[side_flag_off(kch) + g] =
                     sp == 0 ? 0 : (__popc(sp) == 1 ? (uint8_t)(__ffs(sp)) : kSideMany);
+                if (__popc(sp) > 1)      // several side pairs: their members' masks
+                    reinterpret_cast<uint2 *>(xm + side_val_off(kch))[g] = make_uint2(sme, smo);
             }
             if (sp != 0 && __popc(sp) == 1 && ((__ffs(sp) - 1) >> 2) == j) {
                 // the lane holding the group's one side pair stores its values
@@ -436,8 +457,7 @@ __device__ void stage_x_packed(const float *__restrict__ xr, int K, uint8_t *xm,
                         ve = v[2 * q];
                         vo = v[2 * q + 1];
                     }
-                bool se, so;
-                side_pair(ve, vo, E, se, so);
+                const bool se = (sme >> (__ffs(sp) - 1)) & 1u, so = (smo >> (__ffs(sp) - 1)) & 1u;
                 reinterpret_cast<float2 *>(xm + side_val_off(kch))[g] =
                     make_float2(se ? ve : 0.0f, so ? vo : 0.0f);
             }
@@ -626,25 +646,20 @@ __device__ __forceinline__ float side_fast(uint32_t info, float2 vals, const uin
     const uint32_t b = box[row * 128 + (((byte >> 4) ^ (row & 7)) << 4) + (byte & 15)];
     return s * fmaf((float)(b >> 4) - z, vals.y, ((float)(b & 15u) - z) * vals.x);
 }
-// Slow path (more than one side pair in the group): the side elements are
-// found again from the group's x in global memory (xg = its first element)
-// by the staging rules, and their products added exactly.
-__device__ __noinline__ float side_slow(const float *__restrict__ xg, const uint8_t *box,
-                                        int row, int sub, float s, float z) {
-    float amax = 0.0f;
-    for (int i = 0; i < 16; ++i) {
-        const float4 v = __ldg(reinterpret_cast<const float4 *>(xg) + i);
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-    }
-    const int E = group_exponent(amax);
+// Slow path (more than one side pair in the group): the slot holds the masks
+// of the group's side members (even, odd) instead of values; the values come
+// from x in global memory (xg = the group's first element).
+__device__ __noinline__ float side_slow(uint2 masks, const float *__restrict__ xg,
+                                        const uint8_t *box, int row, int sub, float s, float z) {
     float acc = 0.0f;
-    for (int p = 0; p < 32; ++p) {
+    uint32_t pm = masks.x | masks.y;
+    while (pm) {
+        const int p = __ffs(pm) - 1;
+        pm &= pm - 1;
         const float2 v = __ldg(reinterpret_cast<const float2 *>(xg) + p);
-        bool se, so;
-        side_pair(v.x, v.y, E, se, so);
-        if (se || so) acc += side_fast((uint32_t)p + 1, make_float2(se ? v.x : 0.0f,
-                                                                    so ? v.y : 0.0f),
-                                       box, row, sub, s, z);
+        acc += side_fast((uint32_t)p + 1, make_float2(((masks.x >> p) & 1u) ? v.x : 0.0f,
+                                                      ((masks.y >> p) & 1u) ? v.y : 0.0f),
+                         box, row, sub, s, z);
     }
     return acc;
 }
@@ -728,7 +743,8 @@ __device__ __forceinline__ void consume_packed_m1(
                         v += info != kSideMany
                                  ? side_fast(info, sv[4 * w + sub], st + w * kBoxBytes, row, sub,
                                              sc, zc)
-                                 : side_slow(J.x + 512 * k.kc + 64 * (4 * w + sub),
+                                 : side_slow(reinterpret_cast<const uint2 *>(sv)[4 * w + sub],
+                                             J.x + 512 * k.kc + 64 * (4 * w + sub),
                                              st + w * kBoxBytes, row, sub, sc, zc);
                     }
                 }
@@ -889,7 +905,8 @@ __device__ __forceinline__ void consume_packed_mx(
                         v += info != kSideMany
                                  ? side_fast(info, sv[4 * w + sub], st + w * kBoxBytes, row, sub,
                                              sc, zc)
-                                 : side_slow(J.x + (int64_t)m * J.K + 512 * k.kc +
+                                 : side_slow(reinterpret_cast<const uint2 *>(sv)[4 * w + sub],
+                                             J.x + (int64_t)m * J.K + 512 * k.kc +
                                                  64 * (4 * w + sub),
                                              st + w * kBoxBytes, row, sub, sc, zc);
                     }
