@@ -27,9 +27,10 @@
 //     tensor core;
 //   * one thread (warp 1) issues four tcgen05.mma.kind::f16 (K = 16 each)
 //     accumulating fp32 in TMEM, and tcgen05.commit frees the stage;
-//   * four epilogue warps drain the finished accumulator (tcgen05.ld) and
-//     store y with 128-byte coalesced rows, while the next tile accumulates
-//     into the second TMEM buffer.
+//   * eight epilogue warps (two per TMEM lane quarter, each half of the
+//     columns) drain the finished accumulator (tcgen05.ld) and store y with
+//     128-byte coalesced rows, while the next tile accumulates into the
+//     second TMEM buffer.
 // The kernel is persistent (one CTA per SM) and spans every matrix of a
 // grouped launch.  Each CTA owns a contiguous range of tiles chosen on the
 // host so that the ranges cost about the same (a tile costs its K/64 stages
@@ -61,7 +62,7 @@ constexpr int kBM = 128;                    // weight rows per tile
 constexpr int kBK = 64;                     // K per stage (one quant block)
 constexpr int kTmaWarp = 0, kMmaWarp = 1;
 constexpr int kDqWarp0 = 2, kDqWarps = 8;   // warps 2..9
-constexpr int kEpWarp0 = 10, kEpWarps = 4;  // warps 10..13
+constexpr int kEpWarp0 = 10, kEpWarps = 8;  // warps 10..17 (two per TMEM lane quarter)
 constexpr int kThreads = 32 * (kEpWarp0 + kEpWarps);
 constexpr int kMaxJobs = 80;
 constexpr int kMaxCtas = 160;
@@ -142,14 +143,18 @@ __device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 // Bounded wait; false (and a recorded timeout, once per CTA) if it ran out
-// or if another role of this CTA already gave up.
+// or if another role of this CTA already gave up.  SLEEP lets the thread
+// sleep between tests (the dequant and epilogue warps, which wait long and
+// would otherwise take issue slots); the producer and the MMA issuer spin,
+// since a wake-up delay there lengthens every stage.
+template <bool SLEEP = true>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int *abort_flag) {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
     const long long limit = *(volatile long long *)&g_gemm_wait_limit;
     while (true) {
-        if (mbar_try_sleep(bar, parity)) return true;
+        if (SLEEP ? mbar_try_sleep(bar, parity) : mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
         if (clock64() - t0 > limit) {
             if (atomicExch((int *)abort_flag, 1) == 0)
@@ -413,7 +418,7 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
                 for (int kb = 0; kb < kblocks; ++kb, ++g) {
                     const int s = g % C::kStages;
                     const uint32_t ph = (g / C::kStages) & 1;
-                    if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag)) break;
+                    if (!mbar_wait<false>(smem_u32(&empty[s]), ph ^ 1, abort_flag)) break;
                     uint8_t *st = smem + s * C::kStageBytes;
                     const uint32_t fb = smem_u32(&full_tma[s]);
                     if constexpr (WF == kPacked) {
@@ -458,7 +463,8 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
             const int kblocks = sjobs[j].K / kBK;
             const int buf = lt & 1;
             const uint32_t aph = (lt >> 1) & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag)))
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait<false>(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag)))
                 break;
             tc::fence_after();
             const uint32_t d_tmem = tmem_base + buf * BNX;
@@ -466,8 +472,8 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
             for (int kb = 0; kb < kblocks; ++kb, ++g) {
                 const int s = g % C::kStages;
                 const uint32_t ph = (g / C::kStages) & 1;
-                bool w = mbar_wait(smem_u32(&full_tma[s]), ph, abort_flag);
-                if (w) w = mbar_wait(smem_u32(&full_dq[s]), ph, abort_flag);
+                bool w = mbar_wait<false>(smem_u32(&full_tma[s]), ph, abort_flag);
+                if (w) w = mbar_wait<false>(smem_u32(&full_dq[s]), ph, abort_flag);
                 if (!__all_sync(0xffffffffu, w)) {
                     ok = false;
                     break;
@@ -591,8 +597,9 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
             }
         }
     } else {
-        // epilogue: warp quarter q reads TMEM lanes 32q..32q+31 (weight rows)
-        const int q = warp & 3;
+        // epilogue: warp quarter q reads TMEM lanes 32q..32q+31 (weight rows),
+        // half hh of the accumulator's columns (x rows)
+        const int q = warp & 3, hh = (warp - kEpWarp0) >> 2;
         int lt = 0;
         for (int tile = t_begin; tile < t_end && !*abort_flag; ++tile, ++lt) {
             const int j = find_job(sjobs, P.count, tile);
@@ -606,7 +613,7 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
             const int n = nb * kBM + 32 * q + lane;
             const int m0 = xb * BNX;
 #pragma unroll 1
-            for (int c = 0; c < BNX / 32; ++c) {
+            for (int c = hh * (BNX / 64); c < (hh + 1) * (BNX / 64); ++c) {
                 uint32_t v[32];
                 tc::ld32(tmem_base + ((uint32_t)(32 * q) << 16) + buf * BNX + c * 32, v);
                 if (n < J.N) {
