@@ -12,32 +12,45 @@
 // Enargeia's tiled-matmul ladder: tiling and register blocking decide
 // matmul speed; here the tiles feed tcgen05 from shared memory and TMEM.
 //
-// Tile = 128 weight rows (the MMA's M, i.e. TMEM lanes) x BNX activation
-// rows (the MMA's N) x 64 along K (one quantization block, one 128-byte
-// swizzle atom row of bf16).  Per 64-block of K:
-//   * one thread (warp 0) issues the TMA loads of a stage: the bf16 x tile
-//     (128B-swizzled, K-major) and the weights -- 128 x 32 bytes of packed
-//     codes, or the 128 x 64 fp16 weights themselves, landed 128B-swizzled
-//     in the stage's A tile;
-//   * eight dequant warps form bf16 w' = (q - z) * s in the same
-//     128B-swizzled K-major layout the MMA reads (packed: exact q - z in
-//     bf16 arithmetic and one rounding for the scale; runtime: the exact RTN
-//     code of each fp16 weight, then one rounding of (q - z) s, written over
-//     the weight it came from), then fence the generic-proxy writes for the
-//     tensor core;
-//   * one thread (warp 1) issues four tcgen05.mma.kind::f16 (K = 16 each)
-//     accumulating fp32 in TMEM, and tcgen05.commit frees the stage;
-//   * eight epilogue warps (two per TMEM lane quarter, each half of the
-//     columns) drain the finished accumulator (tcgen05.ld) and store y with
-//     128-byte coalesced rows, while the next tile accumulates into the
-//     second TMEM buffer.
-// The kernel is persistent (one CTA per SM) and spans every matrix of a
-// grouped launch.  Each CTA owns a contiguous range of tiles chosen on the
-// host so that the ranges cost about the same (a tile costs its K/64 stages
-// plus its epilogue), instead of a round-robin stride that leaves SMs idle
-// when matrices of very different K share a launch.  All waits are bounded:
+// Two SMs (a cluster of two CTAs) share one tile of 256 weight rows x BNX
+// activation rows: one tcgen05.mma.cta_group::2 (M = 256, N = BNX, K = 16)
+// reads the 128 dequantized weight rows of each CTA (A) and the BNX/2
+// activation rows each CTA loaded (B), and accumulates fp32 into the TMEM
+// of both.  Each SM therefore loads half the activation tile that a
+// one-SM tile of the same shape would: on 128 x 256 one-SM tiles the
+// activation traffic from L2 set the pace (each 64-wide K step waited
+// about 3400 cycles for its loads), not the tensor cores.
+//
+// Per CTA, per 64-block of K (one quantization block):
+//   * a code producer (warp 0) loads the CTA's weights into a ring of
+//     their own (they are read once, by the dequant warps): packed codes
+//     four blocks at a time (128 rows of 128 bytes: whole L2 lines, where
+//     one block's 32 bytes per row made 32-byte requests), or the 128 x 64
+//     fp16 weights of one block;
+//   * an activation producer (warp 2) loads the CTA's BNX/2 rows of bf16 x
+//     (128B-swizzled, K-major) into the activation ring, which the MMA
+//     frees;
+//   * sixteen dequant warps (two groups of eight taking alternate blocks)
+//     form bf16 w' = (q - z) * s into one of four A buffers in the
+//     128B-swizzled K-major layout the MMA reads (packed:
+//     exact q - z in bf16 arithmetic and one rounding for the scale;
+//     runtime: the exact RTN code of each fp16 weight, then one rounding of
+//     (q - z) s), fence the generic-proxy writes for the tensor core and
+//     arrive on the first CTA's "A ready" barrier (cluster scope);
+//   * the first CTA's MMA warp waits for both CTAs' A buffers and its own
+//     activation stage (the second CTA's dequant warps wait for theirs
+//     before they arrive), issues four MMAs and commits to the "free"
+//     barriers of both CTAs at once (commit multicast);
+//   * eight epilogue warps per CTA drain the finished accumulator
+//     (tcgen05.ld) and store y with coalesced rows while the next tile
+//     accumulates into the second TMEM buffer.
+// The kernel is persistent (one cluster per SM pair) and spans every matrix
+// of a grouped launch; each pair owns a contiguous range of tiles chosen on
+// the host so that the ranges cost about the same.  All waits are bounded:
 // a wait that runs out records a timeout, the CTA stops, waits (bounded) for
-// its own copies and MMAs in flight and frees its TMEM.
+// its own copies and MMAs in flight, meets its partner at the cluster
+// barrier and frees its TMEM.  No load uses cluster multicast: every CTA
+// loads its own tiles.
 #include "bc_internal.cuh"
 #include "bc_rtn.cuh"
 #include "bc_tc.cuh"
@@ -58,14 +71,15 @@ __device__ long long g_gemm_wait_limit = 4000000000LL;
 
 namespace {
 
-constexpr int kBM = 128;                    // weight rows per tile
+constexpr int kBM = 128;                    // weight rows per CTA (TMEM lanes)
+constexpr int kPairRows = 2 * kBM;          // weight rows per tile (the MMA's M)
 constexpr int kBK = 64;                     // K per stage (one quant block)
-constexpr int kTmaWarp = 0, kMmaWarp = 1;
-constexpr int kDqWarp0 = 2, kDqWarps = 8;   // warps 2..9
-constexpr int kEpWarp0 = 10, kEpWarps = 8;  // warps 10..17 (two per TMEM lane quarter)
+constexpr int kCodeWarp = 0, kMmaWarp = 1, kXWarp = 2;
+constexpr int kDqWarp0 = 3, kDqWarps = 16;  // warps 3..18
+constexpr int kEpWarp0 = 19, kEpWarps = 8;  // warps 19..26 (two per TMEM lane quarter)
 constexpr int kThreads = 32 * (kEpWarp0 + kEpWarps);
 constexpr int kMaxJobs = 80;
-constexpr int kMaxCtas = 160;
+constexpr int kMaxPairs = 80;
 constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 2 GHz
 
 // Weight forms.
@@ -82,10 +96,10 @@ struct GemmJobDev {
 };
 
 struct __align__(64) GemmParams {
-    CUtensorMap xmap[kMaxJobs];     // bf16 x [M][K], box {64, BNX}, SW128
-    CUtensorMap wmap[kMaxJobs];     // packed u8 [N][K/2] box {32, 128}; fp16 W [N][K] box {64, 128} SW128
+    CUtensorMap xmap[kMaxJobs];     // bf16 x [M][K], box {64, BNX/2}, SW128
+    CUtensorMap wmap[kMaxJobs];     // packed u8 [N][K/2] box {128, 128}; fp16 W [N][K] box {64, 128}; SW128
     GemmJobDev jobs[kMaxJobs];
-    int cta_begin[kMaxCtas + 1];    // tile range of each CTA
+    int pair_begin[kMaxPairs + 1];  // tile range of each CTA pair
     int count, total_tiles, M;
     int bits;                       // runtime: 2..8 or 16 (passthrough)
     int range;                      // runtime: s holds per-group ranges
@@ -93,29 +107,74 @@ struct __align__(64) GemmParams {
 static_assert(sizeof(GemmParams) <= 32000, "kernel parameter space");
 
 template <int BNX, int WF> struct Cfg {
-    static constexpr int kABytes = kBM * 128;          // 16 KB (runtime: W lands here)
-    static constexpr int kBBytes = BNX * 128;
-    static constexpr int kCBytes = WF == kPacked ? kBM * 32 : 0;   // 4 KB of codes
-    static constexpr int kStageBytes = kABytes + kBBytes + kCBytes;  // multiple of 1024
-    static constexpr int kBarBytes = 4096;     // barriers + job table copy
-    static constexpr int kStages =
-        std::min(6, (227 * 1024 - kBarBytes - 1024) / kStageBytes);
-    static constexpr int kTmemCols = 2 * BNX;
-    static constexpr int kSmem = kStages * kStageBytes + kBarBytes + 1024;
-    // instruction descriptor: D f32, A/B bf16, K-major both, N, M = 128
-    static constexpr uint32_t kIdesc = tc::idesc_bf16(kBM, BNX);
-    static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+    static constexpr int kXHalf = BNX / 2;                       // x rows per CTA
+    static constexpr int kXBytes = kXHalf * 128;                 // 16 or 8 KB
+    // One weight box covers kGroup 64-blocks of K: packed codes of four
+    // blocks are 128-byte rows (whole L2 lines; one 32-byte piece per block
+    // would be a 32-byte request per row), fp16 weights one block.
+    static constexpr int kGroup = WF == kPacked ? 4 : 1;
+    static constexpr int kDqGroups = WF == kPacked ? 2 : 1;     // dequant warp groups
+    static constexpr int kWRow = WF == kPacked ? 32 * kGroup : 128;   // bytes per row
+    static constexpr int kWBytes = kBM * kWRow;                   // 16 KB
+    static constexpr int kABytes = kBM * 128;                    // 16 KB
+    static constexpr int kAStages = 4;
+    // even: each dequant group sees every other phase of an x (and A)
+    // barrier, and the parity test is sound only if the ring depth keeps a
+    // slot's stages in one group
+    static constexpr int kXStages = BNX == 256 ? (WF == kPacked ? 6 : 4) : 8;
+    static constexpr int kWStages = WF == kPacked ? (BNX == 256 ? 3 : 4) : 5;
+    static constexpr int kAOff = 0;
+    static constexpr int kXOff = kAOff + kAStages * kABytes;
+    static constexpr int kWOff = kXOff + kXStages * kXBytes;
+    static constexpr int kBarOff = kWOff + kWStages * kWBytes;
+    static constexpr int kBarBytes = 5120;     // barriers + job table copy
+    static constexpr int kSmem = kBarOff + kBarBytes + 1024;
+    static constexpr int kTmemCols = 2 * BNX;  // two accumulators of BNX columns
+    // instruction descriptor: D f32, A/B bf16, K-major both, M = 256, N = BNX
+    static constexpr uint32_t kIdesc = tc::idesc_bf16(kPairRows, BNX);
+    static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+    static_assert(kXStages % 2 == 0 && kAStages % 2 == 0, "rings of even depth");
+    static_assert(kXBytes % 1024 == 0 && kWBytes % 1024 == 0 && kABytes % 1024 == 0,
+                  "rings keep the 1024-byte swizzle alignment");
 };
 
 // ---- small PTX wrappers ----------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+// The address of the same shared-memory location in the pair's first CTA.
+__device__ __forceinline__ uint32_t in_leader(uint32_t local) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(r) : "r"(local));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
 }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Arrive on a barrier of the pair (cluster address).  Default semantics
+// (release at CTA scope): the data it announces is this CTA's own shared
+// memory, already fenced for the tensor core (fence.proxy.async), which the
+// MMA reads on this CTA's SM; a cluster-scope release would also wait for
+// this thread's outstanding global loads (the scale/zero look-ahead).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cbar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cbar) : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
@@ -142,26 +201,72 @@ __device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity) {
         : "=r"(ok) : "r"(bar), "r"(parity), "r"(20000u) : "memory");
     return ok != 0;
 }
+// How a role waits.  kSpin polls without pause (the MMA issuer: a late
+// wake-up lengthens every stage).  kSleep lets the thread sleep with a
+// suspend hint until the phase completes (waits on this CTA's own loads).
+// kBackoff polls with a short nanosleep between tests: the producers and
+// the epilogue, which wait long on barriers that the partner CTA may
+// complete (a thread sleeping with a hint there wakes thousands of cycles
+// late) and which, spinning, take issue slots from the dequant warps that
+// share their scheduler.
+constexpr int kSpin = 0, kSleep = 1, kBackoff = 2;
+
 // Bounded wait; false (and a recorded timeout, once per CTA) if it ran out
-// or if another role of this CTA already gave up.  SLEEP lets the thread
-// sleep between tests (the dequant and epilogue warps, which wait long and
-// would otherwise take issue slots); the producer and the MMA issuer spin,
-// since a wake-up delay there lengthens every stage.
-template <bool SLEEP = true>
+// or if another role of this CTA already gave up.
+template <int MODE = kSleep>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int *abort_flag) {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
     const long long limit = *(volatile long long *)&g_gemm_wait_limit;
     while (true) {
-        if (SLEEP ? mbar_try_sleep(bar, parity) : mbar_try(bar, parity)) return true;
+        if (MODE == kSleep ? mbar_try_sleep(bar, parity) : mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
         if (clock64() - t0 > limit) {
             if (atomicExch((int *)abort_flag, 1) == 0)
                 atomicAdd(&g_gemm_timeouts, 1u);
             return false;
         }
+        if (MODE == kBackoff) __nanosleep(128);
     }
+}
+// Drain wait of the exit paths: fixed limit, no abort test.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try(bar, parity) && clock64() - t0 < kWaitCycles) {
+    }
+}
+// tcgen05 forms of the pair (cta_group::2).
+__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate) : "memory");
+}
+// Arrive once on `bar` (same offset) in both CTAs of the pair when every
+// MMA issued so far has completed.
+__device__ __forceinline__ void commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;"
+        ::"r"(bar), "h"((uint16_t)0x3) : "memory");
+}
+// Arrive once on this CTA's `bar` when every MMA issued so far has completed.
+__device__ __forceinline__ void commit_local(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+        ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t slot_smem, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(slot_smem), "r"(cols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t base, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
+                 ::"r"(base), "r"(cols) : "memory");
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map,
                                             int x, int y, uint32_t bar) {
@@ -170,12 +275,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         " [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
-}
-// Bring one weight box of a later tile into L2 (no shared memory, no
-// barrier): the TMA of that stage then meets L2 instead of HBM latency.
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
-                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
 }
 __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
@@ -260,12 +359,28 @@ __device__ __forceinline__ int find_job(const GemmJobDev *jobs, int count, int t
     return lo;
 }
 
+// Position of a tile: matrix j, 256-row weight block nb, BNX-row x block xb.
+struct TilePos {
+    int j, nb, xb, kblocks;
+};
+__device__ __forceinline__ TilePos tile_pos(const GemmJobDev *jobs, int count, int tile) {
+    TilePos t;
+    t.j = find_job(jobs, count, tile);
+    const GemmJobDev &J = jobs[t.j];
+    const int local = tile - J.tile_begin;
+    t.nb = local / J.xblocks;
+    t.xb = local % J.xblocks;
+    t.kblocks = J.K / kBK;
+    return t;
+}
+
 constexpr int kLook = 4;     // scale/zero look-ahead, in 64-blocks of K
+static_assert(kLook % 2 == 0, "two dequant groups take alternate look-ahead slots");
 
 // Walks the (tile, 64-block) sequence a dequant thread consumes and loads
 // the scale and zero of its weight row for each position.
 template <int WF> struct SzCursor {
-    int tile, t_end, kb, kblocks, group;
+    int tile, t_end, kb, kblocks, group, row0;
     const void *srow;
     const void *zrow;
     const GemmJobDev *jobs;
@@ -277,7 +392,7 @@ template <int WF> struct SzCursor {
         }
         const GemmJobDev &J = jobs[find_job(jobs, P.count, tile)];
         const int nb = (tile - J.tile_begin) / J.xblocks;
-        const int row = nb * kBM + r;
+        const int row = nb * kPairRows + row0 + r;
         kblocks = J.K / kBK;
         group = J.group;
         const int64_t G = J.K / J.group;
@@ -290,11 +405,12 @@ template <int WF> struct SzCursor {
         }
     }
     __device__ __forceinline__ void init(const GemmParams &P, const GemmJobDev *sj, int first,
-                                         int last, int r) {
+                                         int last, int rank_rows, int r) {
         jobs = sj;
         tile = first;
         t_end = last;
         kb = 0;
+        row0 = rank_rows;
         bind(P, r);
     }
     __device__ __forceinline__ void advance(const GemmParams &P, int r) {
@@ -304,30 +420,58 @@ template <int WF> struct SzCursor {
             bind(P, r);
         }
     }
-    // (s, z) of the current position
-    __device__ __forceinline__ void load(const GemmParams &P, float &s, float &z) const {
-        s = 0.0f;
-        z = 0.0f;
+    // Raw words of the scale and zero at the current position (fp16 bits,
+    // fp32 bits, or the packed range word).  Only the load is issued here;
+    // decode() converts them when the block is dequantized, kLook blocks
+    // later: converting at once would stall the warp on the load.
+    __device__ __forceinline__ void load(const GemmParams &P, uint32_t &sw, uint32_t &zw) const {
+        sw = 0u;
+        zw = 0u;
         if (!srow) return;
         if constexpr (WF == kPacked) {
-            s = __half2float(__ldg(static_cast<const __half *>(srow) + kb));
-            z = __half2float(__ldg(static_cast<const __half *>(zrow) + kb));
+            sw = __ldg(static_cast<const unsigned short *>(srow) + kb);
+            zw = __ldg(static_cast<const unsigned short *>(zrow) + kb);
         } else {
             if (P.bits == 16) return;
             const int gi = (kb * kBK) / group;
             if (P.range) {
-                const float2 rg =
-                    range_of_word(__ldg(static_cast<const uint32_t *>(srow) + gi));
-                const float2 sz = rtn_params_from_range(rg.x, rg.y, P.bits);
-                s = sz.x;
-                z = sz.y;
+                sw = __ldg(static_cast<const uint32_t *>(srow) + gi);
+                zw = 1u;          // marks a loaded range (a zero word is a valid range)
             } else {
-                s = __ldg(static_cast<const float *>(srow) + gi);
-                z = __ldg(static_cast<const float *>(zrow) + gi);
+                sw = __ldg(static_cast<const uint32_t *>(srow) + gi);
+                zw = __ldg(static_cast<const uint32_t *>(zrow) + gi);
             }
         }
     }
 };
+
+template <int WF>
+__device__ __forceinline__ void decode_sz(const GemmParams &P, uint32_t sw, uint32_t zw,
+                                          float &s, float &z) {
+    if constexpr (WF == kPacked) {
+        s = __half2float(__ushort_as_half((unsigned short)sw));
+        z = __half2float(__ushort_as_half((unsigned short)zw));
+    } else if (P.range) {
+        s = 0.0f;
+        z = 0.0f;
+        if (zw) {
+            const float2 rg = range_of_word(sw);
+            const float2 sz = rtn_params_from_range(rg.x, rg.y, P.bits);
+            s = sz.x;
+            z = sz.y;
+        }
+    } else {
+        s = __uint_as_float(sw);
+        z = __uint_as_float(zw);
+    }
+}
+
+// Offset of 16-byte chunk c (0..7) of row r in a 128B-swizzled K-major tile
+// of 128-byte rows (8-row atoms of 1024 bytes): the layout a TMA box with
+// SWIZZLE_128B writes and the MMA's shared-memory descriptor reads.
+__device__ __forceinline__ int sw128_off(int r, int c) {
+    return (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4);
+}
 
 template <int BNX, int WF>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -336,16 +480,24 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t *bar_area = smem + C::kStages * C::kStageBytes;
-    uint64_t *full_tma = reinterpret_cast<uint64_t *>(bar_area);
-    uint64_t *full_dq = full_tma + C::kStages;
-    uint64_t *empty = full_dq + C::kStages;
-    uint64_t *acc_full = empty + C::kStages;
-    uint64_t *acc_empty = acc_full + 2;
+    uint8_t *a_ring = smem + C::kAOff;
+    uint8_t *x_ring = smem + C::kXOff;
+    uint8_t *w_ring = smem + C::kWOff;
+    uint64_t *w_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *w_empty = w_full + C::kWStages;
+    uint64_t *x_full = w_empty + C::kWStages;
+    uint64_t *x_empty = x_full + C::kXStages;
+    uint64_t *a_full = x_empty + C::kXStages;    // used in the first CTA of the pair
+    uint64_t *a_empty = a_full + C::kAStages;
+    uint64_t *acc_full = a_empty + C::kAStages;
+    uint64_t *acc_empty = acc_full + 2;          // used in the first CTA of the pair
     uint64_t *mma_done = acc_empty + 2;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(mma_done + 1);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1) + 1;
-    GemmJobDev *sjobs = reinterpret_cast<GemmJobDev *>(mma_done + 2);
+    GemmJobDev *sjobs = reinterpret_cast<GemmJobDev *>(smem + C::kBarOff + 512);
+    static_assert((2 * C::kWStages + 2 * C::kXStages + 2 * C::kAStages + 5) * 8 + 8 <= 512,
+                  "barrier block");
+    static_assert(512 + kMaxJobs * sizeof(GemmJobDev) <= C::kBarBytes, "job table");
     {
         const uint32_t *src = reinterpret_cast<const uint32_t *>(P.jobs);
         uint32_t *dst = reinterpret_cast<uint32_t *>(sjobs);
@@ -354,167 +506,188 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
     }
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t_begin = P.cta_begin[blockIdx.x], t_end = P.cta_begin[blockIdx.x + 1];
+    const int rank = (int)cluster_rank();           // 0: issues the MMAs
+    const int pair = (int)cluster_id();
+    const int t_begin = P.pair_begin[pair], t_end = P.pair_begin[pair + 1];
+    const int rank_rows = rank * kBM;               // this CTA's weight rows in a tile
+    const int rank_xrows = rank * C::kXHalf;        // this CTA's x rows in a tile
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(smem_u32(&full_tma[s]), 1);
-            mbar_init(smem_u32(&full_dq[s]), kDqWarps);
-            mbar_init(smem_u32(&empty[s]), 1);
+        for (int s = 0; s < C::kWStages; ++s) {
+            mbar_init(smem_u32(&w_full[s]), 1);
+            mbar_init(smem_u32(&w_empty[s]), kDqWarps);
+        }
+        for (int s = 0; s < C::kXStages; ++s) {
+            mbar_init(smem_u32(&x_full[s]), 1);
+            mbar_init(smem_u32(&x_empty[s]), 1);
+        }
+        for (int s = 0; s < C::kAStages; ++s) {
+            mbar_init(smem_u32(&a_full[s]), 2 * kDqWarps / C::kDqGroups);  // one group per CTA
+            mbar_init(smem_u32(&a_empty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&acc_full[b]), 1);
-            mbar_init(smem_u32(&acc_empty[b]), kEpWarps);
+            mbar_init(smem_u32(&acc_empty[b]), 2 * kEpWarps);
         }
         mbar_init(smem_u32(mma_done), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == kMmaWarp) {
-        tc::alloc(smem_u32(tmem_slot), C::kTmemCols);
-    }
+    if (warp == kMmaWarp) tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
     tc::fence_before();
     __syncthreads();
+    cluster_sync();      // the partner's barriers exist before anything arrives on them
     tc::fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == kTmaWarp) {
+    if (warp == kCodeWarp || warp == kXWarp) {
+        // producers: one lane each; the code producer fills the weight
+        // ring, the activation producer the x ring
         if (lane == 0) {
-            uint32_t g = 0;                       // k-block counter over tiles
-            uint32_t armed = 0;                   // stages with a load issued
+            const bool codes = warp == kCodeWarp;
+            const int stages = codes ? C::kWStages : C::kXStages;
+            uint64_t *full = codes ? w_full : x_full;
+            uint64_t *empty = codes ? w_empty : x_empty;
+            uint8_t *ring = codes ? w_ring : x_ring;
+            const int bytes = codes ? C::kWBytes : C::kXBytes;
+            uint32_t g = 0;
             for (int tile = t_begin; tile < t_end && !*abort_flag; ++tile) {
-                const int j = find_job(sjobs, P.count, tile);
-                const GemmJobDev &J = sjobs[j];
-                const int local = tile - J.tile_begin;
-                const int nb = local / J.xblocks, xb = local % J.xblocks;
-                const int kblocks = J.K / kBK;
-                if (tile + 1 < t_end) {
-                    // the next tile's weights (and their scales/zeros) to L2
-                    // while this one streams, unless it reuses these rows
-                    const int j2 = find_job(sjobs, P.count, tile + 1);
-                    const GemmJobDev &J2 = sjobs[j2];
-                    const int nb2 = (tile + 1 - J2.tile_begin) / J2.xblocks;
-                    if (j2 != j || nb2 != nb) {
-                        const int kb2 = J2.K / kBK;
-                        for (int q = 0; q < kb2; ++q)
-                            tma_prefetch_2d(&P.wmap[j2], WF == kPacked ? q * (kBK / 2) : q * kBK,
-                                            nb2 * kBM);
-                        const int64_t G2 = J2.K / J2.group;
-                        const int rows = min(kBM, J2.N - nb2 * kBM);
-                        const int64_t es = WF == kPacked ? 2 : 4;
-                        const int64_t bytes = rows * G2 * es;
-                        const char *sb = static_cast<const char *>(J2.s) + (int64_t)nb2 * kBM * G2 * es;
-                        const char *zb = J2.z ? static_cast<const char *>(J2.z) +
-                                                    (int64_t)nb2 * kBM * G2 * es
-                                              : nullptr;
-                        for (int64_t o = 0; o < bytes; o += 128) {
-                            if (P.bits != 16 || WF == kPacked) {
+                const TilePos tp = tile_pos(sjobs, P.count, tile);
+                if (codes && tile + 1 < t_end) {
+                    // scales/zeros of the next tile's rows to L2 (the dequant
+                    // warps read them a few stages ahead)
+                    const TilePos tn = tile_pos(sjobs, P.count, tile + 1);
+                    if (tn.j != tp.j || tn.nb != tp.nb) {
+                        const GemmJobDev &J2 = sjobs[tn.j];
+                        const int row = tn.nb * kPairRows + rank_rows;
+                        if (row < J2.N && !(WF == kRuntime && P.bits == 16)) {
+                            const int64_t G2 = J2.K / J2.group;
+                            const int64_t es = WF == kPacked ? 2 : 4;
+                            const int64_t n = (int64_t)min(kBM, J2.N - row) * G2 * es;
+                            const char *sb = static_cast<const char *>(J2.s) + row * G2 * es;
+                            const char *zb =
+                                J2.z ? static_cast<const char *>(J2.z) + row * G2 * es : nullptr;
+                            for (int64_t o = 0; o < n; o += 128) {
                                 prefetch_l2(sb + o);
                                 if (zb) prefetch_l2(zb + o);
                             }
                         }
                     }
                 }
-                for (int kb = 0; kb < kblocks; ++kb, ++g) {
-                    const int s = g % C::kStages;
-                    const uint32_t ph = (g / C::kStages) & 1;
-                    if (!mbar_wait<false>(smem_u32(&empty[s]), ph ^ 1, abort_flag)) break;
-                    uint8_t *st = smem + s * C::kStageBytes;
-                    const uint32_t fb = smem_u32(&full_tma[s]);
-                    if constexpr (WF == kPacked) {
-                        mbar_expect_tx(fb, C::kBBytes + C::kCBytes);
-                        tma_load_2d(smem_u32(st + C::kABytes + C::kBBytes), &P.wmap[j],
-                                    kb * (kBK / 2), nb * kBM, fb);
-                    } else {
-                        mbar_expect_tx(fb, C::kBBytes + C::kABytes);
-                        tma_load_2d(smem_u32(st), &P.wmap[j], kb * kBK, nb * kBM, fb);
+                bool ok = true;
+                const int step = codes ? C::kGroup : 1;
+                for (int kb = 0; kb < tp.kblocks; kb += step, ++g) {
+                    const int s = g % stages;
+                    const uint32_t ph = (g / stages) & 1;
+                    if (!mbar_wait<kBackoff>(smem_u32(&empty[s]), ph ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
                     }
-                    tma_load_2d(smem_u32(st + C::kABytes), &P.xmap[j], kb * kBK, xb * BNX, fb);
-                    armed |= 1u << s;
+                    const uint32_t fb = smem_u32(&full[s]);
+                    mbar_expect_tx(fb, bytes);
+                    const uint32_t dst = smem_u32(ring + s * bytes);
+                    if (codes)
+                        tma_load_2d(dst, &P.wmap[tp.j],
+                                    WF == kPacked ? kb * (kBK / 2) : kb * kBK,
+                                    tp.nb * kPairRows + rank_rows, fb);
+                    else
+                        tma_load_2d(dst, &P.xmap[tp.j], kb * kBK,
+                                    tp.xb * BNX + rank_xrows, fb);
                 }
+                if (!ok) break;
             }
             // drain: every load this thread issued has landed before exit
             // (on the normal path each stage was consumed, so these pass)
-            for (uint32_t q = 0; q < (uint32_t)C::kStages && g > 0; ++q) {
-                if (!(armed & (1u << q))) continue;
-                // the last use of stage q had index g_last = largest g' < g with
-                // g' % kStages == q
-                const uint32_t gl = (g - 1) - (((g - 1) % C::kStages + C::kStages - q) %
-                                               C::kStages);
-                const long long t0 = clock64();
-                while (!mbar_try(smem_u32(&full_tma[q]), (gl / C::kStages) & 1) &&
-                       clock64() - t0 < kWaitCycles) {
-                }
+            for (uint32_t q = 0; q < (uint32_t)stages && g > 0; ++q) {
+                if (q >= g) break;
+                // the last use of stage q had index gl = largest g' < g with
+                // g' % stages == q
+                const uint32_t gl = (g - 1) - (((g - 1) % stages + stages - q) % stages);
+                mbar_drain(smem_u32(&full[q]), (gl / stages) & 1);
             }
         }
     } else if (warp == kMmaWarp) {
-        // The whole warp walks the tiles and waits; one elected lane issues a
-        // stage's four MMAs and commits.  Descriptors are formed once and
-        // advanced by constant offsets (16-byte units of the start address):
-        // an MMA issued from a lone diverged lane with descriptors rebuilt per
-        // instruction costs several times the tensor core's own time.
-        const uint64_t adesc0 = tc::sw128_desc(smem_u32(smem));
-        const uint64_t bdesc0 = tc::sw128_desc(smem_u32(smem + C::kABytes));
-        uint32_t g = 0;
-        int lt = 0;
-        for (int tile = t_begin;
-             tile < t_end && !__shfl_sync(0xffffffffu, (int)*abort_flag, 0); ++tile, ++lt) {
-            const int j = find_job(sjobs, P.count, tile);
-            const int kblocks = sjobs[j].K / kBK;
-            const int buf = lt & 1;
-            const uint32_t aph = (lt >> 1) & 1;
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait<false>(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag)))
-                break;
-            tc::fence_after();
-            const uint32_t d_tmem = tmem_base + buf * BNX;
-            bool ok = true;
-            for (int kb = 0; kb < kblocks; ++kb, ++g) {
-                const int s = g % C::kStages;
-                const uint32_t ph = (g / C::kStages) & 1;
-                bool w = mbar_wait<false>(smem_u32(&full_tma[s]), ph, abort_flag);
-                if (w) w = mbar_wait<false>(smem_u32(&full_dq[s]), ph, abort_flag);
-                if (!__all_sync(0xffffffffu, w)) {
-                    ok = false;
+        if (rank == 0) {
+            // The whole warp walks the tiles and waits; one elected lane
+            // issues a stage's four MMAs and commits.  Descriptors are formed
+            // once and advanced by constant offsets (16-byte units of the
+            // start address): an MMA issued from a lone diverged lane with
+            // descriptors rebuilt per instruction costs several times the
+            // tensor core's own time.
+            const uint64_t adesc0 = tc::sw128_desc(smem_u32(a_ring));
+            const uint64_t bdesc0 = tc::sw128_desc(smem_u32(x_ring));
+            uint32_t g = 0;
+            int lt = 0;
+            for (int tile = t_begin;
+                 tile < t_end && !__shfl_sync(0xffffffffu, (int)*abort_flag, 0); ++tile, ++lt) {
+                const int kblocks = sjobs[find_job(sjobs, P.count, tile)].K / kBK;
+                const int buf = lt & 1;
+                const uint32_t aph = (lt >> 1) & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait<kSpin>(smem_u32(&acc_empty[buf]),
+                                                                     aph ^ 1, abort_flag)))
                     break;
-                }
                 tc::fence_after();
-                const uint64_t so = (uint64_t)((s * C::kStageBytes) >> 4);
-                if (tc::elect_one()) {
+                const uint32_t d_tmem = tmem_base + buf * BNX;
+                bool ok = true;
+                for (int kb = 0; kb < kblocks; ++kb, ++g) {
+                    const int sx = g % C::kXStages, sa = g % C::kAStages;
+                    bool w = mbar_wait<kSpin>(smem_u32(&x_full[sx]), (g / C::kXStages) & 1,
+                                              abort_flag);
+                    if (w)
+                        w = mbar_wait<kSpin>(smem_u32(&a_full[sa]),
+                                                   (g / C::kAStages) & 1, abort_flag);
+                    if (!__all_sync(0xffffffffu, w)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after();
+                    const uint64_t ao = (uint64_t)((sa * C::kABytes) >> 4);
+                    const uint64_t bo = (uint64_t)((sx * C::kXBytes) >> 4);
+                    if (tc::elect_one()) {
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc::mma_bf16_ss(d_tmem, adesc0 + so + 2 * kk, bdesc0 + so + 2 * kk,
-                                        C::kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
-                    tc::commit(smem_u32(&empty[s]));        // stage reusable
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            mma_pair(d_tmem, adesc0 + ao + 2 * kk, bdesc0 + bo + 2 * kk,
+                                     C::kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        commit_pair(smem_u32(&x_empty[sx]));    // x stage reusable
+                        commit_pair(smem_u32(&a_empty[sa]));    // A buffer reusable
+                    }
+                    __syncwarp();
                 }
+                if (!ok) break;
+                if (tc::elect_one()) commit_pair(smem_u32(&acc_full[buf]));   // tile done
                 __syncwarp();
             }
-            if (!ok) break;
-            if (tc::elect_one()) tc::commit(smem_u32(&acc_full[buf]));   // tile accumulated
+            // every MMA issued has finished before TMEM is freed
+            if (tc::elect_one()) commit_local(smem_u32(mma_done));
+            __syncwarp();
+            if (lane == 0) mbar_drain(smem_u32(mma_done), 0);
             __syncwarp();
         }
-        // every MMA issued has finished before TMEM is freed
-        if (tc::elect_one()) tc::commit(smem_u32(mma_done));
-        __syncwarp();
-        if (lane == 0) {
-            const long long t0 = clock64();
-            while (!mbar_try(smem_u32(mma_done), 0) && clock64() - t0 < kWaitCycles) {
-            }
-        }
-        __syncwarp();
     } else if (warp < kDqWarp0 + kDqWarps) {
-        // dequant: thread -> (row r, half h) of the 128 x 64 weight tile.
-        // Scale/zero come from global memory.  They are fetched kLook blocks
-        // ahead into a window of kLook register slots indexed at compile
-        // time (slot j serves blocks g with g % kLook == j), so no register
-        // copy waits on a load that is still in flight.
-        const int t = threadIdx.x - 32 * kDqWarp0;
-        const int r = t & (kBM - 1), h = t >> 7;
+        // dequant: kDqGroups groups of warps take alternate stages (group
+        // gi the stages g with g % kDqGroups == gi), so with two groups a
+        // group has two stages' time for one (packed codes; the runtime
+        // requantization, heavier in registers, runs one group).  Thread ->
+        // (row r, part) of the 128 x 64 weight tile, kCpt 16-byte chunks
+        // (8 k values each) per thread.  Scale/zero come from
+        // global memory, fetched kLook blocks ahead into a window of kLook
+        // register slots indexed at compile time (slot j serves blocks g
+        // with g % kLook == j), so no register copy waits on a load in flight.
+        constexpr int kGroupWarps = kDqWarps / C::kDqGroups;
+        constexpr int kCpt = 2 * C::kDqGroups;          // chunks per thread
+        const int dw = warp - kDqWarp0;
+        const int gi = dw / kGroupWarps;
+        const int t = (dw % kGroupWarps) * 32 + lane;
+        const int r = t & (kBM - 1), part = t >> 7;
         const float L = (float)((1 << (P.bits & 15)) - 1);
         const bool pass = WF == kRuntime && P.bits == 16;
+        // In the second CTA the first warp of each group also waits for the
+        // CTA's own x stage before arriving: the MMA issued by the first CTA
+        // reads it.
+        const bool x_gate = rank == 1 && dw % kGroupWarps == 0;
         SzCursor<WF> la;                    // look-ahead cursor
-        la.init(P, sjobs, t_begin, t_end, r);
-        float sq[kLook], zq[kLook];
+        la.init(P, sjobs, t_begin, t_end, rank_rows, r);
+        uint32_t sq[kLook], zq[kLook];
 #pragma unroll
         for (int i = 0; i < kLook; ++i) {
             la.load(P, sq[i], zq[i]);
@@ -527,67 +700,89 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
             const GemmJobDev &J = sjobs[find_job(sjobs, P.count, tile)];
             const int nb = (tile - J.tile_begin) / J.xblocks;
             kblocks = J.K / kBK;
-            valid = nb * kBM + r < J.N;
+            valid = nb * kPairRows + rank_rows + r < J.N;
         };
         bind();
-        uint32_t g = 0;
+        uint32_t g = 0, cg = 0;            // stages, weight boxes consumed
         bool ok = true;
+        int aoff[kCpt];
+#pragma unroll
+        for (int i = 0; i < kCpt; ++i) aoff[i] = sw128_off(r, kCpt * part + i);
         while (ok && tile < t_end && !*abort_flag) {
 #pragma unroll
             for (int j = 0; j < kLook; ++j) {
                 if (tile >= t_end) break;
-                const float sf = sq[j], zf = zq[j];
-                la.load(P, sq[j], zq[j]);          // refill slot j, kLook ahead
-                la.advance(P, r);
-                const int s = g % C::kStages;
-                const uint32_t ph = (g / C::kStages) & 1;
-                if (!mbar_wait(smem_u32(&full_tma[s]), ph, abort_flag)) {
+                const int sw = cg % C::kWStages;
+                // Both groups wait for every weight box, the one whose blocks
+                // they skip too: a barrier's parity test is only sound for a
+                // waiter at most one phase ahead, and a group that skipped
+                // boxes could otherwise release a slot's next phase early.
+                if (!mbar_wait(smem_u32(&w_full[sw]), (cg / C::kWStages) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                uint8_t *st = smem + s * C::kStageBytes;
-                uint8_t *arow = st + (r >> 3) * 1024 + (r & 7) * 128;
-                if (!valid) {
+                if (j % C::kDqGroups == gi) {   // kLook % kDqGroups == 0: g ≡ j
+                    float sf, zf;
+                    decode_sz<WF>(P, sq[j], zq[j], sf, zf);
+                    const uint8_t *wt = w_ring + sw * C::kWBytes;
+                    uint4 o[kCpt];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int chunk = h * 4 + i;
-                        *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                } else if constexpr (WF == kRuntime) {
-                    // the 8 fp16 of each chunk are replaced by their 8 bf16 w'
+                    for (int i = 0; i < kCpt; ++i) o[i] = make_uint4(0, 0, 0, 0);
+                    if (valid) {
+                        if constexpr (WF == kRuntime) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint4 *p = reinterpret_cast<uint4 *>(arow + (((h * 4 + i) ^ (r & 7)) << 4));
-                        *p = requant8(*p, sf, zf, L, pass);
-                    }
-                } else {
-                    const uint4 codes = *reinterpret_cast<const uint4 *>(
-                        st + C::kABytes + C::kBBytes + r * 32 + h * 16);
-                    const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
-                    if (fabsf(zf) <= 128.0f) {
-                        const __nv_bfloat16 zb1 = __float2bfloat16_rn(128.0f + zf);
-                        const __nv_bfloat16 sb1 = __float2bfloat16_rn(sf);
-                        const __nv_bfloat162 zb = __halves2bfloat162(zb1, zb1);
-                        const __nv_bfloat162 sb = __halves2bfloat162(sb1, sb1);
+                            for (int i = 0; i < kCpt; ++i)
+                                o[i] = requant8(*reinterpret_cast<const uint4 *>(wt + aoff[i]), sf,
+                                                zf, L, pass);
+                        } else {
+                            static_assert(C::kDqGroups == 2, "packed: one 16-byte code chunk");
+                            // 16 bytes at (kb % 4) * 32 + part * 16 of the row's
+                            // 128 (128B-swizzled)
+                            const int chunk = (kb % C::kGroup) * 2 + part;
+                            const uint4 cw = *reinterpret_cast<const uint4 *>(
+                                wt + r * 128 + ((chunk ^ (r & 7)) << 4));
+                            const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+                            if (fabsf(zf) <= 128.0f) {
+                                const __nv_bfloat16 zb1 = __float2bfloat16_rn(128.0f + zf);
+                                const __nv_bfloat16 sb1 = __float2bfloat16_rn(sf);
+                                const __nv_bfloat162 zb = __halves2bfloat162(zb1, zb1);
+                                const __nv_bfloat162 sb = __halves2bfloat162(sb1, sb1);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int chunk = h * 4 + i;
-                            *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) =
-                                dequant8(cw[i], zb, sb);
-                        }
-                    } else {
+                                for (int i = 0; i < 4; ++i) o[i] = dequant8(w4[i], zb, sb);
+                            } else {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int chunk = h * 4 + i;
-                            *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) =
-                                dequant8_wide(cw[i], zf, sf);
+                                for (int i = 0; i < 4; ++i) o[i] = dequant8_wide(w4[i], zf, sf);
+                            }
                         }
                     }
+                    const int sa = g % C::kAStages;
+                    // completed by the first CTA's commit (multicast): no sleep hint
+                    if (!mbar_wait<kBackoff>(smem_u32(&a_empty[sa]), ((g / C::kAStages) & 1) ^ 1,
+                                             abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *at = a_ring + sa * C::kABytes;
+#pragma unroll
+                    for (int i = 0; i < kCpt; ++i) *reinterpret_cast<uint4 *>(at + aoff[i]) = o[i];
+                    fence_proxy_async_smem();
+                    if (x_gate && !mbar_wait(smem_u32(&x_full[g % C::kXStages]),
+                                             (g / C::kXStages) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(in_leader(smem_u32(&a_full[sa])));
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&full_dq[s]));
+                la.load(P, sq[j], zq[j]);          // refill slot j, kLook ahead
+                la.advance(P, r);
+                // the weight box is released by both groups after its last
+                // block (this group's values are in registers or stored)
+                if (kb % C::kGroup == C::kGroup - 1 || kb == kblocks - 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&w_empty[sw]));
+                    ++cg;
+                }
                 ++g;
                 if (++kb == kblocks) {
                     kb = 0;
@@ -602,16 +797,14 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
         const int q = warp & 3, hh = (warp - kEpWarp0) >> 2;
         int lt = 0;
         for (int tile = t_begin; tile < t_end && !*abort_flag; ++tile, ++lt) {
-            const int j = find_job(sjobs, P.count, tile);
-            const GemmJobDev &J = sjobs[j];
-            const int local = tile - J.tile_begin;
-            const int nb = local / J.xblocks, xb = local % J.xblocks;
+            const TilePos tp = tile_pos(sjobs, P.count, tile);
+            const GemmJobDev &J = sjobs[tp.j];
             const int buf = lt & 1;
             const uint32_t aph = (lt >> 1) & 1;
-            if (!mbar_wait(smem_u32(&acc_full[buf]), aph, abort_flag)) break;
+            if (!mbar_wait<kBackoff>(smem_u32(&acc_full[buf]), aph, abort_flag)) break;
             tc::fence_after();
-            const int n = nb * kBM + 32 * q + lane;
-            const int m0 = xb * BNX;
+            const int n = tp.nb * kPairRows + rank_rows + 32 * q + lane;
+            const int m0 = tp.xb * BNX;
 #pragma unroll 1
             for (int c = hh * (BNX / 64); c < (hh + 1) * (BNX / 64); ++c) {
                 uint32_t v[32];
@@ -626,15 +819,18 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
             }
             tc::fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[buf]));
+            if (lane == 0) mbar_arrive_cluster(in_leader(smem_u32(&acc_empty[buf])));
         }
     }
 
     tc::fence_before();
     __syncthreads();
+    // neither CTA leaves (or frees TMEM) while the pair's MMAs, commits or
+    // arrivals may still touch its memory
+    cluster_sync();
     if (warp == kMmaWarp) {
         tc::fence_after();
-        tc::dealloc(tmem_base, C::kTmemCols);
+        tmem_dealloc_pair(tmem_base, C::kTmemCols);
     }
 }
 
@@ -669,10 +865,11 @@ bool encode_codes(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m,
                   const void *w, int64_t N, int64_t K) {
     cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
     cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    cuuint32_t box[2] = {(cuuint32_t)(kBK / 2), (cuuint32_t)kBM};
+    // four 64-blocks (128 bytes) of 128 rows, 128B-swizzled
+    cuuint32_t box[2] = {(cuuint32_t)(2 * kBK), (cuuint32_t)kBM};
     cuuint32_t es[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(w), dims, strides,
-               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -690,10 +887,10 @@ bool encode_w16(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const voi
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Contiguous tile ranges per CTA that minimise the costliest range (binary
-// search on the bound, greedy fill).  A tile costs its K/64 stages plus a
-// fixed share for its epilogue.
-void partition_tiles(GemmParams &P, const std::vector<double> &tcost, int grid) {
+// Contiguous tile ranges per CTA pair that minimise the costliest range
+// (binary search on the bound, greedy fill).  A tile costs its K/64 stages
+// plus a fixed share for its epilogue.
+void partition_tiles(GemmParams &P, const std::vector<double> &tcost, int pairs) {
     const int n = (int)tcost.size();
     double total = 0, tmax = 0;
     for (double c : tcost) {
@@ -701,26 +898,26 @@ void partition_tiles(GemmParams &P, const std::vector<double> &tcost, int grid) 
         tmax = std::max(tmax, c);
     }
     auto fill = [&](double T, bool out) -> int {
-        int ctas = 1;
+        int used = 1;
         double cur = 0;
-        if (out) P.cta_begin[0] = 0;
+        if (out) P.pair_begin[0] = 0;
         for (int i = 0; i < n; ++i) {
             if (cur > 0 && cur + tcost[i] > T) {
-                if (out && ctas < grid) P.cta_begin[ctas] = i;
-                ++ctas;
+                if (out && used < pairs) P.pair_begin[used] = i;
+                ++used;
                 cur = 0;
             }
             cur += tcost[i];
         }
-        return ctas;
+        return used;
     };
-    double lo = std::max(tmax, total / grid), hi = total + tmax;
+    double lo = std::max(tmax, total / pairs), hi = total + tmax;
     for (int it = 0; it < 60 && hi - lo > 0.5; ++it) {
         const double mid = 0.5 * (lo + hi);
-        if (fill(mid, false) <= grid) hi = mid; else lo = mid;
+        if (fill(mid, false) <= pairs) hi = mid; else lo = mid;
     }
-    const int used = std::min(fill(hi, true), grid);
-    for (int c = used; c <= grid; ++c) P.cta_begin[c] = n;
+    const int used = std::min(fill(hi, true), pairs);
+    for (int c = used; c <= pairs; ++c) P.pair_begin[c] = n;
 }
 
 template <int BNX, int WF>
@@ -730,17 +927,35 @@ bc_status launch_cfg(const GemmJob *jobs, int count, int64_t M, int bits, bool r
     auto enc = get_encoder();
     if (!enc) return BC_ERR_CUDA;
     static std::mutex mu;
-    static int attr_set[64] = {};
+    static int max_pairs[64] = {};     // per device, 0 = not yet set up
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return BC_ERR_CUDA;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     {
         std::lock_guard<std::mutex> lock(mu);
-        if (!attr_set[dev]) {
+        if (!max_pairs[dev]) {
             if (cudaFuncSetAttribute(gemm_kernel<BNX, WF>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      C::kSmem) != cudaSuccess)
                 return BC_ERR_CUDA;
-            attr_set[dev] = 1;
+            // pairs that can be resident at once (one CTA per SM)
+            cfg.gridDim = dim3(2 * kMaxPairs);
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<BNX, WF>, &cfg) !=
+                    cudaSuccess ||
+                clusters < 1)
+                return BC_ERR_CUDA;
+            max_pairs[dev] = std::min({clusters, std::max(1, sm_count / 2), kMaxPairs});
         }
     }
     thread_local GemmParams *Pp = nullptr;
@@ -754,13 +969,13 @@ bc_status launch_cfg(const GemmJob *jobs, int count, int64_t M, int bits, bool r
         tcost.clear();
         for (int i = 0; i < n; ++i) {
             const GemmJob &J = jobs[b + i];
-            if (!encode_x(enc, &P.xmap[i], J.x, M, J.K, BNX)) return BC_ERR_CUDA;
+            if (!encode_x(enc, &P.xmap[i], J.x, M, J.K, C::kXHalf)) return BC_ERR_CUDA;
             const bool ok = WF == kPacked ? encode_codes(enc, &P.wmap[i], J.w, J.N, J.K)
                                           : encode_w16(enc, &P.wmap[i], J.w, J.N, J.K);
             if (!ok) return BC_ERR_CUDA;
             P.jobs[i] = GemmJobDev{J.s, J.z, J.y, (int)J.N, (int)J.K, (int)J.group, tiles,
                                    xblocks};
-            const int nt = (int)((J.N + kBM - 1) / kBM) * xblocks;
+            const int nt = (int)((J.N + kPairRows - 1) / kPairRows) * xblocks;
             tiles += nt;
             // cost in stages: K/64 of MMA plus the epilogue (BNX/32 loads of
             // 32 columns and their stores), about two stages' worth
@@ -771,9 +986,10 @@ bc_status launch_cfg(const GemmJob *jobs, int count, int64_t M, int bits, bool r
         P.M = (int)M;
         P.bits = bits;
         P.range = range ? 1 : 0;
-        const int grid = std::max(1, std::min({tiles, sm_count, kMaxCtas}));
-        partition_tiles(P, tcost, grid);
-        gemm_kernel<BNX, WF><<<grid, kThreads, C::kSmem, s>>>(P);
+        const int pairs = std::max(1, std::min(tiles, max_pairs[dev]));
+        partition_tiles(P, tcost, pairs);
+        cfg.gridDim = dim3(2 * pairs);
+        if (cudaLaunchKernelEx(&cfg, gemm_kernel<BNX, WF>, P) != cudaSuccess) return BC_ERR_CUDA;
         bc_status st = cuda_status();
         if (st != BC_OK) return st;
     }
