@@ -31,7 +31,7 @@
 //     (128B-swizzled, K-major) into the activation ring, which the MMA
 //     frees;
 //   * sixteen dequant warps (two groups of eight taking alternate blocks)
-//     form bf16 w' = (q - z) * s into one of four A buffers in the
+//     form bf16 w' = (q - z) * s into one of six A buffers in the
 //     128B-swizzled K-major layout the MMA reads (packed:
 //     exact q - z in bf16 arithmetic and one rounding for the scale;
 //     runtime: the exact RTN code of each fp16 weight, then one rounding of
@@ -117,11 +117,11 @@ template <int BNX, int WF> struct Cfg {
     static constexpr int kWRow = WF == kPacked ? 32 * kGroup : 128;   // bytes per row
     static constexpr int kWBytes = kBM * kWRow;                   // 16 KB
     static constexpr int kABytes = kBM * 128;                    // 16 KB
-    static constexpr int kAStages = 4;
+    static constexpr int kAStages = WF == kPacked ? 6 : 4;
     // even: each dequant group sees every other phase of an x (and A)
     // barrier, and the parity test is sound only if the ring depth keeps a
     // slot's stages in one group
-    static constexpr int kXStages = BNX == 256 ? (WF == kPacked ? 6 : 4) : 8;
+    static constexpr int kXStages = BNX == 256 ? 4 : (WF == kPacked ? 6 : 8);
     static constexpr int kWStages = WF == kPacked ? (BNX == 256 ? 3 : 4) : 5;
     static constexpr int kAOff = 0;
     static constexpr int kXOff = kAOff + kAStages * kABytes;
@@ -756,8 +756,9 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
                         }
                     }
                     const int sa = g % C::kAStages;
-                    // completed by the first CTA's commit (multicast): no sleep hint
-                    if (!mbar_wait<kBackoff>(smem_u32(&a_empty[sa]), ((g / C::kAStages) & 1) ^ 1,
+                    // completed by the first CTA's commit (multicast): polled, the
+                    // MMA waits on what this warp writes next
+                    if (!mbar_wait<kSpin>(smem_u32(&a_empty[sa]), ((g / C::kAStages) & 1) ^ 1,
                                              abort_flag)) {
                         ok = false;
                         break;
