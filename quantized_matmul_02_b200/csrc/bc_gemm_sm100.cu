@@ -45,8 +45,8 @@
 //     (tcgen05.ld) and store y with coalesced rows while the next tile
 //     accumulates into the second TMEM buffer.
 // The kernel is persistent (one cluster per SM pair) and spans every matrix
-// of a grouped launch; each pair owns a contiguous range of tiles chosen on
-// the host so that the ranges cost about the same.  All waits are bounded:
+// of a grouped launch; the pairs walk one tile list side by side (see
+// pair_tile), so that the tiles in flight share their activation block.  All waits are bounded:
 // a wait that runs out records a timeout, the CTA stops, waits (bounded) for
 // its own copies and MMAs in flight, meets its partner at the cluster
 // barrier and frees its TMEM.  No load uses cluster multicast: every CTA
@@ -92,15 +92,17 @@ struct GemmJobDev {
     float *y;
     int N, K, group;       // group: 64, or K (runtime per channel)
     int tile_begin;
-    int xblocks;           // ceil(M / BNX)
+    int nblocks;           // ceil(N / 256): weight blocks (fastest in the tile order)
 };
 
 struct __align__(64) GemmParams {
     CUtensorMap xmap[kMaxJobs];     // bf16 x [M][K], box {64, BNX/2}, SW128
     CUtensorMap wmap[kMaxJobs];     // packed u8 [N][K/2] box {128, 128}; fp16 W [N][K] box {64, 128}; SW128
     GemmJobDev jobs[kMaxJobs];
-    int pair_begin[kMaxPairs + 1];  // tile range of each CTA pair
     int count, total_tiles, M;
+    int pairs;                      // CTA pairs launched
+    int ranges;                     // 1: pair p takes tiles [pair_begin[p], pair_begin[p+1])
+    int pair_begin[kMaxPairs + 1];
     int bits;                       // runtime: 2..8 or 16 (passthrough)
     int range;                      // runtime: s holds per-group ranges
 };
@@ -359,6 +361,30 @@ __device__ __forceinline__ int find_job(const GemmJobDev *jobs, int count, int t
     return lo;
 }
 
+// The tiles of a launch form one list: matrices by decreasing K, within a
+// matrix x block by x block, and within an x block its 256-row weight
+// blocks.  Pair p takes the list in rounds of `pairs` tiles, forward in even
+// rounds and backward in odd ones (tile i * pairs + p, or + pairs - 1 - p):
+// the pairs run through the list side by side, so at any time they work on
+// neighbouring tiles, which share one x block (read from DRAM once, then
+// from L2 by every pair), and the snake order evens out the extra cost of
+// the long-K tiles dealt first.  (Contiguous per-pair ranges put every pair
+// on a different matrix: at M = 2048 their x blocks did not fit in L2 and
+// were re-read from DRAM, 4.8 GB of reads per 24-layer step against 0.9 GB
+// of inputs.)
+// With one x block per matrix (M <= BNX) nothing is shared between tiles of
+// a matrix, and pair p instead takes a contiguous range of the list chosen
+// on the host so that the ranges cost about the same (a round-robin deal of
+// 76-block and 14-block tiles left a fifth of the time idle at M = 128).
+// Returns total_tiles past the pair's last tile.
+__device__ __forceinline__ int pair_tile(const GemmParams &P, int pair, int i) {
+    if (P.ranges) {
+        const int t = P.pair_begin[pair] + i;
+        return t < P.pair_begin[pair + 1] ? t : P.total_tiles;
+    }
+    return min(i * P.pairs + ((i & 1) ? P.pairs - 1 - pair : pair), P.total_tiles);
+}
+
 // Position of a tile: matrix j, 256-row weight block nb, BNX-row x block xb.
 struct TilePos {
     int j, nb, xb, kblocks;
@@ -368,8 +394,8 @@ __device__ __forceinline__ TilePos tile_pos(const GemmJobDev *jobs, int count, i
     t.j = find_job(jobs, count, tile);
     const GemmJobDev &J = jobs[t.j];
     const int local = tile - J.tile_begin;
-    t.nb = local / J.xblocks;
-    t.xb = local % J.xblocks;
+    t.nb = local % J.nblocks;
+    t.xb = local / J.nblocks;
     t.kblocks = J.K / kBK;
     return t;
 }
@@ -380,18 +406,18 @@ static_assert(kLook % 2 == 0, "two dequant groups take alternate look-ahead slot
 // Walks the (tile, 64-block) sequence a dequant thread consumes and loads
 // the scale and zero of its weight row for each position.
 template <int WF> struct SzCursor {
-    int tile, t_end, kb, kblocks, group, row0;
+    int it, tile, pair, kb, kblocks, group, row0;
     const void *srow;
     const void *zrow;
     const GemmJobDev *jobs;
     __device__ __forceinline__ void bind(const GemmParams &P, int r) {
-        if (tile >= t_end) {
+        if (tile >= P.total_tiles) {
             srow = zrow = nullptr;
             kblocks = 1;
             return;
         }
         const GemmJobDev &J = jobs[find_job(jobs, P.count, tile)];
-        const int nb = (tile - J.tile_begin) / J.xblocks;
+        const int nb = (tile - J.tile_begin) % J.nblocks;
         const int row = nb * kPairRows + row0 + r;
         kblocks = J.K / kBK;
         group = J.group;
@@ -404,11 +430,12 @@ template <int WF> struct SzCursor {
             srow = zrow = nullptr;
         }
     }
-    __device__ __forceinline__ void init(const GemmParams &P, const GemmJobDev *sj, int first,
-                                         int last, int rank_rows, int r) {
+    __device__ __forceinline__ void init(const GemmParams &P, const GemmJobDev *sj, int pr,
+                                         int rank_rows, int r) {
         jobs = sj;
-        tile = first;
-        t_end = last;
+        it = 0;
+        pair = pr;
+        tile = pair_tile(P, pair, 0);
         kb = 0;
         row0 = rank_rows;
         bind(P, r);
@@ -416,7 +443,7 @@ template <int WF> struct SzCursor {
     __device__ __forceinline__ void advance(const GemmParams &P, int r) {
         if (++kb == kblocks) {
             kb = 0;
-            ++tile;
+            tile = pair_tile(P, pair, ++it);
             bind(P, r);
         }
     }
@@ -508,7 +535,7 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)cluster_rank();           // 0: issues the MMAs
     const int pair = (int)cluster_id();
-    const int t_begin = P.pair_begin[pair], t_end = P.pair_begin[pair + 1];
+    const int t_first = pair_tile(P, pair, 0), T = P.total_tiles;
     const int rank_rows = rank * kBM;               // this CTA's weight rows in a tile
     const int rank_xrows = rank * C::kXHalf;        // this CTA's x rows in a tile
 
@@ -551,12 +578,14 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
             uint8_t *ring = codes ? w_ring : x_ring;
             const int bytes = codes ? C::kWBytes : C::kXBytes;
             uint32_t g = 0;
-            for (int tile = t_begin; tile < t_end && !*abort_flag; ++tile) {
+            for (int i = 0, tile = t_first; tile < T && !*abort_flag;
+                 tile = pair_tile(P, pair, ++i)) {
                 const TilePos tp = tile_pos(sjobs, P.count, tile);
-                if (codes && tile + 1 < t_end) {
+                const int tile2 = pair_tile(P, pair, i + 1);
+                if (codes && tile2 < T) {
                     // scales/zeros of the next tile's rows to L2 (the dequant
                     // warps read them a few stages ahead)
-                    const TilePos tn = tile_pos(sjobs, P.count, tile + 1);
+                    const TilePos tn = tile_pos(sjobs, P.count, tile2);
                     if (tn.j != tp.j || tn.nb != tp.nb) {
                         const GemmJobDev &J2 = sjobs[tn.j];
                         const int row = tn.nb * kPairRows + rank_rows;
@@ -618,8 +647,9 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
             const uint64_t bdesc0 = tc::sw128_desc(smem_u32(x_ring));
             uint32_t g = 0;
             int lt = 0;
-            for (int tile = t_begin;
-                 tile < t_end && !__shfl_sync(0xffffffffu, (int)*abort_flag, 0); ++tile, ++lt) {
+            for (int i = 0, tile = t_first;
+                 tile < T && !__shfl_sync(0xffffffffu, (int)*abort_flag, 0);
+                 tile = pair_tile(P, pair, ++i), ++lt) {
                 const int kblocks = sjobs[find_job(sjobs, P.count, tile)].K / kBK;
                 const int buf = lt & 1;
                 const uint32_t aph = (lt >> 1) & 1;
@@ -686,19 +716,19 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
         // reads it.
         const bool x_gate = rank == 1 && dw % kGroupWarps == 0;
         SzCursor<WF> la;                    // look-ahead cursor
-        la.init(P, sjobs, t_begin, t_end, rank_rows, r);
+        la.init(P, sjobs, pair, rank_rows, r);
         uint32_t sq[kLook], zq[kLook];
 #pragma unroll
         for (int i = 0; i < kLook; ++i) {
             la.load(P, sq[i], zq[i]);
             la.advance(P, r);
         }
-        int tile = t_begin, kb = 0, kblocks = 1;
+        int it = 0, tile = t_first, kb = 0, kblocks = 1;
         bool valid = false;
         auto bind = [&]() {
-            if (tile >= t_end) return;
+            if (tile >= T) return;
             const GemmJobDev &J = sjobs[find_job(sjobs, P.count, tile)];
-            const int nb = (tile - J.tile_begin) / J.xblocks;
+            const int nb = (tile - J.tile_begin) % J.nblocks;
             kblocks = J.K / kBK;
             valid = nb * kPairRows + rank_rows + r < J.N;
         };
@@ -708,10 +738,10 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
         int aoff[kCpt];
 #pragma unroll
         for (int i = 0; i < kCpt; ++i) aoff[i] = sw128_off(r, kCpt * part + i);
-        while (ok && tile < t_end && !*abort_flag) {
+        while (ok && tile < T && !*abort_flag) {
 #pragma unroll
             for (int j = 0; j < kLook; ++j) {
-                if (tile >= t_end) break;
+                if (tile >= T) break;
                 const int sw = cg % C::kWStages;
                 // Both groups wait for every weight box, the one whose blocks
                 // they skip too: a barrier's parity test is only sound for a
@@ -787,7 +817,7 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
                 ++g;
                 if (++kb == kblocks) {
                     kb = 0;
-                    ++tile;
+                    tile = pair_tile(P, pair, ++it);
                     bind();
                 }
             }
@@ -797,7 +827,8 @@ gemm_kernel(const __grid_constant__ GemmParams P) {
         // half hh of the accumulator's columns (x rows)
         const int q = warp & 3, hh = (warp - kEpWarp0) >> 2;
         int lt = 0;
-        for (int tile = t_begin; tile < t_end && !*abort_flag; ++tile, ++lt) {
+        for (int i = 0, tile = t_first; tile < T && !*abort_flag;
+             tile = pair_tile(P, pair, ++i), ++lt) {
             const TilePos tp = tile_pos(sjobs, P.count, tile);
             const GemmJobDev &J = sjobs[tp.j];
             const int buf = lt & 1;
@@ -962,25 +993,31 @@ bc_status launch_cfg(const GemmJob *jobs, int count, int64_t M, int bits, bool r
     thread_local GemmParams *Pp = nullptr;
     if (!Pp) Pp = new GemmParams();
     GemmParams &P = *Pp;
+    std::vector<int> order;
     std::vector<double> tcost;
     for (int b = 0; b < count; b += kMaxJobs) {
         const int n = std::min(kMaxJobs, count - b);
         int tiles = 0;
         const int xblocks = (int)((M + BNX - 1) / BNX);
+        // matrices by decreasing K (stable): the long-K tiles are dealt first
+        order.resize(n);
         tcost.clear();
+        for (int i = 0; i < n; ++i) order[i] = b + i;
+        std::stable_sort(order.begin(), order.end(),
+                         [&](int p, int q) { return jobs[p].K > jobs[q].K; });
         for (int i = 0; i < n; ++i) {
-            const GemmJob &J = jobs[b + i];
+            const GemmJob &J = jobs[order[i]];
             if (!encode_x(enc, &P.xmap[i], J.x, M, J.K, C::kXHalf)) return BC_ERR_CUDA;
             const bool ok = WF == kPacked ? encode_codes(enc, &P.wmap[i], J.w, J.N, J.K)
                                           : encode_w16(enc, &P.wmap[i], J.w, J.N, J.K);
             if (!ok) return BC_ERR_CUDA;
+            const int nblocks = (int)((J.N + kPairRows - 1) / kPairRows);
             P.jobs[i] = GemmJobDev{J.s, J.z, J.y, (int)J.N, (int)J.K, (int)J.group, tiles,
-                                   xblocks};
-            const int nt = (int)((J.N + kPairRows - 1) / kPairRows) * xblocks;
-            tiles += nt;
+                                   nblocks};
+            tiles += nblocks * xblocks;
             // cost in stages: K/64 of MMA plus the epilogue (BNX/32 loads of
             // 32 columns and their stores), about two stages' worth
-            tcost.insert(tcost.end(), nt, (double)(J.K / kBK) + 2.0 * BNX / 128.0);
+            tcost.insert(tcost.end(), nblocks * xblocks, (double)(J.K / kBK) + 2.0 * BNX / 128.0);
         }
         P.count = n;
         P.total_tiles = tiles;
@@ -988,7 +1025,9 @@ bc_status launch_cfg(const GemmJob *jobs, int count, int64_t M, int bits, bool r
         P.bits = bits;
         P.range = range ? 1 : 0;
         const int pairs = std::max(1, std::min(tiles, max_pairs[dev]));
-        partition_tiles(P, tcost, pairs);
+        P.pairs = pairs;
+        P.ranges = xblocks == 1 ? 1 : 0;
+        if (P.ranges) partition_tiles(P, tcost, pairs);
         cfg.gridDim = dim3(2 * pairs);
         if (cudaLaunchKernelEx(&cfg, gemm_kernel<BNX, WF>, P) != cudaSuccess) return BC_ERR_CUDA;
         bc_status st = cuda_status();
