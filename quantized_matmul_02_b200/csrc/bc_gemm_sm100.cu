@@ -30,13 +30,14 @@
 //   * an activation producer (warp 2) loads the CTA's BNX/2 rows of bf16 x
 //     (128B-swizzled, K-major) into the activation ring, which the MMA
 //     frees;
-//   * sixteen dequant warps (two groups of eight taking alternate blocks)
-//     form bf16 w' = (q - z) * s into one of six A buffers in the
-//     128B-swizzled K-major layout the MMA reads (packed:
-//     exact q - z in bf16 arithmetic and one rounding for the scale;
-//     runtime: the exact RTN code of each fp16 weight, then one rounding of
-//     (q - z) s), fence the generic-proxy writes for the tensor core and
-//     arrive on the first CTA's "A ready" barrier (cluster scope);
+//   * sixteen dequant warps form bf16 w' = (q - z) * s into one of the A
+//     buffers (six for packed codes, four for the runtime form) in the
+//     128B-swizzled K-major layout the MMA reads (packed: two groups of
+//     eight warps on alternate blocks, exact q - z in bf16 arithmetic and
+//     one rounding for the scale; runtime: one group of sixteen, the exact
+//     RTN code of each fp16 weight, then one rounding of (q - z) s), fence
+//     the generic-proxy writes for the tensor core and arrive on the first
+//     CTA's "A ready" barrier (a cluster address);
 //   * the first CTA's MMA warp waits for both CTAs' A buffers and its own
 //     activation stage (the second CTA's dequant warps wait for theirs
 //     before they arrive), issues four MMAs and commits to the "free"
@@ -46,11 +47,11 @@
 //     accumulates into the second TMEM buffer.
 // The kernel is persistent (one cluster per SM pair) and spans every matrix
 // of a grouped launch; the pairs walk one tile list side by side (see
-// pair_tile), so that the tiles in flight share their activation block.  All waits are bounded:
-// a wait that runs out records a timeout, the CTA stops, waits (bounded) for
-// its own copies and MMAs in flight, meets its partner at the cluster
-// barrier and frees its TMEM.  No load uses cluster multicast: every CTA
-// loads its own tiles.
+// pair_tile), so that the tiles in flight share their activation block.
+// All waits are bounded: a wait that runs out records a timeout, the CTA
+// stops, waits (bounded) for its own copies and MMAs in flight, meets its
+// partner at the cluster barrier and frees its TMEM.  No load uses cluster
+// multicast: every CTA loads its own tiles.
 #include "bc_internal.cuh"
 #include "bc_rtn.cuh"
 #include "bc_tc.cuh"
