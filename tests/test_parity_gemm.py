@@ -116,6 +116,12 @@ def test_prefill_qwen25_two_layers_m2048_sampled(cuda_lib):
     _prefill_set(cuda_lib, 2, 2048, sample_rows=24)
 
 
+def test_prefill_qwen25_full_set_m2048_sampled(cuda_lib):
+    """The full 24-layer set at M = 2048: 168 matrices, three launches, the
+    pairs dealing the x-block-major tile list in snake rounds."""
+    _prefill_set(cuda_lib, 24, 2048, sample_rows=8)
+
+
 # ---- runtime RTN prefill (fp16 W re-quantized inline in the dequant stage) --
 # BITCRUSH BC-06, "Under the hood" (codes computed as the weights are read,
 # at any lever position) and "The machine" (THE LEVER 16 -> 2).
