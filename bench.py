@@ -371,43 +371,68 @@ def _oracle_x(name: str, seed: int, m) -> np.ndarray:
 def cpu_baseline_sample(name: str, target_s: float = 12.0):
     """The oracle (as it stands) on a bounded sample of the workload: for
     whole matrices of the first layers, dequantize the codes and multiply
-    (the work one GPU step does), until about `target_s` seconds pass."""
+    (the work one GPU step does), until about `target_s` seconds of that
+    work have passed.  When one pass over the set takes less, the matrices
+    prepared in the first pass (up to ~1 GB of weights) are run again."""
     import oracle
     shape_set, layers, mode, bits, group, M, seed = WORKLOADS[name]
     mats = wl.layer_set(shape_set, layers)
     sigma = wl.SIGMA[shape_set]
     done_bytes, done_flops, spent = 0, 0, 0.0
     done = 0
-    for m in mats:
-        W = wl.weight(seed, m.layer, m.name, m.K, m.N, sigma)
-        x = _oracle_x(name, seed, m)
-        g = m.K if group == 0 else group
+    cache, cache_bytes = [], 0
+
+    def work(item):
+        x, W, q, s, z, g = item
+        t0 = time.perf_counter()
         if mode == "runtime" and bits == 16:
-            t0 = time.perf_counter()
             oracle.matmul(x, oracle.half_to_f64(W))
-            spent += time.perf_counter() - t0
         else:
-            s, z = oracle.group_params(W, bits, g, mode == "packed")
-            q = oracle.codes(W, s, z, bits, g)
-            t0 = time.perf_counter()
             if mode != "packed":    # runtime mode re-derives the codes per step
                 s, z = oracle.group_params(W, bits, g, False)
                 q = oracle.codes(W, s, z, bits, g)
             oracle.matmul(x, oracle.dequant(q, s, z, g))
-            spent += time.perf_counter() - t0
-        done_bytes += wl.gemv_bytes(m.K, m.N, M, mode, bits, g,
-                                    x_bytes_per_elem=2 if is_prefill(name) else 4)
-        done_flops += 2 * M * m.N * m.K
+        return time.perf_counter() - t0
+
+    for m in mats:
+        W = wl.weight(seed, m.layer, m.name, m.K, m.N, sigma)
+        x = _oracle_x(name, seed, m)
+        g = m.K if group == 0 else group
+        q = s = z = None
+        if not (mode == "runtime" and bits == 16):
+            s, z = oracle.group_params(W, bits, g, mode == "packed")
+            q = oracle.codes(W, s, z, bits, g)
+        item = (x, W, q, s, z, g)
+        spent += work(item)
+        mb = wl.gemv_bytes(m.K, m.N, M, mode, bits, g,
+                           x_bytes_per_elem=2 if is_prefill(name) else 4)
+        mf = 2 * M * m.N * m.K
+        done_bytes += mb
+        done_flops += mf
         done += 1
+        if cache_bytes < (1 << 30):
+            cache.append((item, mb, mf))
+            cache_bytes += W.nbytes + (q.nbytes if q is not None else 0)
         if spent >= target_s:
             break
+    passes = 1
+    while spent < target_s and cache:
+        for item, mb, mf in cache:
+            spent += work(item)
+            done_bytes += mb
+            done_flops += mf
+            done += 1
+            if spent >= target_s:
+                break
+        passes += 1
     if is_prefill(name):
         value, unit = done_flops / spent / 1e12, "TFLOP/s"
     else:
         value, unit = done_bytes / spent / 1e9, "GB/s"
     return {"value": value, "unit": unit,
             "cores": oracle.threads(), "kind": "oracle",
-            "sample": f"{done} of {len(mats)} matrices of {name} (first layers), "
+            "sample": f"{done} matrix products over {min(len(cache), len(mats))} of the "
+                      f"{len(mats)} matrices of {name} (first layers, {passes} passes), "
                       f"fp64 dequant + matmul, {spent:.1f} s"}
 
 
