@@ -121,3 +121,14 @@ def test_traffic_digest_covers_the_tcgen05_header(tmp_path, monkeypatch):
     assert bench.recorded_traffic("w") == 7
     (csrc / "bc_tc.cuh").write_text("changed")
     assert bench.recorded_traffic("w") is None
+
+
+def test_cpu_baseline_repeats_until_target():
+    """The CPU baseline runs the oracle on prepared matrices until its time
+    target, and says how many products over how many matrices it timed."""
+    r = bench.cpu_baseline_sample("single-1024-rtn3-decode", target_s=0.2)
+    assert r["kind"] == "oracle" and r["unit"] == "GB/s" and r["value"] > 0
+    assert r["cores"] >= 1
+    assert "over 1 of the 1 matrices" in r["sample"]
+    products = int(r["sample"].split(" matrix products")[0])
+    assert products >= 2          # one matrix, run again until the target
